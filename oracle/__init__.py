@@ -1,0 +1,176 @@
+"""Reference oracle for Loki-style low-rank-key sparse decode attention.
+
+TEST INFRASTRUCTURE. Only the tests, the smoke check and the benchmark's
+CPU-baseline leg import this package. It is a thin numpy/ctypes wrapper around
+oracle.c (plain binary64 C); every step of the arithmetic lives there, with
+its citation to the pages. It shares no code with the CUDA library.
+"""
+import ctypes
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+_lib_path = None
+
+_D = ctypes.POINTER(ctypes.c_double)
+_I32 = ctypes.POINTER(ctypes.c_int32)
+_U16 = ctypes.POINTER(ctypes.c_uint16)
+
+
+def use_library(path=None):
+    """Point the wrapper at another build of oracle.c (None: the default).
+
+    The mutation tests use this to check that the pins reject planted
+    mistakes in a modified copy of the oracle."""
+    global _lib, _lib_path
+    _lib, _lib_path = None, path
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(_lib_path or _build.build())
+        lib.oracle_round_bf16.restype = ctypes.c_double
+        lib.oracle_round_bf16.argtypes = [ctypes.c_double]
+        lib.oracle_round_bf16_array.restype = None
+        lib.oracle_round_bf16_array.argtypes = [_D, ctypes.c_int64, _D, _U16]
+        lib.oracle_rotate.restype = None
+        lib.oracle_rotate.argtypes = [_D, _D, ctypes.c_int64, ctypes.c_int, _D]
+        lib.oracle_append.restype = None
+        lib.oracle_append.argtypes = [_D, _D, ctypes.c_int64, ctypes.c_int, ctypes.c_int, _D]
+        lib.oracle_attend_set.restype = None
+        lib.oracle_attend_set.argtypes = [_D, _D, _D, _I32, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_double, _D, _D]
+        lib.oracle_decode_pair.restype = ctypes.c_int
+        lib.oracle_decode_pair.argtypes = [_D, _D, _D, _D, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                           _D, _I32, ctypes.POINTER(ctypes.c_int), _D, _D]
+        lib.oracle_dense_pair.restype = None
+        lib.oracle_dense_pair.argtypes = [_D, _D, _D, _D, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_double, _D]
+        lib.oracle_decode_batch.restype = ctypes.c_int
+        lib.oracle_decode_batch.argtypes = [ctypes.c_int, _D, _D, _D, _D, _I32, ctypes.c_int,
+                                            ctypes.c_int, ctypes.c_int, ctypes.c_int, _I32,
+                                            ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_double, _D, _I32]
+        lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_num_threads.argtypes = []
+        _lib = lib
+    return _lib
+
+
+def _f64(a):
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _p(a, t=_D):
+    return a.ctypes.data_as(t) if a is not None else None
+
+
+def round_bf16(x):
+    """Round binary64 values to bfloat16 (nearest, ties to even), one step.
+
+    Returns (values as float64, bit patterns as uint16)."""
+    x = _f64(x)
+    out = np.empty_like(x)
+    bits = np.empty(x.shape, dtype=np.uint16)
+    _load().oracle_round_bf16_array(_p(x), x.size, _p(out), _p(bits, _U16))
+    return out, bits
+
+
+def rotate(x, P):
+    """x_hat = x P for row vectors x [n, d]."""
+    x = _f64(x)
+    P = _f64(P)
+    n, d = x.shape
+    out = np.empty((n, d))
+    _load().oracle_rotate(_p(x), _p(P), n, d, _p(out))
+    return out
+
+
+def append(k_new, P, dtype):
+    """Keys rotated into the PCA basis and rounded to the cache type.
+
+    dtype: 'bf16' or 'f32'."""
+    k_new = _f64(k_new)
+    P = _f64(P)
+    n, d = k_new.shape
+    out = np.empty((n, d))
+    _load().oracle_append(_p(k_new), _p(P), n, d, 1 if dtype == "bf16" else 0, _p(out))
+    return out
+
+
+def attend_set(Kt, V, qhat, T, scale=0.0, return_weights=False):
+    """Exact softmax attention of the rows of qhat [g, d] over token set T."""
+    Kt, V, qhat = _f64(Kt), _f64(V), _f64(qhat)
+    T = np.ascontiguousarray(T, dtype=np.int32)
+    g, d = qhat.shape
+    out = np.empty((g, d))
+    w = np.empty((g, len(T))) if return_weights else None
+    _load().oracle_attend_set(_p(Kt), _p(V), _p(qhat), _p(T, _I32), len(T), d, g,
+                              scale, _p(out), _p(w))
+    return (out, w) if return_weights else out
+
+
+class PairResult:
+    __slots__ = ("out", "sel", "n_sel", "scores", "kth")
+
+
+def decode_pair(Kt, V, q, P, r, k, W=0, group_max=False, scale=0.0):
+    """One (sequence, kv head) decode step; see oracle_decode_pair in oracle.c."""
+    Kt, V, q, P = _f64(Kt), _f64(V), _f64(q), _f64(P)
+    L, d = Kt.shape
+    g = q.shape[0]
+    res = PairResult()
+    res.out = np.empty((g, d))
+    res.sel = np.empty(k + W, dtype=np.int32)
+    n_sel = ctypes.c_int(0)
+    res.scores = np.empty(L)
+    kth = ctypes.c_double(0.0)
+    rc = _load().oracle_decode_pair(_p(Kt), _p(V), _p(q), _p(P), L, d, g, r, k, W,
+                                    1 if group_max else 0, scale, _p(res.out),
+                                    _p(res.sel, _I32), ctypes.byref(n_sel), _p(res.scores),
+                                    ctypes.byref(kth))
+    if rc != 0:
+        raise ValueError("oracle_decode_pair rejected its arguments")
+    res.n_sel = n_sel.value
+    res.kth = kth.value
+    return res
+
+
+def dense_pair(K, V, q, P=None, scale=0.0):
+    """Dense decode attention; P=None uses K as given (unrotated comparison)."""
+    K, V, q = _f64(K), _f64(V), _f64(q)
+    Pp = _f64(P) if P is not None else None
+    L, d = K.shape
+    g = q.shape[0]
+    out = np.empty((g, d))
+    _load().oracle_dense_pair(_p(K), _p(V), _p(q), _p(Pp), L, d, g, scale, _p(out))
+    return out
+
+
+def decode_batch(Kt, V, q, P, L, r, k_per_pair, W=0, group_max=False, scale=0.0):
+    """Many pairs, one per OpenMP thread.
+
+    Kt, V: [n, Lmax, d]; q: [n, g, d]; P: [n, d, d]; L, k_per_pair: [n]."""
+    Kt, V, q, P = _f64(Kt), _f64(V), _f64(q), _f64(P)
+    n, Lmax, d = Kt.shape
+    g = q.shape[1]
+    L = np.ascontiguousarray(L, dtype=np.int32)
+    kp = np.ascontiguousarray(k_per_pair, dtype=np.int32)
+    kmax = int(kp.max()) if n else 0
+    out = np.empty((n, g, d))
+    sel = np.empty((n, kmax + W), dtype=np.int32)
+    rc = _load().oracle_decode_batch(n, _p(Kt), _p(V), _p(q), _p(P), _p(L, _I32), Lmax, d, g,
+                                     r, _p(kp, _I32), kmax, W, 1 if group_max else 0, scale,
+                                     _p(out), _p(sel, _I32))
+    if rc != 0:
+        raise ValueError("oracle_decode_batch rejected its arguments")
+    return out, sel
+
+
+def num_threads():
+    return _load().oracle_num_threads()

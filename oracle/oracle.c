@@ -1,0 +1,360 @@
+/*
+ * Reference oracle for Loki-style low-rank-key sparse decode attention.
+ *
+ * TEST INFRASTRUCTURE ONLY. This file is compiled into liboracle.so, which only
+ * the test suite, the smoke check and the benchmark's CPU-baseline leg load.
+ * The product library (rank_key_top_b200/csrc) never links, includes or calls
+ * it, and it shares no header, helper, table or constant with that library.
+ *
+ * Everything here is plain, slow, single-threaded-per-problem C in binary64.
+ * Each function restates one step of the method as the pages state it, in the
+ * pages' order and notation, so that a reader can check it by eye:
+ *
+ *   AQUA page ("AQUA: Attention via QUery mAgnitudes ..."), decode-step
+ *     equations (1)-(5): cache update, scores S = q K^T, scaling by
+ *     1/sqrt(d_head), softmax, context c = A V.
+ *   AQUA page, information-retention paragraph: projection is the row-vector
+ *     product v_hat = v P.
+ *   AQUA page, related work on LoKi: an offline projection transforms query and
+ *     key vectors, the trailing dimensions are sliced off (the first ones are
+ *     kept), and tokens are temporarily dropped based on the resulting
+ *     approximate scores.
+ *   Loki page ("Loki: Low-rank Keys for Efficient Sparse Attention"), abstract:
+ *     tokens are ranked and selected by attention scores computed in the
+ *     low-dimensional space.
+ *   aitopics page "low rank approximation", LRQK abstract: the top-k tokens
+ *     plus a small fixed set of recent tokens are kept and attended exactly.
+ *   AQUA page, appendix on rotation invariance: q_hat K_hat^T = q K^T for an
+ *     orthogonal P (used by the tests, not here).
+ *
+ * Readings taken where the pages are silent (each is listed in the design
+ * notes of the repository):
+ *   - group reduction for grouped-query attention: the approximate score of a
+ *     token for a kv head is the SUM over the group's query heads (option MAX);
+ *   - ties in the approximate score go to the lower token index;
+ *   - the recent window W is forced, top-k is taken among the other tokens;
+ *   - the exact logits use the full head dimension and 1/sqrt(d) by default;
+ *   - softmax is renormalised over the kept set only.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------------- */
+/* Rounding of an exact binary64 value to the cache storage types.           */
+/* ------------------------------------------------------------------------- */
+
+/* Round-to-nearest-even of a binary64 value to bfloat16 (1 sign bit, 8
+ * exponent bits, 7 stored mantissa bits; 8 significant bits), done in one step
+ * from binary64 so that no double rounding through binary32 can occur.
+ * Returned as the binary64 value of the rounded bfloat16. */
+double oracle_round_bf16(double v)
+{
+    if (v == 0.0 || isnan(v) || isinf(v))
+        return v;
+    int e;
+    frexp(v, &e);                 /* v = m * 2^e with 0.5 <= |m| < 1 */
+    int spacing_exp = e - 8;      /* 8 significant bits in this binade */
+    if (spacing_exp < -133)       /* subnormal bfloat16 spacing is 2^-133 */
+        spacing_exp = -133;
+    double steps = nearbyint(ldexp(v, -spacing_exp)); /* ties to even */
+    double r = ldexp(steps, spacing_exp);
+    const double bf16_max = ldexp(255.0, 120);         /* (2 - 2^-7) * 2^127 */
+    if (fabs(r) > bf16_max)
+        r = copysign(INFINITY, v);
+    return r;
+}
+
+/* bfloat16 bit pattern of a value that oracle_round_bf16 returned. */
+uint16_t oracle_bf16_bits(double rounded)
+{
+    float f = (float)rounded;     /* exact: every bfloat16 is a binary32 */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(u >> 16);
+}
+
+void oracle_round_bf16_array(const double* x, int64_t n, double* out, uint16_t* bits)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        out[i] = oracle_round_bf16(x[i]);
+        if (bits)
+            bits[i] = oracle_bf16_bits(out[i]);
+    }
+}
+
+/* ------------------------------------------------------------------------- */
+/* Projection into the PCA basis: row vectors, v_hat = v P.                  */
+/* AQUA page, information-retention paragraph and appendix step 1            */
+/* ("projecting the current query and key with P").                          */
+/* ------------------------------------------------------------------------- */
+void oracle_rotate(const double* x, const double* P, int64_t n, int d, double* out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        for (int c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (int a = 0; a < d; ++a)
+                acc += x[i * d + a] * P[(int64_t)a * d + c];
+            out[i * d + c] = acc;
+        }
+}
+
+/* Cache update of a decode step (AQUA page, equations (1)-(2)) for keys kept
+ * in the PCA basis: k_tilde = round(k P) to the cache type. dtype 1 = bf16,
+ * dtype 0 = binary32. */
+void oracle_append(const double* k_new, const double* P, int64_t n, int d, int dtype,
+                   double* out)
+{
+    oracle_rotate(k_new, P, n, d, out);
+    for (int64_t i = 0; i < n * d; ++i)
+        out[i] = dtype == 1 ? oracle_round_bf16(out[i]) : (double)(float)out[i];
+}
+
+/* ------------------------------------------------------------------------- */
+/* Exact attention over a given token set T, for the g query heads of one    */
+/* kv head. AQUA page, equations (3)-(5): z = q_hat k_tilde^T * scale over    */
+/* the full head dimension, A = softmax(z) over T, c = A V.                   */
+/* qhat: [g][d] (already in the PCA basis). Kt, V: [L][d]. out: [g][d].       */
+/* scale 0 means 1/sqrt(d).                                                   */
+/* weights (nullable): [g][nT], the softmax weights in the order of T.        */
+/* ------------------------------------------------------------------------- */
+void oracle_attend_set(const double* Kt, const double* V, const double* qhat,
+                       const int32_t* T, int nT, int d, int g, double scale,
+                       double* out, double* weights)
+{
+    if (scale == 0.0)
+        scale = 1.0 / sqrt((double)d);
+    double* z = (double*)malloc(sizeof(double) * (size_t)(nT > 0 ? nT : 1));
+    for (int j = 0; j < g; ++j) {
+        for (int c = 0; c < d; ++c)
+            out[j * d + c] = 0.0;
+        if (nT == 0)
+            continue;
+        /* equation (3), scaled as in equation (4) */
+        double zmax = -INFINITY;
+        for (int i = 0; i < nT; ++i) {
+            const double* k = Kt + (int64_t)T[i] * d;
+            double s = 0.0;
+            for (int c = 0; c < d; ++c)
+                s += qhat[j * d + c] * k[c];
+            z[i] = s * scale;
+            if (z[i] > zmax)
+                zmax = z[i];
+        }
+        /* softmax of equation (4), shifted by the maximum for range only */
+        double denom = 0.0;
+        for (int i = 0; i < nT; ++i) {
+            z[i] = exp(z[i] - zmax);
+            denom += z[i];
+        }
+        /* context vector, equation (5) */
+        for (int i = 0; i < nT; ++i) {
+            double a = z[i] / denom;
+            if (weights)
+                weights[(int64_t)j * nT + i] = a;
+            const double* v = V + (int64_t)T[i] * d;
+            for (int c = 0; c < d; ++c)
+                out[j * d + c] += a * v[c];
+        }
+    }
+    free(z);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Top-k with ties to the lower index: sort candidates by (score descending, */
+/* index ascending) and keep the first k.                                    */
+/* ------------------------------------------------------------------------- */
+typedef struct {
+    double s;
+    int32_t t;
+} scored_token;
+
+static int by_score_then_index(const void* pa, const void* pb)
+{
+    const scored_token* a = (const scored_token*)pa;
+    const scored_token* b = (const scored_token*)pb;
+    if (a->s > b->s) return -1;
+    if (a->s < b->s) return 1;
+    return (a->t > b->t) - (a->t < b->t);
+}
+
+static int by_index(const void* pa, const void* pb)
+{
+    int32_t a = *(const int32_t*)pa, b = *(const int32_t*)pb;
+    return (a > b) - (a < b);
+}
+
+/* ------------------------------------------------------------------------- */
+/* One decode step of Loki-style sparse attention for one (sequence, kv      */
+/* head) pair and its g query heads.                                         */
+/*                                                                           */
+/* Kt  [L][d]  keys as stored in the cache, already in the PCA basis          */
+/* V   [L][d]  values as stored                                               */
+/* q   [g][d]  unrotated queries of the group                                 */
+/* P   [d][d]  projection, row-major; the PCA basis is v_hat = v P            */
+/* r           number of leading rotated dimensions used for scoring          */
+/* k           tokens kept by score; W recent tokens always kept              */
+/* group_max   0: group score = sum over heads; 1: maximum over heads         */
+/* scale       exact-logit scale; 0 means 1/sqrt(d)                           */
+/* out [g][d]  attention output                                               */
+/* sel [k+W]   kept token indices, ascending, -1 padded (nullable)            */
+/* n_sel       number of kept tokens (nullable)                               */
+/* scores [L]  approximate scores of the candidates, NaN elsewhere (nullable) */
+/* kth         score of the last token kept by score, NaN if none (nullable)  */
+/* Returns 0, or -1 when k = 0 and W = 0 (nothing could ever be kept).        */
+/* ------------------------------------------------------------------------- */
+int oracle_decode_pair(const double* Kt, const double* V, const double* q, const double* P,
+                       int L, int d, int g, int r, int k, int W, int group_max, double scale,
+                       double* out, int32_t* sel, int* n_sel, double* scores, double* kth)
+{
+    if (k < 0 || W < 0 || (k == 0 && W == 0) || r < 1 || r > d || L < 0)
+        return -1;
+    if (scale == 0.0)
+        scale = 1.0 / sqrt((double)d);
+
+    /* Step 1: rotate the queries into the PCA basis (AQUA appendix, step 1). */
+    double* qhat = (double*)malloc(sizeof(double) * (size_t)g * d);
+    oracle_rotate(q, P, g, d, qhat);
+
+    /* Step 2: candidates are the tokens outside the forced recent window.    */
+    int w_eff = W < L ? W : L;
+    int ncand = L - w_eff;
+
+    /* Step 3: approximate scores from the leading r rotated dimensions only  */
+    /* (LoKi as described on the AQUA page: slice the trailing dimensions;    */
+    /* Loki abstract: scores computed in the low-dimensional space).          */
+    scored_token* cand = (scored_token*)malloc(sizeof(scored_token) * (size_t)(ncand > 0 ? ncand : 1));
+    for (int t = 0; t < ncand; ++t) {
+        const double* kt = Kt + (int64_t)t * d;
+        double s = group_max ? -INFINITY : 0.0;
+        for (int j = 0; j < g; ++j) {
+            double sj = 0.0;
+            for (int c = 0; c < r; ++c)
+                sj += qhat[j * d + c] * kt[c];
+            if (group_max)
+                s = sj > s ? sj : s;
+            else
+                s += sj;
+        }
+        cand[t].s = s;
+        cand[t].t = t;
+    }
+    if (scores) {
+        for (int t = 0; t < L; ++t)
+            scores[t] = NAN;
+        for (int t = 0; t < ncand; ++t)
+            scores[t] = cand[t].s;
+    }
+
+    /* Step 4: keep the k best candidates, ties to the lower index, and add   */
+    /* the recent window (LRQK: top-k tokens plus a fixed set of recent ones). */
+    int keff = k < ncand ? k : ncand;
+    qsort(cand, (size_t)ncand, sizeof(scored_token), by_score_then_index);
+    if (kth)
+        *kth = keff > 0 ? cand[keff - 1].s : NAN;
+    int nT = keff + w_eff;
+    int32_t* T = (int32_t*)malloc(sizeof(int32_t) * (size_t)(nT > 0 ? nT : 1));
+    for (int i = 0; i < keff; ++i)
+        T[i] = cand[i].t;
+    qsort(T, (size_t)keff, sizeof(int32_t), by_index);
+    for (int i = 0; i < w_eff; ++i)
+        T[keff + i] = ncand + i;
+
+    /* Step 5: exact softmax attention over the kept set (equations (3)-(5)). */
+    oracle_attend_set(Kt, V, qhat, T, nT, d, g, scale, out, NULL);
+
+    if (sel) {
+        for (int i = 0; i < k + W; ++i)
+            sel[i] = i < nT ? T[i] : -1;
+    }
+    if (n_sel)
+        *n_sel = nT;
+    free(T);
+    free(cand);
+    free(qhat);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Dense decode attention for one (sequence, kv head) pair: equations (3)-(5) */
+/* over every token, written independently of the sparse path. With P = NULL */
+/* the keys are used as given (the unrotated comparison); otherwise the       */
+/* queries are rotated by P first and K holds keys in the PCA basis.         */
+/* ------------------------------------------------------------------------- */
+void oracle_dense_pair(const double* K, const double* V, const double* q, const double* P,
+                       int L, int d, int g, double scale, double* out)
+{
+    if (scale == 0.0)
+        scale = 1.0 / sqrt((double)d);
+    double* qq = (double*)malloc(sizeof(double) * (size_t)g * d);
+    if (P)
+        oracle_rotate(q, P, g, d, qq);
+    else
+        memcpy(qq, q, sizeof(double) * (size_t)g * d);
+    double* z = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+    for (int j = 0; j < g; ++j) {
+        double zmax = -INFINITY;
+        for (int t = 0; t < L; ++t) {
+            double s = 0.0;
+            for (int c = 0; c < d; ++c)
+                s += qq[j * d + c] * K[(int64_t)t * d + c];
+            z[t] = s * scale;
+            zmax = z[t] > zmax ? z[t] : zmax;
+        }
+        double denom = 0.0;
+        for (int t = 0; t < L; ++t) {
+            z[t] = exp(z[t] - zmax);
+            denom += z[t];
+        }
+        for (int c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (int t = 0; t < L; ++t)
+                acc += z[t] / denom * V[(int64_t)t * d + c];
+            out[j * d + c] = L > 0 ? acc : 0.0;
+        }
+    }
+    free(z);
+    free(qq);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Many independent pairs at once (the same computation as above, one pair   */
+/* per OpenMP thread). Pair p reads Kt/V at p*Lmax*d, q at p*g*d, P at p*d*d */
+/* and writes out at p*g*d, sel at p*(kmax+W).                                */
+/* ------------------------------------------------------------------------- */
+int oracle_decode_batch(int n_pairs, const double* Kt, const double* V, const double* q,
+                        const double* P, const int32_t* L, int Lmax, int d, int g, int r,
+                        const int32_t* k_per_pair, int kmax, int W, int group_max,
+                        double scale, double* out, int32_t* sel)
+{
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int p = 0; p < n_pairs; ++p) {
+        int32_t* s = (int32_t*)malloc(sizeof(int32_t) * (size_t)(k_per_pair[p] + W));
+        int rc = oracle_decode_pair(Kt + (int64_t)p * Lmax * d, V + (int64_t)p * Lmax * d,
+                                    q + (int64_t)p * g * d, P + (int64_t)p * d * d, L[p], d, g,
+                                    r, k_per_pair[p], W, group_max, scale,
+                                    out + (int64_t)p * g * d, s, NULL, NULL, NULL);
+        if (rc != 0)
+            bad = 1;
+        if (sel)
+            for (int i = 0; i < kmax + W; ++i)
+                sel[(int64_t)p * (kmax + W) + i] = i < k_per_pair[p] + W ? s[i] : -1;
+        free(s);
+    }
+    return bad ? -1 : 0;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

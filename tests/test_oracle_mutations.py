@@ -1,0 +1,81 @@
+"""The pins must reject plausible mistakes in the oracle.
+
+Each case copies oracle.c, plants one mistake (a transposed operand, the wrong
+slice, a reversed tie rule, a dropped term ...), builds the copy on the CPU and
+runs the pins against it: at least one pin must fail. The real oracle is left
+untouched."""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from oracle import build as oracle_build
+from tests import test_oracle_pins as pins
+
+MUTATIONS = {
+    "rotation transposed": ("acc += x[i * d + a] * P[(int64_t)a * d + c];",
+                            "acc += x[i * d + a] * P[(int64_t)c * d + a];"),
+    "trailing dims scored": ("for (int c = 0; c < r; ++c)\n                sj +=",
+                             "for (int c = d - r; c < d; ++c)\n                sj +="),
+    "ties to the higher index": ("return (a->t > b->t) - (a->t < b->t);",
+                                 "return (a->t < b->t) - (a->t > b->t);"),
+    "scale dropped": ("z[i] = s * scale;", "z[i] = s;"),
+    "softmax sign": ("z[i] = exp(z[i] - zmax);", "z[i] = exp(zmax - z[i]);"),
+    "recent window shifted": ("T[keff + i] = ncand + i;", "T[keff + i] = ncand + i - 1;"),
+    "group: last head only": ("                s += sj;", "                s = sj;"),
+    "bf16 truncates": ("nearbyint(ldexp(v, -spacing_exp))", "trunc(ldexp(v, -spacing_exp))"),
+    "dense unnormalised": ("acc += z[t] / denom * V[(int64_t)t * d + c];",
+                           "acc += z[t] * V[(int64_t)t * d + c];"),
+    "window not excluded": ("int ncand = L - w_eff;", "int ncand = L - w_eff + (w_eff > 0);"),
+    "k off by one": ("int keff = k < ncand ? k : ncand;", "int keff = k < ncand ? k - (k > 1) : ncand;"),
+}
+
+PIN_FUNCS = [
+    pins.test_round_bf16_matches_torch_on_binary32_values,
+    pins.test_round_bf16_hand_cases,
+    pins.test_append_with_identity_and_signed_permutation,
+    pins.test_rotation_invariance_of_full_rank_scores,
+    pins.test_rotation_transposed_would_fail,
+    pins.test_dense_is_rotation_invariant,
+    pins.test_dense_matches_textbook_softmax,
+    pins.test_leading_dims_are_the_first_r_columns,
+    pins.test_group_sum_and_max_readings,
+    pins.test_k1_returns_the_argmax_row_exactly,
+    pins.test_equal_scores_keep_the_lowest_indices,
+    pins.test_zero_keys_average_the_kept_values,
+    pins.test_one_hot_values_expose_the_softmax_weights,
+    pins.test_recent_window_only,
+    pins.test_head_permutation_within_group,
+] + [lambda t=t: pins.test_topk_brute_force(t) for t in range(20)] + [
+    lambda n=n: pins.test_golden_fixture(n)
+    for n in sorted(x for x in os.listdir(pins.GOLDEN) if x.endswith(".json"))
+]
+
+
+def build_mutant(tmp_path, old, new):
+    src = open(oracle_build.SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not unique or missing: {old!r}"
+    path = tmp_path / "oracle_mutant.c"
+    path.write_text(src.replace(old, new))
+    lib = tmp_path / "liboracle_mutant.so"
+    subprocess.run(["gcc", "-std=c11", "-O2", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off",
+                    str(path), "-o", str(lib), "-lm"], check=True)
+    return str(lib)
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_reject_mutant(name, tmp_path):
+    old, new = MUTATIONS[name]
+    lib = build_mutant(tmp_path, old, new)
+    failures = 0
+    oracle.use_library(lib)
+    try:
+        for fn in PIN_FUNCS:
+            try:
+                fn()
+            except (AssertionError, ValueError):
+                failures += 1
+    finally:
+        oracle.use_library(None)
+    assert failures > 0, f"no pin caught the planted mistake: {name}"

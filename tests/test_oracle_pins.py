@@ -1,0 +1,458 @@
+"""Pins of the reference oracle to facts fixed outside the oracle itself.
+
+Each test checks the oracle against mathematics the pages state or imply, a
+library routine, a closed form, brute force on tiny inputs, or a hand-derived
+fixture, so that a plausible mistake in the oracle (a dropped term, a wrong
+sign or index, a transposed operand, the wrong slice, the wrong tie rule)
+fails at least one of them. No GPU is used.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def orthonormal(d, seed):
+    rng = np.random.default_rng(seed)
+    qm, rm = np.linalg.qr(rng.standard_normal((d, d)))
+    return qm * np.sign(np.diag(rm))
+
+
+def signed_permutation(d, seed):
+    rng = np.random.default_rng(seed)
+    P = np.zeros((d, d))
+    P[np.arange(d), rng.permutation(d)] = rng.choice([-1.0, 1.0], size=d)
+    return P
+
+
+# --------------------------------------------------------------------------
+# bfloat16 rounding (storage of rotated keys in the cache)
+# --------------------------------------------------------------------------
+
+def test_round_bf16_matches_torch_on_binary32_values():
+    rng = np.random.default_rng(0)
+    mags = 2.0 ** rng.uniform(-140, 127, size=200_000)
+    x = (mags * rng.choice([-1, 1], size=mags.size)).astype(np.float32)
+    # include exact ties and neighbours of ties
+    base = rng.integers(-2 ** 15, 2 ** 15, size=20_000).astype(np.int64) << 16
+    ties = np.concatenate([base | 0x8000, base | 0x7FFF, base | 0x8001]).astype(np.uint32)
+    xt = ties.view(np.float32)
+    xt = xt[np.isfinite(xt)]
+    x = np.concatenate([x, xt, np.float32([0.0, -0.0, 1e-45, -1e-45, 3.3e38])])
+    _, bits = oracle.round_bf16(x.astype(np.float64))
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(bits, ref)
+
+
+def test_round_bf16_hand_cases():
+    cases = [
+        (1.0 + 2.0 ** -8, 1.0),                              # tie -> even (mantissa 0)
+        (1.0 + 3 * 2.0 ** -8, 1.0 + 2.0 ** -6),              # tie -> even (mantissa 2)
+        (1.0 + 2.0 ** -8 + 2.0 ** -30, 1.0 + 2.0 ** -7),     # above the tie: up; through
+                                                             # binary32 it would tie to 1.0
+        (-(1.0 + 2.0 ** -8 + 2.0 ** -30), -(1.0 + 2.0 ** -7)),
+        (255 * 2.0 ** 120, 255 * 2.0 ** 120),                # largest finite bf16
+        (255 * 2.0 ** 120 + 0.4 * 2.0 ** 120, 255 * 2.0 ** 120),
+        (255 * 2.0 ** 120 + 2.0 ** 119, math.inf),           # tie at the top -> even = 2^128
+        (2.0 ** -133, 2.0 ** -133),                          # smallest subnormal
+        (0.75 * 2.0 ** -133, 2.0 ** -133),
+        (0.5 * 2.0 ** -133, 0.0),                            # tie -> even (0)
+    ]
+    x = np.array([c[0] for c in cases])
+    vals, _ = oracle.round_bf16(x)
+    for (xi, want), got in zip(cases, vals):
+        assert got == want, (xi, want, got)
+
+
+def test_append_with_identity_and_signed_permutation():
+    rng = np.random.default_rng(1)
+    k = rng.standard_normal((7, 16))
+    rounded, _ = oracle.round_bf16(k)
+    np.testing.assert_array_equal(oracle.append(k, np.eye(16), "bf16"), rounded)
+    P = signed_permutation(16, 2)
+    # k P permutes and negates columns exactly, so rounding commutes with it
+    np.testing.assert_array_equal(oracle.append(k, P, "bf16"), rounded @ P)
+    np.testing.assert_array_equal(oracle.append(k, P, "f32"),
+                                  (k.astype(np.float32).astype(np.float64)) @ P)
+
+
+# --------------------------------------------------------------------------
+# Rotation invariance (AQUA page, appendix proof: q_hat K_hat^T = q K^T)
+# --------------------------------------------------------------------------
+
+def test_rotation_invariance_of_full_rank_scores():
+    rng = np.random.default_rng(3)
+    d, L, g = 32, 50, 3
+    P = orthonormal(d, 4)
+    K = rng.standard_normal((L, d))
+    q = rng.standard_normal((g, d))
+    V = rng.standard_normal((L, d))
+    res = oracle.decode_pair(K @ P, V, q, P, r=d, k=L, W=0)
+    want = (q @ K.T).sum(axis=0)           # SUM over the group, unrotated keys
+    np.testing.assert_allclose(res.scores, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
+    xr = oracle.rotate(q, P)
+    kr = oracle.rotate(K, P)
+    np.testing.assert_allclose(xr @ kr.T, q @ K.T, rtol=0, atol=1e-12 * np.abs(q @ K.T).max())
+
+
+def test_rotation_transposed_would_fail():
+    """The invariance distinguishes v P from v P^T (a transposed operand)."""
+    rng = np.random.default_rng(5)
+    d = 16
+    P = orthonormal(d, 6)
+    x = rng.standard_normal((4, d))
+    np.testing.assert_allclose(oracle.rotate(x, P), x @ P, rtol=1e-13, atol=1e-13)
+    assert np.abs(oracle.rotate(x, P) - x @ P.T).max() > 1e-3
+
+
+def test_dense_is_rotation_invariant():
+    rng = np.random.default_rng(7)
+    d, L, g = 24, 40, 2
+    P = orthonormal(d, 8)
+    K = rng.standard_normal((L, d))
+    V = rng.standard_normal((L, d))
+    q = rng.standard_normal((g, d))
+    a = oracle.dense_pair(K @ P, V, q, P)
+    b = oracle.dense_pair(K, V, q, None)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Reduction to dense attention: r = d and k = L (and W = 0)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("g", [1, 4])
+def test_full_rank_full_k_equals_dense(g):
+    rng = np.random.default_rng(9 + g)
+    d, L = 32, 77
+    P = orthonormal(d, 10)
+    K = rng.standard_normal((L, d))
+    V = rng.standard_normal((L, d))
+    q = rng.standard_normal((g, d))
+    res = oracle.decode_pair(K @ P, V, q, P, r=d, k=L, W=0)
+    np.testing.assert_allclose(res.out, oracle.dense_pair(K, V, q, None), rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(res.sel[:L], np.arange(L))
+
+
+def test_dense_matches_textbook_softmax():
+    rng = np.random.default_rng(11)
+    d, L, g = 64, 300, 4
+    K = rng.standard_normal((L, d)) * 2
+    V = rng.standard_normal((L, d))
+    q = rng.standard_normal((g, d))
+    want = scipy.special.softmax(q @ K.T / math.sqrt(d), axis=1) @ V
+    np.testing.assert_allclose(oracle.dense_pair(K, V, q, None), want, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(oracle.dense_pair(K, V, q, None, scale=0.3),
+                               scipy.special.softmax(0.3 * q @ K.T, axis=1) @ V, rtol=0, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# Top-k selection: brute force on tiny inputs with integer scores and ties
+# --------------------------------------------------------------------------
+
+def brute_force_topk(scores, k):
+    """Among all k-subsets with the largest score sum, the lexicographically
+    smallest sorted index tuple (= ties to the lower index)."""
+    n = len(scores)
+    best, best_sum = None, None
+    for sub in itertools.combinations(range(n), k):
+        s = sum(scores[i] for i in sub)
+        if best_sum is None or s > best_sum or (s == best_sum and sub < best):
+            best, best_sum = sub, s
+    return list(best) if best is not None else []
+
+
+@pytest.mark.parametrize("trial", range(60))
+def test_topk_brute_force(trial):
+    rng = np.random.default_rng(100 + trial)
+    d = 8
+    L = int(rng.integers(1, 13))
+    k = int(rng.integers(0, 6))
+    W = int(rng.integers(0, 4))
+    if k == 0 and W == 0:
+        k = 1
+    g = int(rng.integers(1, 3))
+    r = int(rng.choice([1, 2, 4, 8]))
+    P = signed_permutation(d, 200 + trial)          # exact in binary64
+    Kt = rng.integers(-2, 3, size=(L, d)).astype(float)
+    V = rng.standard_normal((L, d))
+    q = rng.integers(-2, 3, size=(g, d)).astype(float)
+    res = oracle.decode_pair(Kt, V, q, P, r=r, k=k, W=W)
+    w_eff = min(W, L)
+    ncand = L - w_eff
+    # scores of the candidates are integers; ties are frequent
+    s = res.scores[:ncand]
+    assert np.all(s == np.round(s))
+    keff = min(k, ncand)
+    want = brute_force_topk(list(s), keff) + list(range(ncand, L))
+    assert res.n_sel == keff + w_eff
+    np.testing.assert_array_equal(res.sel[:res.n_sel], want)
+    assert np.all(res.sel[res.n_sel:] == -1)
+
+
+def test_leading_dims_are_the_first_r_columns():
+    """Slicing keeps the FIRST r rotated dimensions (AQUA page, related work on
+    LoKi): keys living only in the trailing columns score zero."""
+    rng = np.random.default_rng(12)
+    d, L, r, k = 16, 30, 4, 5
+    Kt = np.zeros((L, d))
+    Kt[:, r:] = rng.standard_normal((L, d - r))
+    V = rng.standard_normal((L, d))
+    q = rng.standard_normal((1, d))
+    res = oracle.decode_pair(Kt, V, q, np.eye(d), r=r, k=k)
+    assert np.all(res.scores == 0.0)
+    np.testing.assert_array_equal(res.sel[:k], np.arange(k))
+    # keys living only in the leading columns score as with r = d
+    Kt2 = np.zeros((L, d))
+    Kt2[:, :r] = rng.standard_normal((L, r))
+    full = oracle.decode_pair(Kt2, V, q, np.eye(d), r=d, k=k)
+    part = oracle.decode_pair(Kt2, V, q, np.eye(d), r=r, k=k)
+    np.testing.assert_array_equal(part.scores, full.scores)
+
+
+def test_group_sum_and_max_readings():
+    """SUM of the group equals scoring with the summed query (linearity); MAX
+    equals the largest of the single-head scores."""
+    rng = np.random.default_rng(13)
+    d, L, g, r = 16, 40, 4, 6
+    P = orthonormal(d, 14)
+    Kt = rng.standard_normal((L, d))
+    V = rng.standard_normal((L, d))
+    q = rng.standard_normal((g, d))
+    summed = oracle.decode_pair(Kt, V, q, P, r=r, k=7)
+    single = oracle.decode_pair(Kt, V, q.sum(axis=0, keepdims=True), P, r=r, k=7)
+    np.testing.assert_allclose(summed.scores, single.scores, rtol=1e-12, atol=1e-12)
+    np.testing.assert_array_equal(summed.sel, single.sel)
+    per_head = np.stack([oracle.decode_pair(Kt, V, q[j:j + 1], P, r=r, k=7).scores
+                         for j in range(g)])
+    mx = oracle.decode_pair(Kt, V, q, P, r=r, k=7, group_max=True)
+    np.testing.assert_array_equal(mx.scores, per_head.max(axis=0))
+
+
+# --------------------------------------------------------------------------
+# Closed forms and special cases
+# --------------------------------------------------------------------------
+
+def test_k1_returns_the_argmax_row_exactly():
+    rng = np.random.default_rng(15)
+    d, L, g = 16, 64, 2
+    P = orthonormal(d, 16)
+    Kt = rng.standard_normal((L, d))
+    V = rng.standard_normal((L, d))
+    q = rng.standard_normal((g, d))
+    res = oracle.decode_pair(Kt, V, q, P, r=4, k=1)
+    t = int(np.argmax(res.scores))
+    assert res.n_sel == 1 and res.sel[0] == t
+    for j in range(g):
+        np.testing.assert_array_equal(res.out[j], V[t])
+
+
+def test_equal_scores_keep_the_lowest_indices():
+    rng = np.random.default_rng(17)
+    d, L, r, k, W = 16, 50, 8, 9, 3
+    Kt = rng.standard_normal((L, d))
+    Kt[:, :r] = 1.5                       # every candidate has the same score
+    V = rng.standard_normal((L, d))
+    q = rng.standard_normal((2, d))
+    res = oracle.decode_pair(Kt, V, q, np.eye(d), r=r, k=k, W=W)
+    np.testing.assert_array_equal(res.sel[:res.n_sel],
+                                  list(range(k)) + list(range(L - W, L)))
+
+
+def test_constant_values_give_the_constant():
+    rng = np.random.default_rng(18)
+    d, L = 16, 40
+    Kt = rng.standard_normal((L, d)) * 3
+    V = np.tile(rng.standard_normal(d), (L, 1))
+    q = rng.standard_normal((3, d))
+    res = oracle.decode_pair(Kt, V, q, orthonormal(d, 19), r=4, k=11, W=2)
+    np.testing.assert_allclose(res.out, np.tile(V[0], (3, 1)), rtol=1e-15, atol=1e-15)
+
+
+def test_zero_keys_average_the_kept_values():
+    rng = np.random.default_rng(20)
+    d, L, k, W = 16, 40, 6, 4
+    Kt = np.zeros((L, d))
+    V = rng.standard_normal((L, d))
+    q = rng.standard_normal((2, d))
+    res = oracle.decode_pair(Kt, V, q, orthonormal(d, 21), r=4, k=k, W=W)
+    T = list(range(k)) + list(range(L - W, L))
+    np.testing.assert_allclose(res.out, np.tile(V[T].mean(axis=0), (2, 1)), rtol=0, atol=1e-14)
+
+
+def test_single_head_sum_equals_max():
+    rng = np.random.default_rng(22)
+    d, L = 16, 80
+    Kt, V = rng.standard_normal((L, d)), rng.standard_normal((L, d))
+    q = rng.standard_normal((1, d))
+    P = orthonormal(d, 23)
+    a = oracle.decode_pair(Kt, V, q, P, r=4, k=10, W=3)
+    b = oracle.decode_pair(Kt, V, q, P, r=4, k=10, W=3, group_max=True)
+    np.testing.assert_array_equal(a.sel, b.sel)
+    np.testing.assert_array_equal(a.out, b.out)
+
+
+@pytest.mark.parametrize("k,W", [(5, 40), (30, 20), (0, 60), (50, 0), (100, 100)])
+def test_everything_kept_equals_dense(k, W):
+    rng = np.random.default_rng(24)
+    d, L = 16, 50
+    P = orthonormal(d, 25)
+    K = rng.standard_normal((L, d))
+    V = rng.standard_normal((L, d))
+    q = rng.standard_normal((2, d))
+    if k + min(W, L) < L:
+        pytest.skip("not everything kept")
+    res = oracle.decode_pair(K @ P, V, q, P, r=3, k=k, W=W)
+    np.testing.assert_allclose(res.out, oracle.dense_pair(K, V, q, None), rtol=0, atol=1e-12)
+
+
+def test_recent_window_only():
+    rng = np.random.default_rng(26)
+    d, L, W = 8, 20, 5
+    Kt, V = rng.standard_normal((L, d)), rng.standard_normal((L, d))
+    q = rng.standard_normal((1, d))
+    res = oracle.decode_pair(Kt, V, q, np.eye(d), r=2, k=0, W=W)
+    np.testing.assert_array_equal(res.sel[:res.n_sel], np.arange(L - W, L))
+    np.testing.assert_allclose(res.out, oracle.dense_pair(Kt[L - W:], V[L - W:], q, None),
+                               rtol=0, atol=1e-14)
+
+
+def test_empty_sequence_and_rejected_arguments():
+    d = 8
+    res = oracle.decode_pair(np.zeros((0, d)), np.zeros((0, d)), np.ones((1, d)), np.eye(d),
+                             r=2, k=3, W=1)
+    assert res.n_sel == 0 and np.all(res.out == 0) and np.all(res.sel == -1)
+    with pytest.raises(ValueError):
+        oracle.decode_pair(np.zeros((4, d)), np.zeros((4, d)), np.ones((1, d)), np.eye(d),
+                           r=2, k=0, W=0)
+    with pytest.raises(ValueError):
+        oracle.decode_pair(np.zeros((4, d)), np.zeros((4, d)), np.ones((1, d)), np.eye(d),
+                           r=d + 1, k=1, W=0)
+
+
+# --------------------------------------------------------------------------
+# Invariants
+# --------------------------------------------------------------------------
+
+def test_one_hot_values_expose_the_softmax_weights():
+    rng = np.random.default_rng(27)
+    d, L, k, W = 32, 24, 7, 3
+    Kt = rng.standard_normal((L, d))
+    V = np.eye(L, d)                     # out_j[t] = weight of token t
+    q = rng.standard_normal((2, d))
+    res = oracle.decode_pair(Kt, V, q, orthonormal(d, 28), r=5, k=k, W=W)
+    T = res.sel[:res.n_sel]
+    for j in range(2):
+        w = res.out[j, :L]
+        assert abs(w.sum() - 1.0) < 1e-14
+        assert np.all(w[T] > 0)
+        off = np.setdiff1d(np.arange(L), T)
+        assert np.all(w[off] == 0)
+
+
+def test_output_within_the_kept_value_range():
+    rng = np.random.default_rng(29)
+    d, L = 16, 200
+    Kt, V = rng.standard_normal((L, d)) * 4, rng.standard_normal((L, d))
+    q = rng.standard_normal((4, d))
+    res = oracle.decode_pair(Kt, V, q, orthonormal(d, 30), r=4, k=20, W=5)
+    T = res.sel[:res.n_sel]
+    lo, hi = V[T].min(axis=0), V[T].max(axis=0)
+    assert np.all(res.out >= lo - 1e-15) and np.all(res.out <= hi + 1e-15)
+
+
+def test_head_permutation_within_group():
+    rng = np.random.default_rng(31)
+    d, L, g = 16, 90, 4
+    Kt, V = rng.standard_normal((L, d)), rng.standard_normal((L, d))
+    q = rng.standard_normal((g, d))
+    P = orthonormal(d, 32)
+    perm = np.array([2, 0, 3, 1])
+    a = oracle.decode_pair(Kt, V, q, P, r=4, k=12, W=2)
+    b = oracle.decode_pair(Kt, V, q[perm], P, r=4, k=12, W=2)
+    np.testing.assert_array_equal(a.sel, b.sel)
+    np.testing.assert_allclose(b.out, a.out[perm], rtol=0, atol=1e-14)
+
+
+def test_token_permutation_moves_the_selection():
+    rng = np.random.default_rng(33)
+    d, L, W = 16, 60, 4
+    Kt, V = rng.standard_normal((L, d)), rng.standard_normal((L, d))
+    q = rng.standard_normal((2, d))
+    P = orthonormal(d, 34)
+    ncand = L - W
+    pi = np.concatenate([rng.permutation(ncand), np.arange(ncand, L)])  # new row i = old pi[i]
+    a = oracle.decode_pair(Kt, V, q, P, r=4, k=10, W=W)
+    b = oracle.decode_pair(Kt[pi], V[pi], q, P, r=4, k=10, W=W)
+    inv = np.argsort(pi)
+    np.testing.assert_array_equal(np.sort(inv[a.sel[:a.n_sel]]), b.sel[:b.n_sel])
+    np.testing.assert_allclose(a.out, b.out, rtol=0, atol=1e-13)
+
+
+def test_positive_query_scaling_keeps_the_selection():
+    rng = np.random.default_rng(35)
+    d, L = 16, 70
+    Kt, V = rng.standard_normal((L, d)), rng.standard_normal((L, d))
+    q = rng.standard_normal((2, d))
+    P = orthonormal(d, 36)
+    a = oracle.decode_pair(Kt, V, q, P, r=4, k=9)
+    b = oracle.decode_pair(Kt, V, 4.0 * q, P, r=4, k=9)
+    np.testing.assert_array_equal(a.sel, b.sel)
+
+
+def test_attend_set_matches_decode_on_its_own_set():
+    rng = np.random.default_rng(37)
+    d, L, g = 16, 50, 2
+    Kt, V = rng.standard_normal((L, d)), rng.standard_normal((L, d))
+    q = rng.standard_normal((g, d))
+    P = orthonormal(d, 38)
+    res = oracle.decode_pair(Kt, V, q, P, r=4, k=8, W=2)
+    out = oracle.attend_set(Kt, V, oracle.rotate(q, P), res.sel[:res.n_sel])
+    np.testing.assert_array_equal(out, res.out)
+
+
+def test_batch_equals_pairs():
+    rng = np.random.default_rng(39)
+    n, Lmax, d, g = 5, 40, 16, 2
+    Kt, V = rng.standard_normal((n, Lmax, d)), rng.standard_normal((n, Lmax, d))
+    q = rng.standard_normal((n, g, d))
+    P = np.stack([orthonormal(d, 40 + i) for i in range(n)])
+    L = np.array([40, 33, 17, 1, 0])
+    kp = np.array([5, 4, 3, 2, 1])
+    out, sel = oracle.decode_batch(Kt, V, q, P, L, 4, kp, W=2)
+    for p in range(n):
+        res = oracle.decode_pair(Kt[p, :L[p]], V[p, :L[p]], q[p], P[p], r=4, k=int(kp[p]), W=2)
+        np.testing.assert_array_equal(out[p], res.out)
+        np.testing.assert_array_equal(sel[p, :len(res.sel)], res.sel)
+        assert np.all(sel[p, len(res.sel):] == -1)
+
+
+# --------------------------------------------------------------------------
+# Hand-derived fixtures
+# --------------------------------------------------------------------------
+
+def load_golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+@pytest.mark.parametrize("name", sorted(n for n in os.listdir(GOLDEN) if n.endswith(".json")))
+def test_golden_fixture(name):
+    fx = load_golden(name)
+    res = oracle.decode_pair(np.array(fx["Kt"], float), np.array(fx["V"], float),
+                             np.array(fx["q"], float), np.array(fx["P"], float),
+                             r=fx["r"], k=fx["k"], W=fx["W"],
+                             group_max=fx.get("group_max", False), scale=fx.get("scale", 0.0))
+    np.testing.assert_array_equal(res.sel[:res.n_sel], fx["expect_selected"])
+    if "expect_out" in fx:
+        np.testing.assert_allclose(res.out, np.array(fx["expect_out"], float),
+                                   rtol=0, atol=fx.get("atol", 1e-14))
