@@ -1,0 +1,218 @@
+/*
+ * loki.h - C ABI of libloki.so: Loki-style low-rank-key sparse decode
+ * attention on NVIDIA B200 (sm_100a).
+ *
+ * The method (Loki page, "Loki: Low-rank Keys for Efficient Sparse Attention",
+ * abstract; AQUA page, related work on LoKi): keys are kept in the cache in a
+ * PCA basis, K~ = K P. At a decode step the query is rotated into the same
+ * basis, every cached token is scored with only the leading r rotated
+ * dimensions, the k best tokens are kept (plus a fixed window of the most
+ * recent tokens, as in the LRQK abstract on the aitopics page "low rank
+ * approximation"), and exact softmax attention over the full head dimension
+ * runs on just those tokens (AQUA page, decode-step equations (3)-(5)).
+ *
+ * Conventions for every call:
+ *  - Ownership: the caller owns every buffer. The library never allocates
+ *    device memory and never synchronises a stream inside these calls
+ *    (loki_device_error is the one synchronous call).
+ *  - Pointers: every data pointer is a DEVICE pointer on the current CUDA
+ *    device (cudaMalloc, or the allocator of a framework). The loki_cache and
+ *    loki_batch structs themselves are host structs that the call reads
+ *    before it returns.
+ *  - Execution: launches are asynchronous and ordered on `stream` (a
+ *    cudaStream_t passed as void*; NULL is the legacy default stream).
+ *  - Errors: arguments are validated on the host before any launch; a failed
+ *    check returns a status and launches nothing. A launch failure returns
+ *    LOKI_ERR_CUDA. Values that only the device can see (sequence lengths,
+ *    block ids, per-sequence k) are checked by the kernels: an out-of-range
+ *    value is clamped into range, so memory accesses stay in bounds, and a
+ *    bit is set in the device error word that loki_device_error reads.
+ *  - Row-vector convention throughout: x_hat = x P, P row-major [d][d].
+ *  - Thread safety: calls on different streams may run concurrently.
+ */
+#ifndef LOKI_H
+#define LOKI_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define LOKI_API __attribute__((visibility("default")))
+#else
+#define LOKI_API
+#endif
+
+#define LOKI_ABI_VERSION 1
+#define LOKI_BLOCK_TOKENS 16 /* tokens per paged-cache block */
+
+typedef void* loki_stream_t; /* a cudaStream_t */
+
+typedef enum loki_status {
+    LOKI_OK = 0,
+    LOKI_ERR_INVALID_ARG = 1, /* null pointer, negative size, inconsistent sizes */
+    LOKI_ERR_UNSUPPORTED = 2, /* valid but outside what the kernels implement */
+    LOKI_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required */
+    LOKI_ERR_CUDA = 4         /* a CUDA runtime call or launch failed */
+} loki_status;
+
+typedef enum loki_dtype {
+    LOKI_F32 = 0, /* binary32 cache, queries and new keys */
+    LOKI_BF16 = 1 /* bfloat16 cache, queries and new keys */
+} loki_dtype;
+
+/* How the g query heads that share a kv head combine their approximate
+ * scores into the one score that ranks a token for that kv head. The pages
+ * are silent on grouped-query attention; SUM is the default reading (it
+ * equals scoring with the sum of the group's rotated queries), MAX the
+ * alternative. For g = 1 both are the same. */
+typedef enum loki_group_reduce {
+    LOKI_GROUP_SUM = 0,
+    LOKI_GROUP_MAX = 1
+} loki_group_reduce;
+
+/* Device error word bits (loki_device_error). */
+#define LOKI_DEVERR_SEQ_LEN 0x1u  /* a seq_lens entry outside [0, max_seq_len] */
+#define LOKI_DEVERR_BLOCK_ID 0x2u /* a block-table entry outside [0, num_blocks) */
+#define LOKI_DEVERR_K 0x4u        /* a k_per_seq entry outside [0, k] */
+#define LOKI_DEVERR_TIMEOUT 0x8u  /* a bounded wait on an async copy gave up */
+
+/* Paged KV cache in the library's own layout (LOKI_BLOCK_TOKENS tokens per
+ * block). Physical block p of kv head h holds:
+ *   keys   (PCA basis): [head_dim/16 slabs][16 tokens][16 dims]
+ *   values            : [16 tokens][head_dim]
+ * at element offset ((p * num_kv_heads + h) * 16 * head_dim). The slab layout
+ * makes the leading r dimensions of a block one contiguous run of r*16
+ * elements, which is what rank-r scoring streams. */
+typedef struct loki_cache {
+    void* k_cache;         /* device, loki_cache_bytes(), 16-byte aligned */
+    void* v_cache;         /* device, loki_cache_bytes(), 16-byte aligned */
+    int32_t num_blocks;    /* physical blocks in each cache */
+    int32_t num_kv_heads;  /* >= 1 */
+    int32_t head_dim;      /* 64 or 128 */
+    loki_dtype dtype;
+} loki_cache;
+
+/* Per-sequence addressing of one decode batch. */
+typedef struct loki_batch {
+    const int32_t* block_table; /* device [batch][max_blocks_per_seq]: physical block
+                                   of each 16-token logical block */
+    const int32_t* seq_lens;    /* device [batch]: tokens in the cache per sequence,
+                                   including the current token once appended */
+    int32_t batch;              /* >= 0; 0 makes every call a no-op */
+    int32_t max_blocks_per_seq; /* row length of block_table */
+    int32_t max_seq_len;        /* host-known bound on every seq_lens entry;
+                                   <= 16 * max_blocks_per_seq */
+} loki_batch;
+
+/* Bytes of EACH of k_cache and v_cache for the given shape; 0 for an invalid
+ * shape. */
+LOKI_API size_t loki_cache_bytes(int32_t num_blocks, int32_t num_kv_heads, int32_t head_dim,
+                        loki_dtype dtype);
+
+/* Prefill: write tokens [0, seq_lens[b]) of every sequence into the cache.
+ *
+ * k_rot, v: device [batch][num_kv_heads][max_len][head_dim] in the cache type,
+ * row-major, 16-byte aligned; max_len >= max_seq_len. The keys must already be
+ * in the PCA basis (for example because P was folded into the key projection
+ * weights); this call only lays rows out, it does no arithmetic. Tokens past
+ * seq_lens[b] are not read. */
+LOKI_API loki_status loki_prefill_cache(const loki_cache* cache, const loki_batch* batch,
+                               const void* k_rot, const void* v, int32_t max_len,
+                               loki_stream_t stream);
+
+/* Cache update of one decode step (AQUA page, decode-step equations (1)-(2),
+ * for keys kept in the PCA basis): for every sequence b and kv head h,
+ *   K~[b, h, seq_lens[b]-1, :] = round(k_new[b, h, :] P[h])   (fp32 accumulation,
+ *                                round-to-nearest-even to the cache type)
+ *   V [b, h, seq_lens[b]-1, :] = v_new[b, h, :]
+ * so seq_lens must already count the new token. Sequences with seq_lens[b] = 0
+ * are skipped.
+ *
+ * k_new, v_new: device [batch][num_kv_heads][head_dim] in the cache type.
+ * P: device fp32 [num_kv_heads][head_dim][head_dim], row-major, 16-byte
+ * aligned; NULL means the keys are already in the PCA basis (copied as is). */
+LOKI_API loki_status loki_append_keys(const loki_cache* cache, const loki_batch* batch,
+                             const void* k_new, const void* v_new, const float* P,
+                             loki_stream_t stream);
+
+/* Workspace bytes loki_decode_attention needs for these sizes (may be 0). */
+LOKI_API size_t loki_decode_workspace_bytes(const loki_cache* cache, const loki_batch* batch,
+                                   int32_t num_q_heads, int32_t k, int32_t recent_window);
+
+/* One Loki sparse decode step for every sequence b and query head j, with
+ * kv head h = j / g (g = num_q_heads / num_kv_heads, contiguous groups) and
+ * L = seq_lens[b]:
+ *   1. q_hat_j = q_j P[h]                                (fp32)
+ *   2. candidates t in [0, L - W'), W' = min(recent_window, L); approximate
+ *      score s_t = reduce_{j in group(h)} q_hat_j[:r] . K~[t, :r]
+ *      (AQUA page, related work on LoKi: slicing after projection; Loki
+ *      abstract: scores in the low-dimensional space; reduce = SUM or MAX)
+ *   3. keep the min(k_b, candidates) largest s_t, ties to the lower t, plus
+ *      the W' most recent tokens (aitopics page, LRQK abstract)
+ *   4. out_j = softmax over the kept set of (q_hat_j . K~[t, :] * scale) times V
+ *      (AQUA page, decode-step equations (3)-(5)), fp32.
+ *
+ * q: device [batch][num_q_heads][head_dim] in the cache type, unrotated.
+ * P: device fp32 [num_kv_heads][head_dim][head_dim], 16-byte aligned.
+ * r: leading dimensions used for scoring; a multiple of 16 in [16, head_dim].
+ * k: tokens kept by score (the per-sequence maximum when k_per_seq is given).
+ * k_per_seq: nullable device int32 [batch]; entries clamped to [0, k].
+ * recent_window: W >= 0; k = 0 together with W = 0 is invalid.
+ * scale: exact-logit scale; 0 means 1/sqrt(head_dim).
+ * out: device fp32 [batch][num_q_heads][head_dim].
+ * selected_idx: nullable device int32 [batch][num_kv_heads][k + recent_window]:
+ *   the kept token indices of each (sequence, kv head) in ascending order,
+ *   then -1 padding.
+ * workspace: device, >= loki_decode_workspace_bytes(); may be NULL if that is 0.
+ *
+ * Unsupported (LOKI_ERR_UNSUPPORTED): head_dim other than 64/128, group size
+ * other than 1, 2, 4, 8, r not a multiple of 16, or max_seq_len above
+ * loki_decode_max_seq_len(). */
+LOKI_API loki_status loki_decode_attention(const loki_cache* cache, const loki_batch* batch,
+                                  const void* q, int32_t num_q_heads, const float* P,
+                                  int32_t r, int32_t k, const int32_t* k_per_seq,
+                                  int32_t recent_window, loki_group_reduce group_reduce,
+                                  float scale, float* out, int32_t* selected_idx,
+                                  void* workspace, size_t workspace_bytes,
+                                  loki_stream_t stream);
+
+/* Largest max_seq_len loki_decode_attention accepts for this cache shape. */
+LOKI_API int32_t loki_decode_max_seq_len(int32_t head_dim, loki_dtype dtype);
+
+/* Workspace bytes loki_dense_attention needs for these sizes. */
+LOKI_API size_t loki_dense_workspace_bytes(const loki_cache* cache, const loki_batch* batch,
+                                  int32_t num_q_heads);
+
+/* Dense decode attention, the full-attention comparison path (AQUA page,
+ * decode-step equations (3)-(5) over every cached token):
+ *   out_j = softmax over t in [0, L) of (q_hat_j . K~[t, :] * scale) times V
+ * with q_hat_j = q_j P[h]; by the rotation invariance of the AQUA page's
+ * appendix this equals attention with the unrotated keys.
+ * Arguments as for loki_decode_attention. Runs as flash-decode split-K: each
+ * split writes (max, sum, unnormalised output) partials to the workspace and a
+ * second kernel merges them. */
+LOKI_API loki_status loki_dense_attention(const loki_cache* cache, const loki_batch* batch,
+                                 const void* q, int32_t num_q_heads, const float* P,
+                                 float scale, float* out, void* workspace,
+                                 size_t workspace_bytes, loki_stream_t stream);
+
+/* Reads (and with clear != 0 resets) the device error word of the current
+ * device: an OR of LOKI_DEVERR_* bits set by kernels since the last clear.
+ * Synchronises the device. */
+LOKI_API loki_status loki_device_error(int32_t clear, uint32_t* bits);
+
+/* Static description of a status code. */
+LOKI_API const char* loki_status_string(loki_status status);
+
+/* LOKI_ABI_VERSION of the loaded library. */
+LOKI_API int32_t loki_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LOKI_H */

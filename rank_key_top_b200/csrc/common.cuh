@@ -1,0 +1,221 @@
+// Device-side helpers shared by the libloki kernels: cache layout, typed
+// loads, order-preserving score keys, mbarrier + bulk-copy (TMA) wrappers and
+// the device error word. Included once, by loki.cu, so that every kernel and
+// the error word live in one translation unit.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/loki.h"
+
+namespace loki {
+
+constexpr int kBlockTokens = LOKI_BLOCK_TOKENS;  // tokens per paged block
+constexpr int kSlabDims = 16;                    // dims per key slab
+
+// Sticky device error word (LOKI_DEVERR_* bits), one per device.
+__device__ uint32_t g_device_error;
+
+__device__ __forceinline__ void flag_error(uint32_t bits) { atomicOr(&g_device_error, bits); }
+
+// ---------------------------------------------------------------------------
+// Paged cache layout. Block p of kv head h starts at element
+// (p * Hkv + h) * 16 * D in both caches.
+//   keys:   [D/16 slabs][16 tokens][16 dims]
+//   values: [16 tokens][D]
+// ---------------------------------------------------------------------------
+__host__ __device__ __forceinline__ int64_t page_offset(int64_t block, int h, int Hkv, int D) {
+    return (block * Hkv + h) * (int64_t)(kBlockTokens * D);
+}
+__host__ __device__ __forceinline__ int key_offset_in_page(int token, int dim) {
+    return (dim / kSlabDims) * (kBlockTokens * kSlabDims) + token * kSlabDims + (dim % kSlabDims);
+}
+__host__ __device__ __forceinline__ int value_offset_in_page(int token, int dim, int D) {
+    return token * D + dim;
+}
+
+// ---------------------------------------------------------------------------
+// Typed element access.
+// ---------------------------------------------------------------------------
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+    static __device__ __forceinline__ float to_f(float x) { return x; }
+    static __device__ __forceinline__ float from_f(float x) { return x; }
+};
+template <> struct Elem<__nv_bfloat16> {
+    static __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+    static __device__ __forceinline__ __nv_bfloat16 from_f(float x) { return __float2bfloat16_rn(x); }
+};
+
+// N consecutive elements (N * sizeof(T) in {4, 8, 16, 32} bytes, naturally
+// aligned) loaded with the widest vector load and converted to fp32.
+template <typename T, int N> struct Vec;
+
+template <int N> struct Vec<__nv_bfloat16, N> {
+    static_assert(N == 2 || N == 4 || N == 8, "bf16 vector width");
+    using raw_t = typename std::conditional<N == 2, uint32_t,
+                  typename std::conditional<N == 4, uint2, uint4>::type>::type;
+    static __device__ __forceinline__ raw_t load(const __nv_bfloat16* p) {
+        return *reinterpret_cast<const raw_t*>(p);
+    }
+    static __device__ __forceinline__ void unpack_word(uint32_t w, float* f) {
+        f[0] = __uint_as_float(w << 16);
+        f[1] = __uint_as_float(w & 0xffff0000u);
+    }
+    static __device__ __forceinline__ void to_float(const raw_t& r, float* f) {
+        if constexpr (N == 2) {
+            unpack_word(r, f);
+        } else if constexpr (N == 4) {
+            unpack_word(r.x, f);
+            unpack_word(r.y, f + 2);
+        } else {
+            unpack_word(r.x, f);
+            unpack_word(r.y, f + 2);
+            unpack_word(r.z, f + 4);
+            unpack_word(r.w, f + 6);
+        }
+    }
+};
+
+template <int N> struct Vec<float, N> {
+    static_assert(N == 2 || N == 4 || N == 8, "f32 vector width");
+    struct raw8 { float4 a, b; };
+    using raw_t = typename std::conditional<N == 2, float2,
+                  typename std::conditional<N == 4, float4, raw8>::type>::type;
+    static __device__ __forceinline__ raw_t load(const float* p) {
+        if constexpr (N == 8) {
+            raw8 r;
+            r.a = *reinterpret_cast<const float4*>(p);
+            r.b = *reinterpret_cast<const float4*>(p + 4);
+            return r;
+        } else {
+            return *reinterpret_cast<const raw_t*>(p);
+        }
+    }
+    static __device__ __forceinline__ void to_float(const raw_t& r, float* f) {
+        if constexpr (N == 2) {
+            f[0] = r.x; f[1] = r.y;
+        } else if constexpr (N == 4) {
+            f[0] = r.x; f[1] = r.y; f[2] = r.z; f[3] = r.w;
+        } else {
+            f[0] = r.a.x; f[1] = r.a.y; f[2] = r.a.z; f[3] = r.a.w;
+            f[4] = r.b.x; f[5] = r.b.y; f[6] = r.b.z; f[7] = r.b.w;
+        }
+    }
+};
+
+// ---------------------------------------------------------------------------
+// Order-preserving map of an fp32 score to a uint32 key: a > b (as floats,
+// with -0 == +0) iff key(a) > key(b). -0 is canonicalised to +0 first.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t score_key(float s) {
+    uint32_t u = __float_as_uint(s + 0.0f);  // -0 + 0 = +0 under round-to-nearest
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier and bulk async copy (TMA engine, non-tensor form) wrappers.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbarrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+// Bulk copy global -> this CTA's shared memory, completing on `bar`.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for phase `parity` of `bar`. Gives up after kWaitLimit polls
+// (each poll may suspend the thread for a while in hardware), sets
+// LOKI_DEVERR_TIMEOUT and returns false; the caller then treats the data as
+// absent and keeps going so that every barrier of the CTA is still reached.
+constexpr uint32_t kWaitLimit = 1u << 22;
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kWaitLimit; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    flag_error(LOKI_DEVERR_TIMEOUT);
+    return false;
+}
+
+// ---------------------------------------------------------------------------
+// Warp helpers.
+// ---------------------------------------------------------------------------
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ float warp_max_xor(float v, int lo_bit, int hi_bit) {
+    for (int b = lo_bit; b < hi_bit; ++b) v = fmaxf(v, __shfl_xor_sync(kFull, v, 1 << b));
+    return v;
+}
+__device__ __forceinline__ float warp_sum_xor(float v, int lo_bit, int hi_bit) {
+    for (int b = lo_bit; b < hi_bit; ++b) v += __shfl_xor_sync(kFull, v, 1 << b);
+    return v;
+}
+
+// Transpose-reduce: every lane holds NV partial values; afterwards the values
+// are summed over all 32 lanes and lane l holds the total of value index
+// (l >> (5 - log2(NV))). Uses NV - 1 + (5 - log2 NV) shuffles instead of
+// 5 * NV.
+template <int NV>
+__device__ __forceinline__ float transpose_reduce(float (&v)[NV], int lane) {
+    static_assert(NV >= 1 && NV <= 32 && (NV & (NV - 1)) == 0, "NV power of two <= 32");
+    int n = NV;
+    int mask = 16;
+#pragma unroll
+    for (int level = 0; level < 5; ++level) {
+        if (n > 1) {
+            const int half = n >> 1;
+            const bool upper = (lane & mask) != 0;
+#pragma unroll
+            for (int i = 0; i < NV / 2; ++i) {
+                if (i < half) {
+                    float send = upper ? v[i] : v[i + half];
+                    float keep = upper ? v[i + half] : v[i];
+                    v[i] = keep + __shfl_xor_sync(kFull, send, mask);
+                }
+            }
+            n = half;
+        } else {
+            v[0] += __shfl_xor_sync(kFull, v[0], mask);
+        }
+        mask >>= 1;
+    }
+    return v[0];
+}
+
+}  // namespace loki

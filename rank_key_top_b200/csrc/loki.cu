@@ -1,0 +1,441 @@
+// libloki: host entry points of the C ABI declared in include/loki.h.
+// Every kernel is included here so that the device error word and all
+// kernels share one translation unit.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <map>
+#include <mutex>
+
+#include "cache_kernels.cuh"
+#include "dense.cuh"
+#include "sparse_decode.cuh"
+
+using namespace loki;
+
+namespace {
+
+constexpr double kLog2e = 1.4426950408889634;
+
+size_t elem_size(loki_dtype dt) { return dt == LOKI_BF16 ? 2 : 4; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape checks shared by every call that reads a cache.
+loki_status check_cache(const loki_cache* c) {
+    if (!c) return LOKI_ERR_INVALID_ARG;
+    if (c->dtype != LOKI_F32 && c->dtype != LOKI_BF16) return LOKI_ERR_INVALID_ARG;
+    if (c->num_blocks < 0 || c->num_kv_heads < 1 || c->head_dim < 1) return LOKI_ERR_INVALID_ARG;
+    if (c->head_dim != 64 && c->head_dim != 128) return LOKI_ERR_UNSUPPORTED;
+    if (c->num_blocks > 0 && (!c->k_cache || !c->v_cache)) return LOKI_ERR_INVALID_ARG;
+    if (!aligned16(c->k_cache) || !aligned16(c->v_cache)) return LOKI_ERR_INVALID_ARG;
+    return LOKI_OK;
+}
+
+loki_status check_batch(const loki_batch* bt) {
+    if (!bt) return LOKI_ERR_INVALID_ARG;
+    if (bt->batch < 0 || bt->max_blocks_per_seq < 0 || bt->max_seq_len < 0) return LOKI_ERR_INVALID_ARG;
+    if (bt->batch == 0) return LOKI_OK;
+    if (!bt->block_table || !bt->seq_lens) return LOKI_ERR_INVALID_ARG;
+    if ((int64_t)bt->max_seq_len > (int64_t)bt->max_blocks_per_seq * kBlockTokens) return LOKI_ERR_INVALID_ARG;
+    return LOKI_OK;
+}
+
+loki_status launch_status() {
+    return cudaPeekAtLastError() == cudaSuccess ? LOKI_OK : LOKI_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Dispatch over element type, head dim and group size.
+// ---------------------------------------------------------------------------
+template <template <typename, int, int> class F, typename... A>
+loki_status dispatch_tdg(loki_dtype dt, int D, int G, A&&... a) {
+#define LOKI_CASE(T_, D_, G_) \
+    if (D == D_ && G == G_) return F<T_, D_, G_>::run(std::forward<A>(a)...);
+#define LOKI_CASES_D(T_, D_) LOKI_CASE(T_, D_, 1) LOKI_CASE(T_, D_, 2) LOKI_CASE(T_, D_, 4) LOKI_CASE(T_, D_, 8)
+    if (dt == LOKI_BF16) {
+        LOKI_CASES_D(__nv_bfloat16, 64)
+        LOKI_CASES_D(__nv_bfloat16, 128)
+    } else {
+        LOKI_CASES_D(float, 64)
+        LOKI_CASES_D(float, 128)
+    }
+#undef LOKI_CASES_D
+#undef LOKI_CASE
+    return LOKI_ERR_UNSUPPORTED;
+}
+
+// ---------------------------------------------------------------------------
+// Sparse decode launch geometry.
+// ---------------------------------------------------------------------------
+struct DeviceInfo {
+    int sms = 0;
+    int max_smem_optin = 0;
+};
+
+DeviceInfo device_info() {
+    static std::mutex mu;
+    static DeviceInfo cache[64];
+    static bool have[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev >= 0 && dev < 64 && have[dev]) return cache[dev];
+    DeviceInfo di;
+    cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&di.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (dev >= 0 && dev < 64) {
+        cache[dev] = di;
+        have[dev] = true;
+    }
+    return di;
+}
+
+void sparse_layout(SparseParams& p, int D, int G, size_t esize) {
+    auto align = [](int x) { return (x + 127) & ~127; };
+    int off = 0;
+    p.off_keys = off;
+    off = align(off + std::max(p.cta_tokens * 4, D * D * 4));
+    p.off_ring = off;
+    off = align(off + kWarps * kRingBytesPerWarp);
+    p.off_list = off;
+    off = align(off + p.cta_tokens * 2);
+    p.off_qf = off;
+    off = align(off + G * D * 4);
+    p.off_qhat = off;
+    off = align(off + G * D * 4);
+    p.off_qs = off;
+    off = align(off + D * 4);
+    p.off_tbl = off;
+    off = align(off + (p.cta_tokens / kBlockTokens) * 4);
+    p.off_hist = off;
+    off = align(off + 2 * kHistBins * 4);
+    p.off_bars = off;
+    off = align(off + (kWarps * kMaxSlots + 1) * 8);
+    p.off_part = off;
+    off = align(off + G * (D + 2) * 4);
+    p.off_misc = off;
+    off = align(off + 64 * 4);
+    p.smem_bytes = off;
+    p.slot_bytes = p.r * kBlockTokens * (int)esize;
+    p.slots = std::min(kMaxSlots, std::max(1, kRingBytesPerWarp / p.slot_bytes));
+}
+
+// Whether at least one cluster of this shape can be resident on the device,
+// cached per kernel instantiation, cluster size and shared-memory size.
+template <typename K>
+bool cluster_fits(K kern, const cudaLaunchConfig_t& cfg, std::map<std::pair<int, int>, bool>& known,
+                  std::mutex& mu) {
+    const std::pair<int, int> key(cfg.gridDim.x, (int)cfg.dynamicSmemBytes);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = known.find(key);
+    if (it != known.end()) return it->second;
+    int n = 0;
+    cudaLaunchConfig_t probe = cfg;
+    probe.gridDim = dim3(cfg.gridDim.x, 1, 1);
+    const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kern, &probe);
+    if (e != cudaSuccess) cudaGetLastError();
+    const bool fits = e == cudaSuccess && n > 0;
+    known[key] = fits;
+    return fits;
+}
+
+template <typename T, int D, int G>
+struct SparseLaunch {
+    static loki_status run(SparseParams p, int pairs, cudaStream_t stream) {
+        auto kern = sparse_decode_kernel<T, D, G>;
+        static std::once_flag once;
+        static cudaError_t attr_err = cudaSuccess;
+        std::call_once(once, [&] {
+            attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+            if (attr_err == cudaSuccess)
+                attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        });
+        if (attr_err != cudaSuccess) return LOKI_ERR_CUDA;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(p.C, pairs, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = p.smem_bytes;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = p.C;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        // a cluster that can never be resident is reported, not launched
+        static std::map<std::pair<int, int>, bool> known;
+        static std::mutex known_mu;
+        if (!cluster_fits(kern, cfg, known, known_mu)) return LOKI_ERR_UNSUPPORTED;
+        if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return LOKI_ERR_CUDA;
+        return launch_status();
+    }
+};
+
+// Cluster size: enough CTAs that each holds at most kCtaTokenCap tokens, then
+// as many as still fit every cluster on the GPU at once (one CTA per SM),
+// keeping at least 512 tokens per CTA.
+int choose_cluster(int max_seq_len, int pairs, int sms) {
+    const int nblk = (max_seq_len + kBlockTokens - 1) / kBlockTokens;
+    const int cap_blocks = kCtaTokenCap / kBlockTokens;
+    int C = std::max(1, (nblk + cap_blocks - 1) / cap_blocks);
+    if (C > 16) return -1;
+    for (int cand = C + 1; cand <= 16; ++cand) {
+        if ((int64_t)pairs * cand > sms) break;
+        if (nblk / cand < 32) break;
+        C = cand;
+    }
+    return C;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t loki_cache_bytes(int32_t num_blocks, int32_t num_kv_heads, int32_t head_dim, loki_dtype dtype) {
+    if (num_blocks < 0 || num_kv_heads < 1 || (head_dim != 64 && head_dim != 128)) return 0;
+    if (dtype != LOKI_F32 && dtype != LOKI_BF16) return 0;
+    return (size_t)num_blocks * num_kv_heads * kBlockTokens * head_dim * elem_size(dtype);
+}
+
+int32_t loki_abi_version(void) { return LOKI_ABI_VERSION; }
+
+const char* loki_status_string(loki_status s) {
+    switch (s) {
+        case LOKI_OK: return "ok";
+        case LOKI_ERR_INVALID_ARG: return "invalid argument";
+        case LOKI_ERR_UNSUPPORTED: return "unsupported shape or option";
+        case LOKI_ERR_WORKSPACE: return "workspace missing or too small";
+        case LOKI_ERR_CUDA: return "CUDA runtime error";
+    }
+    return "unknown status";
+}
+
+loki_status loki_device_error(int32_t clear, uint32_t* bits) {
+    if (!bits) return LOKI_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return LOKI_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(bits, g_device_error, sizeof(uint32_t)) != cudaSuccess) return LOKI_ERR_CUDA;
+    if (clear) {
+        const uint32_t zero = 0;
+        if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(uint32_t)) != cudaSuccess) return LOKI_ERR_CUDA;
+    }
+    return LOKI_OK;
+}
+
+loki_status loki_prefill_cache(const loki_cache* cache, const loki_batch* batch, const void* k_rot,
+                               const void* v, int32_t max_len, loki_stream_t stream) {
+    loki_status st = check_cache(cache);
+    if (st != LOKI_OK) return st;
+    if ((st = check_batch(batch)) != LOKI_OK) return st;
+    if (batch->batch == 0 || batch->max_blocks_per_seq == 0) return LOKI_OK;
+    if (!k_rot || !v || max_len < batch->max_seq_len) return LOKI_ERR_INVALID_ARG;
+    if (!aligned16(k_rot) || !aligned16(v)) return LOKI_ERR_INVALID_ARG;
+    if ((int64_t)batch->batch * cache->num_kv_heads > 65535) return LOKI_ERR_UNSUPPORTED;
+    PrefillParams p;
+    p.k_cache = cache->k_cache;
+    p.v_cache = cache->v_cache;
+    p.block_table = batch->block_table;
+    p.seq_lens = batch->seq_lens;
+    p.k_rot = k_rot;
+    p.v = v;
+    p.num_blocks = cache->num_blocks;
+    p.Hkv = cache->num_kv_heads;
+    p.max_blocks = batch->max_blocks_per_seq;
+    p.max_seq_len = batch->max_seq_len;
+    p.max_len = max_len;
+    const int nblk = (batch->max_seq_len + kBlockTokens - 1) / kBlockTokens;
+    if (nblk == 0) return LOKI_OK;
+    dim3 grid(nblk, batch->batch * cache->num_kv_heads);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int D = cache->head_dim;
+    if (cache->dtype == LOKI_BF16) {
+        if (D == 64) prefill_kernel<__nv_bfloat16, 64><<<grid, 256, 0, s>>>(p);
+        else prefill_kernel<__nv_bfloat16, 128><<<grid, 256, 0, s>>>(p);
+    } else {
+        if (D == 64) prefill_kernel<float, 64><<<grid, 256, 0, s>>>(p);
+        else prefill_kernel<float, 128><<<grid, 256, 0, s>>>(p);
+    }
+    return launch_status();
+}
+
+loki_status loki_append_keys(const loki_cache* cache, const loki_batch* batch, const void* k_new,
+                             const void* v_new, const float* P, loki_stream_t stream) {
+    loki_status st = check_cache(cache);
+    if (st != LOKI_OK) return st;
+    if ((st = check_batch(batch)) != LOKI_OK) return st;
+    if (batch->batch == 0) return LOKI_OK;
+    if (!k_new || !v_new) return LOKI_ERR_INVALID_ARG;
+    if ((int64_t)batch->batch * cache->num_kv_heads > INT32_MAX / 2) return LOKI_ERR_UNSUPPORTED;
+    AppendParams p;
+    p.k_cache = cache->k_cache;
+    p.v_cache = cache->v_cache;
+    p.block_table = batch->block_table;
+    p.seq_lens = batch->seq_lens;
+    p.k_new = k_new;
+    p.v_new = v_new;
+    p.P = P;
+    p.num_blocks = cache->num_blocks;
+    p.Hkv = cache->num_kv_heads;
+    p.max_blocks = batch->max_blocks_per_seq;
+    p.max_seq_len = batch->max_seq_len;
+    const int grid = batch->batch * cache->num_kv_heads;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int D = cache->head_dim;
+    if (cache->dtype == LOKI_BF16) {
+        if (D == 64) append_kernel<__nv_bfloat16, 64><<<grid, 64, 0, s>>>(p);
+        else append_kernel<__nv_bfloat16, 128><<<grid, 128, 0, s>>>(p);
+    } else {
+        if (D == 64) append_kernel<float, 64><<<grid, 64, 0, s>>>(p);
+        else append_kernel<float, 128><<<grid, 128, 0, s>>>(p);
+    }
+    return launch_status();
+}
+
+int32_t loki_decode_max_seq_len(int32_t head_dim, loki_dtype dtype) {
+    (void)dtype;
+    if (head_dim != 64 && head_dim != 128) return 0;
+    return 16 * kCtaTokenCap;
+}
+
+size_t loki_decode_workspace_bytes(const loki_cache* cache, const loki_batch* batch, int32_t num_q_heads,
+                                   int32_t k, int32_t recent_window) {
+    (void)cache;
+    (void)batch;
+    (void)num_q_heads;
+    (void)k;
+    (void)recent_window;
+    return 0;  // the fused kernel keeps every intermediate on chip
+}
+
+loki_status loki_decode_attention(const loki_cache* cache, const loki_batch* batch, const void* q,
+                                  int32_t num_q_heads, const float* P, int32_t r, int32_t k,
+                                  const int32_t* k_per_seq, int32_t recent_window,
+                                  loki_group_reduce group_reduce, float scale, float* out,
+                                  int32_t* selected_idx, void* workspace, size_t workspace_bytes,
+                                  loki_stream_t stream) {
+    (void)workspace;
+    (void)workspace_bytes;
+    loki_status st = check_cache(cache);
+    if (st != LOKI_OK) return st;
+    if ((st = check_batch(batch)) != LOKI_OK) return st;
+    const int Hkv = cache->num_kv_heads, D = cache->head_dim;
+    if (num_q_heads < 1 || num_q_heads % Hkv != 0) return LOKI_ERR_INVALID_ARG;
+    if (k < 0 || recent_window < 0 || (k == 0 && recent_window == 0)) return LOKI_ERR_INVALID_ARG;
+    if (r < 1 || r > D) return LOKI_ERR_INVALID_ARG;
+    if (group_reduce != LOKI_GROUP_SUM && group_reduce != LOKI_GROUP_MAX) return LOKI_ERR_INVALID_ARG;
+    if (!(scale >= 0.f) || std::isinf(scale)) return LOKI_ERR_INVALID_ARG;
+    if ((int64_t)k + recent_window > INT32_MAX / 2) return LOKI_ERR_INVALID_ARG;
+    if (batch->batch == 0) return LOKI_OK;
+    if (!q || !P || !out) return LOKI_ERR_INVALID_ARG;
+    if (!aligned16(P)) return LOKI_ERR_INVALID_ARG;
+    const int G = num_q_heads / Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return LOKI_ERR_UNSUPPORTED;
+    if (r % kSlabDims != 0) return LOKI_ERR_UNSUPPORTED;
+    const int pairs = batch->batch * Hkv;
+    if ((int64_t)batch->batch * Hkv > 65535) return LOKI_ERR_UNSUPPORTED;
+    if (batch->max_seq_len > loki_decode_max_seq_len(D, cache->dtype)) return LOKI_ERR_UNSUPPORTED;
+
+    const DeviceInfo di = device_info();
+    const int C = choose_cluster(batch->max_seq_len, pairs, di.sms);
+    if (C < 1) return LOKI_ERR_UNSUPPORTED;
+    SparseParams p;
+    p.k_cache = cache->k_cache;
+    p.v_cache = cache->v_cache;
+    p.block_table = batch->block_table;
+    p.seq_lens = batch->seq_lens;
+    p.k_per_seq = k_per_seq;
+    p.q = q;
+    p.P = P;
+    p.out = out;
+    p.sel = selected_idx;
+    p.num_blocks = cache->num_blocks;
+    p.Hkv = Hkv;
+    p.max_blocks = batch->max_blocks_per_seq;
+    p.max_seq_len = batch->max_seq_len;
+    p.r = r;
+    p.k = k;
+    p.W = recent_window;
+    p.group_max = group_reduce == LOKI_GROUP_MAX ? 1 : 0;
+    const double sc = scale == 0.f ? 1.0 / std::sqrt((double)D) : (double)scale;
+    p.scale_log2 = (float)(sc * kLog2e);
+    p.C = C;
+    const int nblk = (batch->max_seq_len + kBlockTokens - 1) / kBlockTokens;
+    p.cta_tokens = std::max(1, (nblk + C - 1) / C) * kBlockTokens;
+    sparse_layout(p, D, G, elem_size(cache->dtype));
+    if (p.smem_bytes > di.max_smem_optin) return LOKI_ERR_UNSUPPORTED;
+    return dispatch_tdg<SparseLaunch>(cache->dtype, D, G, p, pairs, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+namespace {
+
+int dense_splits(int max_seq_len) { return std::max(1, (max_seq_len + kDenseSplitTokens - 1) / kDenseSplitTokens); }
+
+template <typename T, int D, int G>
+struct DenseLaunch {
+    static loki_status run(DenseParams p, int batch, cudaStream_t s) {
+        const int pairs = batch * p.Hkv;
+        rotate_query_kernel<T, D, G><<<pairs, 256, 0, s>>>(p);
+        dense_split_kernel<T, D, G><<<dim3(p.splits, pairs), 256, 0, s>>>(p);
+        merge_kernel<D, G><<<batch * p.Hkv * G, D, 0, s>>>(p);
+        return launch_status();
+    }
+};
+
+}  // namespace
+
+extern "C" {
+
+size_t loki_dense_workspace_bytes(const loki_cache* cache, const loki_batch* batch, int32_t num_q_heads) {
+    if (check_cache(cache) != LOKI_OK || check_batch(batch) != LOKI_OK || num_q_heads < 1) return 0;
+    const size_t D = cache->head_dim;
+    const size_t G = (size_t)num_q_heads / cache->num_kv_heads;
+    const size_t qhat = (size_t)batch->batch * num_q_heads * D * 4;
+    const size_t parts = (size_t)batch->batch * cache->num_kv_heads * dense_splits(batch->max_seq_len) * G *
+                         (D + 2) * 4;
+    return ((qhat + 255) & ~(size_t)255) + parts;
+}
+
+loki_status loki_dense_attention(const loki_cache* cache, const loki_batch* batch, const void* q,
+                                 int32_t num_q_heads, const float* P, float scale, float* out,
+                                 void* workspace, size_t workspace_bytes, loki_stream_t stream) {
+    loki_status st = check_cache(cache);
+    if (st != LOKI_OK) return st;
+    if ((st = check_batch(batch)) != LOKI_OK) return st;
+    const int Hkv = cache->num_kv_heads, D = cache->head_dim;
+    if (num_q_heads < 1 || num_q_heads % Hkv != 0) return LOKI_ERR_INVALID_ARG;
+    if (!(scale >= 0.f) || std::isinf(scale)) return LOKI_ERR_INVALID_ARG;
+    if (batch->batch == 0) return LOKI_OK;
+    if (!q || !P || !out) return LOKI_ERR_INVALID_ARG;
+    const int G = num_q_heads / Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return LOKI_ERR_UNSUPPORTED;
+    const int splits = dense_splits(batch->max_seq_len);
+    if ((int64_t)batch->batch * Hkv > 65535 || splits > INT32_MAX / 4) return LOKI_ERR_UNSUPPORTED;
+    const size_t need = loki_dense_workspace_bytes(cache, batch, num_q_heads);
+    if (!workspace || workspace_bytes < need) return LOKI_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return LOKI_ERR_INVALID_ARG;
+    DenseParams p;
+    p.k_cache = cache->k_cache;
+    p.v_cache = cache->v_cache;
+    p.block_table = batch->block_table;
+    p.seq_lens = batch->seq_lens;
+    p.q = q;
+    p.P = P;
+    p.out = out;
+    const size_t qhat_bytes = ((size_t)batch->batch * num_q_heads * D * 4 + 255) & ~(size_t)255;
+    p.qhat = reinterpret_cast<float*>(workspace);
+    p.parts = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + qhat_bytes);
+    p.num_blocks = cache->num_blocks;
+    p.Hkv = Hkv;
+    p.max_blocks = batch->max_blocks_per_seq;
+    p.max_seq_len = batch->max_seq_len;
+    p.splits = splits;
+    const double sc = scale == 0.f ? 1.0 / std::sqrt((double)D) : (double)scale;
+    p.scale_log2 = (float)(sc * kLog2e);
+    return dispatch_tdg<DenseLaunch>(cache->dtype, D, G, p, batch->batch, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

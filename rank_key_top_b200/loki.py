@@ -1,0 +1,205 @@
+"""Thin ctypes binding of libloki.so (include/loki.h), with the same names.
+
+Argument marshalling only: torch tensors in, raw device pointers and sizes
+out. Every step of the computation runs in the CUDA kernels of libloki.so;
+there is no fallback. Importing this module fails loudly if the library is
+missing. A non-OK status raises LokiError.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libloki.so")
+
+LOKI_OK = 0
+LOKI_ERR_INVALID_ARG = 1
+LOKI_ERR_UNSUPPORTED = 2
+LOKI_ERR_WORKSPACE = 3
+LOKI_ERR_CUDA = 4
+
+LOKI_F32 = 0
+LOKI_BF16 = 1
+LOKI_GROUP_SUM = 0
+LOKI_GROUP_MAX = 1
+
+LOKI_DEVERR_SEQ_LEN = 0x1
+LOKI_DEVERR_BLOCK_ID = 0x2
+LOKI_DEVERR_K = 0x4
+LOKI_DEVERR_TIMEOUT = 0x8
+
+BLOCK_TOKENS = 16
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libloki.so is not built ({LIB_PATH}); run rank_key_top_b200/build.py")
+_lib = ctypes.CDLL(LIB_PATH)
+
+
+class loki_cache(ctypes.Structure):
+    _fields_ = [("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+                ("num_blocks", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("dtype", ctypes.c_int)]
+
+
+class loki_batch(ctypes.Structure):
+    _fields_ = [("block_table", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
+                ("batch", ctypes.c_int32), ("max_blocks_per_seq", ctypes.c_int32),
+                ("max_seq_len", ctypes.c_int32)]
+
+
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_SZ = ctypes.c_size_t
+_C = ctypes.POINTER(loki_cache)
+_B = ctypes.POINTER(loki_batch)
+
+_SIGS = {
+    "loki_cache_bytes": (_SZ, [_I32, _I32, _I32, ctypes.c_int]),
+    "loki_prefill_cache": (ctypes.c_int, [_C, _B, _P, _P, _I32, _P]),
+    "loki_append_keys": (ctypes.c_int, [_C, _B, _P, _P, _P, _P]),
+    "loki_decode_workspace_bytes": (_SZ, [_C, _B, _I32, _I32, _I32]),
+    "loki_decode_attention": (ctypes.c_int, [_C, _B, _P, _I32, _P, _I32, _I32, _P, _I32,
+                                             ctypes.c_int, ctypes.c_float, _P, _P, _P, _SZ, _P]),
+    "loki_decode_max_seq_len": (_I32, [_I32, ctypes.c_int]),
+    "loki_dense_workspace_bytes": (_SZ, [_C, _B, _I32]),
+    "loki_dense_attention": (ctypes.c_int, [_C, _B, _P, _I32, _P, ctypes.c_float, _P, _P, _SZ, _P]),
+    "loki_device_error": (ctypes.c_int, [_I32, ctypes.POINTER(ctypes.c_uint32)]),
+    "loki_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "loki_abi_version": (_I32, []),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+EXPORTED = tuple(_SIGS)
+
+
+class LokiError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__(f"{fn}: {loki_status_string(status)} (status {status})")
+
+
+def _check(fn, status):
+    if status != LOKI_OK:
+        raise LokiError(fn, status)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def dtype_code(dt) -> int:
+    return {torch.bfloat16: LOKI_BF16, torch.float32: LOKI_F32}[dt]
+
+
+# --------------------------------------------------------------------------
+# Struct builders
+# --------------------------------------------------------------------------
+
+class Cache:
+    """Owns a k/v cache pair (torch uint8 buffers) and its loki_cache struct."""
+
+    def __init__(self, num_blocks, num_kv_heads, head_dim, dtype, device="cuda"):
+        code = dtype_code(dtype)
+        nbytes = loki_cache_bytes(num_blocks, num_kv_heads, head_dim, code)
+        if nbytes == 0 and num_blocks > 0:
+            raise ValueError("invalid cache shape")
+        self.dtype = dtype
+        self.k = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+        self.v = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+        self.struct = loki_cache(self.k.data_ptr(), self.v.data_ptr(), num_blocks, num_kv_heads,
+                                 head_dim, code)
+
+
+class Batch:
+    """Keeps the device block table and lengths alive with their struct."""
+
+    def __init__(self, block_table, seq_lens, max_seq_len=None):
+        assert block_table.dtype == torch.int32 and seq_lens.dtype == torch.int32
+        self.block_table = block_table.contiguous()
+        self.seq_lens = seq_lens.contiguous()
+        if max_seq_len is None:
+            max_seq_len = int(seq_lens.max().item()) if seq_lens.numel() else 0
+        B = self.seq_lens.numel()
+        self.struct = loki_batch(self.block_table.data_ptr(), self.seq_lens.data_ptr(), B,
+                                 self.block_table.shape[1] if B else 0, max_seq_len)
+
+
+# --------------------------------------------------------------------------
+# The C ABI, one Python function per entry point
+# --------------------------------------------------------------------------
+
+def loki_cache_bytes(num_blocks, num_kv_heads, head_dim, dtype_code_):
+    return _lib.loki_cache_bytes(num_blocks, num_kv_heads, head_dim, dtype_code_)
+
+
+def loki_prefill_cache(cache, batch, k_rot, v, max_len=None, stream=None):
+    max_len = k_rot.shape[2] if max_len is None else max_len
+    _check("loki_prefill_cache", _lib.loki_prefill_cache(
+        ctypes.byref(cache.struct), ctypes.byref(batch.struct), _ptr(k_rot), _ptr(v), max_len,
+        _stream(stream)))
+
+
+def loki_append_keys(cache, batch, k_new, v_new, P, stream=None):
+    _check("loki_append_keys", _lib.loki_append_keys(
+        ctypes.byref(cache.struct), ctypes.byref(batch.struct), _ptr(k_new), _ptr(v_new), _ptr(P),
+        _stream(stream)))
+
+
+def loki_decode_workspace_bytes(cache, batch, num_q_heads, k, recent_window=0):
+    return _lib.loki_decode_workspace_bytes(ctypes.byref(cache.struct), ctypes.byref(batch.struct),
+                                            num_q_heads, k, recent_window)
+
+
+def loki_decode_attention(cache, batch, q, P, r, k, out, k_per_seq=None, recent_window=0,
+                          group_reduce=LOKI_GROUP_SUM, scale=0.0, selected_idx=None,
+                          workspace=None, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("loki_decode_attention", _lib.loki_decode_attention(
+        ctypes.byref(cache.struct), ctypes.byref(batch.struct), _ptr(q), q.shape[1], _ptr(P), r, k,
+        _ptr(k_per_seq), recent_window, group_reduce, scale, _ptr(out), _ptr(selected_idx),
+        _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def loki_decode_max_seq_len(head_dim, dtype_code_):
+    return _lib.loki_decode_max_seq_len(head_dim, dtype_code_)
+
+
+def loki_dense_workspace_bytes(cache, batch, num_q_heads):
+    return _lib.loki_dense_workspace_bytes(ctypes.byref(cache.struct), ctypes.byref(batch.struct),
+                                           num_q_heads)
+
+
+def loki_dense_attention(cache, batch, q, P, out, workspace, scale=0.0, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("loki_dense_attention", _lib.loki_dense_attention(
+        ctypes.byref(cache.struct), ctypes.byref(batch.struct), _ptr(q), q.shape[1], _ptr(P), scale,
+        _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def loki_device_error(clear=True):
+    bits = ctypes.c_uint32(0)
+    _check("loki_device_error", _lib.loki_device_error(1 if clear else 0, ctypes.byref(bits)))
+    return bits.value
+
+
+def loki_status_string(status):
+    return _lib.loki_status_string(status).decode()
+
+
+def loki_abi_version():
+    return _lib.loki_abi_version()
+
+
+def raw():
+    """The loaded ctypes library (for ABI tests)."""
+    return _lib

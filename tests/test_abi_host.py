@@ -1,0 +1,137 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point that
+include/loki.h declares, and rejects bad arguments on the host before any
+launch. No call here reaches a kernel."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from rank_key_top_b200 import build as lib_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def loki():
+    lib_build.build()
+    from rank_key_top_b200 import loki as mod
+    return mod
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "loki.h")).read()
+    return sorted(set(re.findall(r"LOKI_API\s+[\w\s\*]+?\b(loki_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_symbols()
+    for must in ("loki_append_keys", "loki_decode_attention", "loki_dense_attention",
+                 "loki_prefill_cache", "loki_status_string"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(loki):
+    lib = ctypes.CDLL(loki.LIB_PATH)
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert sorted(loki.EXPORTED) == declared_symbols()
+    assert loki.loki_abi_version() == 1
+
+
+def test_status_strings(loki):
+    for s in range(5):
+        assert loki.loki_status_string(s)
+    assert loki.loki_status_string(99) == "unknown status"
+
+
+def test_cache_bytes(loki):
+    assert loki.loki_cache_bytes(10, 8, 128, loki.LOKI_BF16) == 10 * 8 * 16 * 128 * 2
+    assert loki.loki_cache_bytes(10, 8, 64, loki.LOKI_F32) == 10 * 8 * 16 * 64 * 4
+    assert loki.loki_cache_bytes(10, 8, 96, loki.LOKI_F32) == 0
+    assert loki.loki_cache_bytes(-1, 8, 128, loki.LOKI_F32) == 0
+    assert loki.loki_decode_max_seq_len(128, loki.LOKI_BF16) == 262144
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def structs(loki, *, D=128, Hkv=8, dtype=1, B=2, max_blocks=4, max_len=64, blocks=8):
+    c = loki.loki_cache(FAKE, FAKE, blocks, Hkv, D, dtype)
+    b = loki.loki_batch(FAKE, FAKE, B, max_blocks, max_len)
+    return c, b
+
+
+def decode(loki, c, b, Hq=32, r=32, k=8, W=0, group=0, scale=0.0, q=FAKE, P=FAKE, out=FAKE):
+    return loki.raw().loki_decode_attention(ctypes.byref(c), ctypes.byref(b), q, Hq, P, r, k, None, W,
+                                            group, scale, out, None, None, 0, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(k=0, W=0), 1),            # nothing could be kept
+    (dict(k=-1), 1),
+    (dict(W=-2), 1),
+    (dict(r=0), 1),
+    (dict(r=129), 1),
+    (dict(r=40), 2),                # not a multiple of 16
+    (dict(Hq=30), 1),               # not a multiple of Hkv
+    (dict(Hq=24), 2),               # group 3
+    (dict(Hq=128), 2),              # group 16
+    (dict(group=5), 1),
+    (dict(scale=-1.0), 1),
+    (dict(scale=float("nan")), 1),
+    (dict(q=None), 1),
+    (dict(P=None), 1),
+    (dict(out=None), 1),
+    (dict(P=FAKE + 4), 1),          # P must be 16-byte aligned (bulk copy source)
+])
+def test_decode_rejects(loki, kw, status):
+    c, b = structs(loki)
+    assert decode(loki, c, b, **kw) == status
+
+
+def test_decode_rejects_bad_shapes(loki):
+    c, b = structs(loki, D=96)
+    assert decode(loki, c, b) == 2
+    c, b = structs(loki, max_len=65)       # exceeds 16 * max_blocks_per_seq
+    assert decode(loki, c, b) == 1
+    c, b = structs(loki, max_blocks=20000, max_len=300000)
+    assert decode(loki, c, b) == 2         # above the fused kernel's capacity
+    c, b = structs(loki, B=-1)
+    assert decode(loki, c, b) == 1
+    c = loki.loki_cache(FAKE + 8, FAKE, 8, 8, 128, 1)
+    _, b = structs(loki)
+    assert decode(loki, c, b) == 1         # misaligned cache
+    c = loki.loki_cache(FAKE, FAKE, 8, 8, 128, 7)
+    assert decode(loki, c, b) == 1         # unknown dtype
+    assert loki.raw().loki_decode_attention(None, ctypes.byref(b), FAKE, 32, FAKE, 32, 8, None, 0, 0, 0.0,
+                                            FAKE, None, None, 0, None) == 1
+
+
+def test_empty_batch_is_a_no_op(loki):
+    c, b = structs(loki, B=0)
+    assert decode(loki, c, b, q=None, P=None, out=None) == 0
+    assert loki.raw().loki_append_keys(ctypes.byref(c), ctypes.byref(b), None, None, None, None) == 0
+    assert loki.raw().loki_prefill_cache(ctypes.byref(c), ctypes.byref(b), None, None, 0, None) == 0
+
+
+def test_append_and_prefill_reject(loki):
+    c, b = structs(loki)
+    lib = loki.raw()
+    assert lib.loki_append_keys(ctypes.byref(c), ctypes.byref(b), None, FAKE, FAKE, None) == 1
+    assert lib.loki_append_keys(ctypes.byref(c), ctypes.byref(b), FAKE, None, FAKE, None) == 1
+    assert lib.loki_prefill_cache(ctypes.byref(c), ctypes.byref(b), FAKE, FAKE, 32, None) == 1  # max_len < max_seq_len
+    assert lib.loki_prefill_cache(ctypes.byref(c), ctypes.byref(b), FAKE + 2, FAKE, 64, None) == 1
+
+
+def test_dense_rejects(loki):
+    c, b = structs(loki)
+    lib = loki.raw()
+    need = lib.loki_dense_workspace_bytes(ctypes.byref(c), ctypes.byref(b), 32)
+    assert need > 0
+    args = lambda ws, nbytes, Hq=32: lib.loki_dense_attention(ctypes.byref(c), ctypes.byref(b), FAKE, Hq, FAKE,
+                                                               0.0, FAKE, ws, nbytes, None)
+    assert args(None, 0) == 3
+    assert args(FAKE, need - 1) == 3
+    assert args(FAKE + 16, need) == 1      # workspace must be 256-byte aligned
+    assert args(FAKE, need, Hq=24) == 2

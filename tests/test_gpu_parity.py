@@ -1,0 +1,327 @@
+"""Parity of the CUDA path (through the C ABI) with the oracle, on seeded
+synthetic inputs: small workloads in full, edge cases, and the full-size
+workloads with every (sequence, kv head) pair checked."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from rank_key_top_b200 import synth
+from tests import harness
+
+pytestmark = pytest.mark.gpu
+
+
+def spec(**kw):
+    base = dict(name="edge", batch=1, num_q_heads=4, num_kv_heads=1, head_dim=128, seq_lens=[1000],
+                dtype="bf16", alpha=0.8, r=32, k=64, seed=11)
+    base.update(kw)
+    base["batch"] = len(base["seq_lens"])
+    return synth.Spec(**base)
+
+
+def run_and_check(cuda_lib, s, pairs=None, group_max=False, **dec):
+    wl = synth.make_workload(s)
+    dev = harness.Device(wl, cuda_lib)
+    out, sel = dev.decode(group_max=group_max, **dec)
+    assert cuda_lib.loki_device_error() == 0
+    r = dec.get("r", s.r)
+    k = dec.get("k", s.k)
+    W = dec.get("W", s.recent_window)
+    errs = []
+    for b in range(s.batch):
+        for h in range(s.num_kv_heads):
+            if pairs is not None and (b, h) not in pairs:
+                continue
+            errs.append(harness.check_pair(wl, b, h, out, sel, r, k, W, group_max=group_max,
+                                           scale=dec.get("scale", 0.0)))
+    return wl, dev, out, sel, errs
+
+
+# ---------------------------------------------------------------------------
+# Small named workloads, every pair
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ["single-head-d64-L1024-f32", "mha32-d128-L4096-bf16"])
+def test_small_workloads(cuda_lib, name):
+    run_and_check(cuda_lib, synth.named_spec(name))
+
+
+# ---------------------------------------------------------------------------
+# Edge cases: ragged lengths, empty sequences, windows, k >= L, groups, dims
+# ---------------------------------------------------------------------------
+
+EDGE = {
+    "ragged-g4": dict(num_q_heads=8, num_kv_heads=2, seq_lens=[0, 1, 15, 16, 17, 100, 1000, 5000],
+                      k=50, recent_window=3),
+    "g8-d64-f32": dict(num_q_heads=16, num_kv_heads=2, head_dim=64, dtype="f32", alpha=1.0,
+                       seq_lens=[33, 2000, 7, 4096], r=16, k=7),
+    "g2-r64-window": dict(num_q_heads=4, num_kv_heads=2, seq_lens=[300, 365, 364, 4000], r=64, k=300,
+                          recent_window=64),
+    "g1-full-rank": dict(num_q_heads=3, num_kv_heads=3, seq_lens=[700, 64], r=128, k=1000),
+    "k1": dict(seq_lens=[3000, 17], k=1),
+    "window-only": dict(seq_lens=[900, 10], k=0, recent_window=20),
+    "d64-bf16-g4": dict(num_q_heads=8, num_kv_heads=2, head_dim=64, seq_lens=[2500, 1], r=48, k=40,
+                        recent_window=5),
+    "many-pairs": dict(num_q_heads=32, num_kv_heads=8, seq_lens=[1500] * 4, k=100, recent_window=16),
+}
+
+
+@pytest.mark.parametrize("case", sorted(EDGE))
+def test_edge_cases(cuda_lib, case):
+    run_and_check(cuda_lib, spec(**EDGE[case]))
+
+
+@pytest.mark.parametrize("g", [1, 4, 8])
+def test_group_max(cuda_lib, g):
+    s = spec(num_q_heads=2 * g, num_kv_heads=2, seq_lens=[2048, 777], k=100, recent_window=4)
+    run_and_check(cuda_lib, s, group_max=True)
+
+
+def test_per_sequence_k(cuda_lib):
+    s = spec(seq_lens=[4096, 1000, 33, 5000], k=600, k_per_seq=[512, 125, 4, 600])
+    run_and_check(cuda_lib, s)
+
+
+def test_explicit_scale(cuda_lib):
+    s = spec(seq_lens=[1200], k=100)
+    run_and_check(cuda_lib, s, scale=0.05)
+
+
+def test_longest_supported_sequence(cuda_lib):
+    n = cuda_lib.loki_decode_max_seq_len(128, cuda_lib.LOKI_BF16)
+    s = spec(seq_lens=[n], k=4096, recent_window=64, spare_tokens=0)
+    run_and_check(cuda_lib, s)
+
+
+# ---------------------------------------------------------------------------
+# Exact ties: integer-valued keys and queries with P = I make every score an
+# exact small integer on both sides, so the kept sets must be identical,
+# including which of the tied tokens are kept across the CTAs of a cluster.
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_exact_ties_across_cluster(cuda_lib, seed):
+    s = spec(num_q_heads=8, num_kv_heads=2, seq_lens=[6000, 3001], k=700, recent_window=7, r=16,
+             seed=20 + seed)
+    wl = synth.make_workload(s)
+    g = torch.Generator().manual_seed(seed)
+    wl.Kt = torch.randint(-2, 3, wl.Kt.shape, generator=g).to(torch.bfloat16)
+    for b, L in enumerate(s.seq_lens):
+        wl.Kt[b, :, L:] = 0
+    wl.q = torch.randint(-1, 2, wl.q.shape, generator=g).to(torch.bfloat16)
+    wl.P = torch.eye(s.head_dim).repeat(s.num_kv_heads, 1, 1).contiguous()
+    dev = harness.Device(wl, cuda_lib)
+    out, sel = dev.decode()
+    for b in range(s.batch):
+        for h in range(s.num_kv_heads):
+            Kt, V, qq, P = harness.pair_inputs(wl, b, h)
+            res = oracle.decode_pair(Kt, V, qq, P, r=s.r, k=s.k, W=s.recent_window)
+            np.testing.assert_array_equal(sel[b, h].numpy(), res.sel)
+            harness.check_pair(wl, b, h, out, sel, s.r, s.k, s.recent_window)
+
+
+def test_all_scores_equal_keeps_lowest_indices(cuda_lib):
+    s = spec(seq_lens=[5000], k=333, recent_window=10)
+    wl = synth.make_workload(s)
+    wl.Kt[:, :, :, : s.r] = 0.5
+    dev = harness.Device(wl, cuda_lib)
+    _, sel = dev.decode()
+    want = list(range(333)) + list(range(4990, 5000))
+    np.testing.assert_array_equal(sel[0, 0, :343].numpy(), want)
+
+
+# ---------------------------------------------------------------------------
+# Invariants of the CUDA path itself
+# ---------------------------------------------------------------------------
+
+def test_block_table_shuffle_is_bit_identical(cuda_lib):
+    base = dict(num_q_heads=8, num_kv_heads=2, seq_lens=[3000, 4500], k=256, recent_window=8)
+    outs = []
+    for shuffle in (False, True):
+        wl = synth.make_workload(spec(shuffle_blocks=shuffle, **base))
+        out, sel = harness.Device(wl, cuda_lib).decode()
+        outs.append((out, sel))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
+def test_full_rank_full_k_equals_dense(cuda_lib):
+    s = spec(num_q_heads=8, num_kv_heads=2, seq_lens=[3000, 129], r=128, k=3000)
+    wl = synth.make_workload(s)
+    dev = harness.Device(wl, cuda_lib)
+    out, _ = dev.decode()
+    dense = dev.dense()
+    rel = (out - dense).abs().max() / dense.abs().max()
+    assert rel < 1e-5, rel
+
+
+def test_repeat_calls_identical(cuda_lib):
+    wl = synth.make_workload(spec(seq_lens=[5000, 3333], k=300))
+    dev = harness.Device(wl, cuda_lib)
+    a = dev.decode()
+    b = dev.decode()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+# ---------------------------------------------------------------------------
+# Append (rotate the new key by P and write it into the paged cache)
+# ---------------------------------------------------------------------------
+
+def read_pair(dev, b, h, L):
+    """Reads keys and values of one pair back through the documented cache
+    layout: block p of head h at element (p * Hkv + h) * 16 * D; keys as
+    [D/16 slabs][16 tokens][16 dims], values as [16 tokens][D]."""
+    s = dev.wl.spec
+    dt = synth.torch_dtype(s.dtype)
+    D, Hkv = s.head_dim, s.num_kv_heads
+    kc = dev.cache.k.view(dt).view(-1, Hkv, D // 16, 16, 16)
+    vc = dev.cache.v.view(dt).view(-1, Hkv, 16, D)
+    tbl = dev.wl.block_table[b]
+    nblk = (L + 15) // 16
+    blocks = tbl[:nblk].long().to(kc.device)
+    K = kc[blocks, h].permute(0, 2, 1, 3).reshape(nblk * 16, D)[:L]
+    V = vc[blocks, h].reshape(nblk * 16, D)[:L]
+    return K.cpu(), V.cpu()
+
+
+def test_prefill_layout(cuda_lib):
+    s = spec(num_q_heads=4, num_kv_heads=2, seq_lens=[100, 37], head_dim=64, dtype="f32")
+    wl = synth.make_workload(s)
+    dev = harness.Device(wl, cuda_lib)
+    for b, L in enumerate(s.seq_lens):
+        for h in range(2):
+            K, V = read_pair(dev, b, h, L)
+            assert torch.equal(K, wl.Kt[b, h, :L]) and torch.equal(V, wl.V[b, h, :L])
+
+
+@pytest.mark.parametrize("dtype,D", [("bf16", 128), ("f32", 64), ("bf16", 64)])
+def test_append_matches_oracle(cuda_lib, dtype, D):
+    s = spec(num_q_heads=8, num_kv_heads=4, seq_lens=[31, 32, 100, 0], head_dim=D, dtype=dtype)
+    wl = synth.make_workload(s)
+    dev = harness.Device(wl, cuda_lib)
+    k_new, v_new = synth.draw_new_tokens(s, step=0)
+    lens = torch.tensor([n + 1 for n in s.seq_lens], dtype=torch.int32)
+    batch = cuda_lib.Batch(wl.block_table.cuda(), lens.cuda(), int(lens.max()))
+    before_k = dev.cache.k.clone()
+    cuda_lib.loki_append_keys(dev.cache, batch, k_new.cuda(), v_new.cuda(), dev.P)
+    torch.cuda.synchronize()
+    assert cuda_lib.loki_device_error() == 0
+    for b, L in enumerate(lens.tolist()):
+        for h in range(s.num_kv_heads):
+            K, V = read_pair(dev, b, h, L)
+            assert torch.equal(V[L - 1], v_new[b, h])
+            if L > 1:
+                assert torch.equal(K[: L - 1], wl.Kt[b, h, : L - 1])
+            kk = k_new[b, h].double().numpy()[None]
+            Ph = wl.P[h].double().numpy()
+            want = oracle.append(kk, Ph, dtype)[0]
+            got = K[L - 1].double().numpy()
+            exact = oracle.rotate(kk, Ph)[0]
+            bound = D * 2.0 ** -24 * (np.abs(kk[0][:, None] * Ph)).sum(axis=0)
+            mism = got != want
+            # a mismatch is allowed only where the exact value is within the
+            # fp32 accumulation bound of the rounding midpoint of the two
+            assert np.all(np.abs(exact[mism] - (got[mism] + want[mism]) / 2) <= bound[mism]), (b, h)
+    assert not torch.equal(before_k, dev.cache.k)
+
+
+def test_append_then_decode(cuda_lib):
+    """One whole decode step: append the current token, then attend."""
+    s = spec(num_q_heads=8, num_kv_heads=2, seq_lens=[1999, 3000], k=200, recent_window=4)
+    wl = synth.make_workload(s)
+    dev = harness.Device(wl, cuda_lib)
+    k_new, v_new = synth.draw_new_tokens(s, step=3)
+    lens = [n + 1 for n in s.seq_lens]
+    dev.batch = cuda_lib.Batch(wl.block_table.cuda(), torch.tensor(lens, dtype=torch.int32).cuda(), max(lens))
+    cuda_lib.loki_append_keys(dev.cache, dev.batch, k_new.cuda(), v_new.cuda(), dev.P)
+    out, sel = dev.decode()
+    # the oracle's own view of the cache after the append
+    Kt = torch.zeros(s.batch, s.num_kv_heads, max(lens), s.head_dim, dtype=torch.bfloat16)
+    V = torch.zeros_like(Kt)
+    for b, n in enumerate(s.seq_lens):
+        Kt[b, :, :n] = wl.Kt[b, :, :n]
+        V[b, :, :n] = wl.V[b, :, :n]
+        for h in range(s.num_kv_heads):
+            kk = k_new[b, h].double().numpy()[None]
+            Kt[b, h, n] = torch.from_numpy(oracle.append(kk, wl.P[h].double().numpy(), "bf16")[0]).to(torch.bfloat16)
+            V[b, h, n] = v_new[b, h]
+    wl.Kt, wl.V = Kt, V
+    wl.spec.seq_lens = lens
+    for b in range(s.batch):
+        for h in range(s.num_kv_heads):
+            harness.check_pair(wl, b, h, out, sel, s.r, s.k, s.recent_window)
+
+
+def test_device_checks_flag_bad_lengths_and_blocks(cuda_lib):
+    s = spec(num_q_heads=4, num_kv_heads=1, seq_lens=[500, 600], k=20)
+    wl = synth.make_workload(s)
+    dev = harness.Device(wl, cuda_lib)
+    cuda_lib.loki_device_error(clear=True)
+    bad_lens = torch.tensor([500, 9999], dtype=torch.int32).cuda()   # above max_seq_len
+    dev.batch = cuda_lib.Batch(wl.block_table.cuda(), bad_lens, 600)
+    dev.decode()
+    assert cuda_lib.loki_device_error(clear=True) & cuda_lib.LOKI_DEVERR_SEQ_LEN
+    tbl = wl.block_table.clone()
+    tbl[0, 3] = wl.num_blocks + 5                                    # out of range
+    dev.batch = cuda_lib.Batch(tbl.cuda(), wl.seq_lens.cuda(), 600)
+    dev.decode()
+    assert cuda_lib.loki_device_error(clear=True) & cuda_lib.LOKI_DEVERR_BLOCK_ID
+    kps = torch.tensor([5, 50], dtype=torch.int32).cuda()            # above k
+    dev.batch = cuda_lib.Batch(wl.block_table.cuda(), wl.seq_lens.cuda(), 600)
+    dev.k_per_seq = kps
+    dev.decode()
+    assert cuda_lib.loki_device_error(clear=True) & cuda_lib.LOKI_DEVERR_K
+
+
+# ---------------------------------------------------------------------------
+# Dense comparison path
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ["single-head-d64-L1024-f32", "mha32-d128-L4096-bf16"])
+def test_dense_small(cuda_lib, name):
+    s = synth.named_spec(name)
+    wl = synth.make_workload(s)
+    out = harness.Device(wl, cuda_lib).dense()
+    for b in range(s.batch):
+        for h in range(s.num_kv_heads):
+            harness.check_dense_pair(wl, b, h, out)
+
+
+def test_dense_edge(cuda_lib):
+    s = spec(num_q_heads=16, num_kv_heads=2, seq_lens=[0, 1, 513, 2049], head_dim=64, k=5)
+    wl = synth.make_workload(s)
+    out = harness.Device(wl, cuda_lib).dense()
+    assert torch.all(out[0] == 0)
+    for b in range(1, s.batch):
+        for h in range(s.num_kv_heads):
+            harness.check_dense_pair(wl, b, h, out)
+
+
+# ---------------------------------------------------------------------------
+# Full-size workloads, every pair
+# ---------------------------------------------------------------------------
+
+def test_paged_batched_workload(cuda_lib):
+    run_and_check(cuda_lib, synth.named_spec("paged-b16-mha32-L4k-16k-bf16"))
+
+
+def test_gqa_32k_workload(cuda_lib):
+    s = synth.named_spec("gqa32x8-d128-L32768-bf16")
+    wl, dev, out, sel, errs = run_and_check(cuda_lib, s)
+    dense = dev.dense()
+    for b, h in [(0, 0), (3, 5), (7, 7)]:
+        harness.check_dense_pair(wl, b, h, dense)
+
+
+def test_long_context_outliers_sweep(cuda_lib):
+    s = synth.named_spec("gqa32x8-d128-L131072-bf16-outliers")
+    wl = synth.make_workload(s)
+    dev = harness.Device(wl, cuda_lib)
+    L = s.seq_lens[0]
+    combos = [(r, L // div) for r in (16, 32, 64) for div in (32, 16, 8)]
+    results = {c: dev.decode(r=c[0], k=c[1]) for c in combos}
+    for b in range(s.batch):
+        for h in range(s.num_kv_heads):
+            inputs = harness.pair_inputs(wl, b, h)
+            for (r, k), (out, sel) in results.items():
+                harness.check_pair(wl, b, h, out, sel, r, k, 0, inputs=inputs)
