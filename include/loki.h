@@ -46,7 +46,7 @@ extern "C" {
 #define LOKI_API
 #endif
 
-#define LOKI_ABI_VERSION 1
+#define LOKI_ABI_VERSION 2
 #define LOKI_BLOCK_TOKENS 16 /* tokens per paged-cache block */
 
 typedef void* loki_stream_t; /* a cudaStream_t */
@@ -81,18 +81,25 @@ typedef enum loki_group_reduce {
 #define LOKI_DEVERR_TIMEOUT 0x8u  /* a bounded wait on an async copy gave up */
 
 /* Paged KV cache in the library's own layout (LOKI_BLOCK_TOKENS tokens per
- * block). Physical block p of kv head h holds:
- *   keys   (PCA basis): [head_dim/16 slabs][16 tokens][16 dims]
- *   values            : [16 tokens][head_dim]
- * at element offset ((p * num_kv_heads + h) * 16 * head_dim). The slab layout
- * makes the leading r dimensions of a block one contiguous run of r*16
- * elements, which is what rank-r scoring streams. */
+ * block), plus a low-rank key index. Physical block p of kv head h holds:
+ *   keys (PCA basis)  [16 tokens][head_dim]  at element (p*Hkv + h)*16*head_dim
+ *   values            [16 tokens][head_dim]  at element (p*Hkv + h)*16*head_dim
+ *   key index         [index_dims/16 slabs][16 tokens][16 dims]
+ *                                            at element (p*Hkv + h)*16*index_dims
+ * The key index repeats the leading index_dims rotated dims of every key. Its
+ * slab layout makes the leading r <= index_dims dims of a block one
+ * contiguous run of r*16 elements, which is what rank-r scoring streams; the
+ * key rows stay whole (one contiguous row per token) for the exact attention
+ * over the kept tokens. The index costs index_dims/head_dim of the key cache
+ * (12.5% of keys + values for index_dims = 32, head_dim = 128). */
 typedef struct loki_cache {
     void* k_cache;         /* device, loki_cache_bytes(), 16-byte aligned */
     void* v_cache;         /* device, loki_cache_bytes(), 16-byte aligned */
+    void* k_index;         /* device, loki_index_bytes(), 16-byte aligned */
     int32_t num_blocks;    /* physical blocks in each cache */
     int32_t num_kv_heads;  /* >= 1 */
     int32_t head_dim;      /* 64 or 128 */
+    int32_t index_dims;    /* multiple of 16 in [16, head_dim]; the largest usable r */
     loki_dtype dtype;
 } loki_cache;
 
@@ -111,9 +118,14 @@ typedef struct loki_batch {
 /* Bytes of EACH of k_cache and v_cache for the given shape; 0 for an invalid
  * shape. */
 LOKI_API size_t loki_cache_bytes(int32_t num_blocks, int32_t num_kv_heads, int32_t head_dim,
-                        loki_dtype dtype);
+                                 loki_dtype dtype);
 
-/* Prefill: write tokens [0, seq_lens[b]) of every sequence into the cache.
+/* Bytes of k_index for the given shape; 0 for an invalid shape. */
+LOKI_API size_t loki_index_bytes(int32_t num_blocks, int32_t num_kv_heads, int32_t index_dims,
+                                 loki_dtype dtype);
+
+/* Prefill: write tokens [0, seq_lens[b]) of every sequence into the cache
+ * (key rows, value rows and the key index).
  *
  * k_rot, v: device [batch][num_kv_heads][max_len][head_dim] in the cache type,
  * row-major, 16-byte aligned; max_len >= max_seq_len. The keys must already be
@@ -127,7 +139,8 @@ LOKI_API loki_status loki_prefill_cache(const loki_cache* cache, const loki_batc
 /* Cache update of one decode step (AQUA page, decode-step equations (1)-(2),
  * for keys kept in the PCA basis): for every sequence b and kv head h,
  *   K~[b, h, seq_lens[b]-1, :] = round(k_new[b, h, :] P[h])   (fp32 accumulation,
- *                                round-to-nearest-even to the cache type)
+ *                                round-to-nearest-even to the cache type),
+ *                                its leading index_dims also into the key index
  *   V [b, h, seq_lens[b]-1, :] = v_new[b, h, :]
  * so seq_lens must already count the new token. Sequences with seq_lens[b] = 0
  * are skipped.
@@ -156,9 +169,11 @@ LOKI_API size_t loki_decode_workspace_bytes(const loki_cache* cache, const loki_
  *   4. out_j = softmax over the kept set of (q_hat_j . K~[t, :] * scale) times V
  *      (AQUA page, decode-step equations (3)-(5)), fp32.
  *
- * q: device [batch][num_q_heads][head_dim] in the cache type, unrotated.
+ * q: device [batch][num_q_heads][head_dim] in the cache type, unrotated,
+ *    16-byte aligned.
  * P: device fp32 [num_kv_heads][head_dim][head_dim], 16-byte aligned.
- * r: leading dimensions used for scoring; a multiple of 16 in [16, head_dim].
+ * r: leading dimensions used for scoring; a multiple of 16 in [16, index_dims]
+ *    (r > index_dims is LOKI_ERR_INVALID_ARG).
  * k: tokens kept by score (the per-sequence maximum when k_per_seq is given).
  * k_per_seq: nullable device int32 [batch]; entries clamped to [0, k].
  * recent_window: W >= 0; k = 0 together with W = 0 is invalid.

@@ -7,24 +7,25 @@
 //
 // Work split inside a warp: lane l owns head dimensions [l*DPL, l*DPL + DPL)
 // (DPL = D / 32) of every token's key row and value row, so a token costs one
-// 8-byte (bf16, D = 128) load of its key piece and one of its value piece per
-// lane. A chunk of NCH tokens gives each lane NCH * G partial dot products,
-// which one transpose-reduce sums across the warp.
+// 8-byte (bf16, D = 128) read of its key piece and one of its value piece per
+// lane (from global memory or from a shared-memory staging copy). A chunk of
+// NCH tokens gives each lane NCH * G partial dot products, which one
+// transpose-reduce sums across the warp.
 #pragma once
 
 #include "common.cuh"
 
 namespace loki {
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, int NCH_ = ((G >= 8) ? 4 : 8)>
 struct AttnCore {
     static constexpr int DPL = D / 32;
-    static constexpr int NCH = (G >= 8) ? 4 : 8;       // tokens per chunk
+    static constexpr int NCH = NCH_;                   // tokens per chunk
     static constexpr int NV = NCH * G;                 // values per transpose-reduce
-    static constexpr int LOG_NV = NV == 8 ? 3 : (NV == 16 ? 4 : 5);
+    static constexpr int LOG_NV = NV == 2 ? 1 : NV == 4 ? 2 : NV == 8 ? 3 : NV == 16 ? 4 : 5;
     static constexpr int LOG_G = G == 1 ? 0 : (G == 2 ? 1 : (G == 4 ? 2 : 3));
     static constexpr int SH = 5 - LOG_NV;              // lane >> SH = value index
-    static_assert(NV == 8 || NV == 16 || NV == 32, "chunk geometry");
+    static_assert(NV >= 2 && NV <= 32 && (NV & (NV - 1)) == 0, "chunk geometry");
     using V = Vec<T, DPL>;
     using raw_t = typename V::raw_t;
 
@@ -47,10 +48,10 @@ struct AttnCore {
 
     // Address of this lane's key piece / value piece of `row` in a block.
     static __device__ __forceinline__ const T* key_ptr(const T* kc, int64_t page, int row, int lane) {
-        return kc + page + key_offset_in_page(row, lane * DPL);
+        return kc + page + row_offset_in_page(row, lane * DPL, D);
     }
     static __device__ __forceinline__ const T* val_ptr(const T* vc, int64_t page, int row, int lane) {
-        return vc + page + value_offset_in_page(row, lane * DPL, D);
+        return vc + page + row_offset_in_page(row, lane * DPL, D);
     }
 
     static __device__ __forceinline__ raw_t zero_raw() {

@@ -1,7 +1,9 @@
 // Cache writers: bulk prefill of keys already in the PCA basis, and the
 // per-step append that rotates the new key by P (AQUA page, decode-step
 // equations (1)-(2): the current token's key and value join the cache before
-// scoring; AQUA page, appendix step 1: the key is projected with P).
+// scoring; AQUA page, appendix on complexity, step 1: the key is projected
+// with P). Both write the key row, the value row and the key's leading
+// index dims into the low-rank key index.
 #pragma once
 
 #include "common.cuh"
@@ -11,15 +13,16 @@ namespace loki {
 struct PrefillParams {
     void* k_cache;
     void* v_cache;
+    void* k_index;
     const int32_t* block_table;
     const int32_t* seq_lens;
     const void* k_rot;
     const void* v;
-    int num_blocks, Hkv, max_blocks, max_seq_len, max_len;
+    int num_blocks, Hkv, max_blocks, max_seq_len, max_len, index_dims;
 };
 
 // grid (max_blocks, batch * Hkv); one CTA writes one 16-token block of one
-// kv head; 16-byte vectors of 16 / sizeof(T) dims, all inside one key slab.
+// kv head with 16-byte vectors (16 / sizeof(T) dims, inside one index slab).
 template <typename T, int D>
 __global__ void __launch_bounds__(256) prefill_kernel(const PrefillParams p) {
     constexpr int VEC = 16 / sizeof(T);
@@ -38,11 +41,13 @@ __global__ void __launch_bounds__(256) prefill_kernel(const PrefillParams p) {
         return;
     }
     const int64_t page = page_offset(pb, h, p.Hkv, D);
+    const int64_t ipage = page_offset(pb, h, p.Hkv, p.index_dims);
     const int64_t src_row0 = (((int64_t)b * p.Hkv + h) * p.max_len + (int64_t)jb * kBlockTokens) * D;
     const T* ks = reinterpret_cast<const T*>(p.k_rot) + src_row0;
     const T* vs = reinterpret_cast<const T*>(p.v) + src_row0;
     T* kd = reinterpret_cast<T*>(p.k_cache) + page;
     T* vd = reinterpret_cast<T*>(p.v_cache) + page;
+    T* xd = reinterpret_cast<T*>(p.k_index) + ipage;
     constexpr int per_tok = D / VEC;
     for (int i = threadIdx.x; i < kBlockTokens * per_tok; i += blockDim.x) {
         const int tok = i / per_tok;
@@ -50,60 +55,93 @@ __global__ void __launch_bounds__(256) prefill_kernel(const PrefillParams p) {
         if (jb * kBlockTokens + tok >= L) continue;
         const uint4 kv = *reinterpret_cast<const uint4*>(ks + tok * D + dim);
         const uint4 vv = *reinterpret_cast<const uint4*>(vs + tok * D + dim);
-        *reinterpret_cast<uint4*>(kd + key_offset_in_page(tok, dim)) = kv;
-        *reinterpret_cast<uint4*>(vd + value_offset_in_page(tok, dim, D)) = vv;
+        *reinterpret_cast<uint4*>(kd + row_offset_in_page(tok, dim, D)) = kv;
+        *reinterpret_cast<uint4*>(vd + row_offset_in_page(tok, dim, D)) = vv;
+        if (dim < p.index_dims) *reinterpret_cast<uint4*>(xd + index_offset_in_page(tok, dim)) = kv;
     }
 }
 
 struct AppendParams {
     void* k_cache;
     void* v_cache;
+    void* k_index;
     const int32_t* block_table;
     const int32_t* seq_lens;
     const void* k_new;
     const void* v_new;
     const float* P;  // nullable
-    int num_blocks, Hkv, max_blocks, max_seq_len;
+    int num_blocks, Hkv, max_blocks, max_seq_len, index_dims;
 };
 
-// grid (batch * Hkv), D threads. Thread c computes rotated dim c as an fp32
-// chain over i = 0 .. D-1 of k[i] * P[i][c], then rounds to nearest even.
+// grid (batch * Hkv), 256 threads. k_tilde[c] = sum_i k[i] P[i][c] in fp32:
+// thread (row group rg, column quad cq) sums its D/8 rows for 4 columns from
+// one round of independent 16-byte loads of P; the 8 row groups' partial sums
+// are added in shared memory; the result is rounded to nearest even.
 template <typename T, int D>
-__global__ void __launch_bounds__(D) append_kernel(const AppendParams p) {
+__global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
+    constexpr int NQ = D / 4;         // column quads
+    constexpr int NRG = 256 / NQ;     // row groups (8 for D = 128, 16 for D = 64)
+    constexpr int RPG = D / NRG;      // rows per group
+    __shared__ float part[NRG][D];
     __shared__ float kin[D];
     const int pair = blockIdx.x;
     const int b = pair / p.Hkv, h = pair - b * p.Hkv;
-    const int c = threadIdx.x;
+    const int tid = threadIdx.x;
     int L = p.seq_lens[b];
     if (L < 0 || L > p.max_seq_len) {
-        if (c == 0) flag_error(LOKI_DEVERR_SEQ_LEN);
+        if (tid == 0) flag_error(LOKI_DEVERR_SEQ_LEN);
         return;
     }
     if (L == 0) return;
     const int pos = L - 1;
     int pb = p.block_table[(int64_t)b * p.max_blocks + pos / kBlockTokens];
     if (pb < 0 || pb >= p.num_blocks) {
-        if (c == 0) flag_error(LOKI_DEVERR_BLOCK_ID);
+        if (tid == 0) flag_error(LOKI_DEVERR_BLOCK_ID);
         return;
     }
     const int row = pos % kBlockTokens;
     const int64_t src = ((int64_t)b * p.Hkv + h) * D;
-    kin[c] = Elem<T>::to_f(reinterpret_cast<const T*>(p.k_new)[src + c]);
-    __syncthreads();
-    float x;
+    const int cq = tid % NQ, rg = tid / NQ;
+    float4 pv[RPG];
     if (p.P) {
         const float* Ph = p.P + (int64_t)h * D * D;
-        float a = 0.f;
-#pragma unroll 16
-        for (int i = 0; i < D; ++i) a = fmaf(kin[i], Ph[i * D + c], a);
-        x = a;
-    } else {
-        x = kin[c];
+#pragma unroll
+        for (int i = 0; i < RPG; ++i) pv[i] = *reinterpret_cast<const float4*>(Ph + (rg * RPG + i) * D + 4 * cq);
     }
-    const int64_t page = page_offset(pb, h, p.Hkv, D);
-    reinterpret_cast<T*>(p.k_cache)[page + key_offset_in_page(row, c)] = Elem<T>::from_f(x);
-    reinterpret_cast<T*>(p.v_cache)[page + value_offset_in_page(row, c, D)] =
-        reinterpret_cast<const T*>(p.v_new)[src + c];
+    if (tid < D) kin[tid] = Elem<T>::to_f(reinterpret_cast<const T*>(p.k_new)[src + tid]);
+    __syncthreads();
+    if (p.P) {
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+        for (int i = 0; i < RPG; ++i) {
+            const float x = kin[rg * RPG + i];
+            a0 = fmaf(x, pv[i].x, a0);
+            a1 = fmaf(x, pv[i].y, a1);
+            a2 = fmaf(x, pv[i].z, a2);
+            a3 = fmaf(x, pv[i].w, a3);
+        }
+        *reinterpret_cast<float4*>(&part[rg][4 * cq]) = make_float4(a0, a1, a2, a3);
+    }
+    __syncthreads();
+    if (tid < D) {
+        const int c = tid;
+        float x;
+        if (p.P) {
+            x = 0.f;
+#pragma unroll
+            for (int g = 0; g < NRG; ++g) x += part[g][c];
+        } else {
+            x = kin[c];
+        }
+        const T kt = Elem<T>::from_f(x);
+        const int64_t page = page_offset(pb, h, p.Hkv, D);
+        reinterpret_cast<T*>(p.k_cache)[page + row_offset_in_page(row, c, D)] = kt;
+        if (c < p.index_dims)
+            reinterpret_cast<T*>(p.k_index)[page_offset(pb, h, p.Hkv, p.index_dims) + index_offset_in_page(row, c)] =
+                kt;
+        reinterpret_cast<T*>(p.v_cache)[page + row_offset_in_page(row, c, D)] =
+            reinterpret_cast<const T*>(p.v_new)[src + c];
+    }
 }
 
 }  // namespace loki

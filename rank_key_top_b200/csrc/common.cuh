@@ -8,7 +8,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/loki.h"
+#include "loki.h"
 
 namespace loki {
 
@@ -22,18 +22,20 @@ __device__ __forceinline__ void flag_error(uint32_t bits) { atomicOr(&g_device_e
 
 // ---------------------------------------------------------------------------
 // Paged cache layout. Block p of kv head h starts at element
-// (p * Hkv + h) * 16 * D in both caches.
-//   keys:   [D/16 slabs][16 tokens][16 dims]
-//   values: [16 tokens][D]
+// (p * Hkv + h) * 16 * D in the key and value caches, and at
+// (p * Hkv + h) * 16 * I in the key index (I = index dims).
+//   keys, values: [16 tokens][D]                 (one contiguous row per token)
+//   key index:    [I/16 slabs][16 tokens][16 dims] (the leading r dims of all
+//                 16 tokens are one contiguous run of r*16 elements)
 // ---------------------------------------------------------------------------
 __host__ __device__ __forceinline__ int64_t page_offset(int64_t block, int h, int Hkv, int D) {
     return (block * Hkv + h) * (int64_t)(kBlockTokens * D);
 }
-__host__ __device__ __forceinline__ int key_offset_in_page(int token, int dim) {
-    return (dim / kSlabDims) * (kBlockTokens * kSlabDims) + token * kSlabDims + (dim % kSlabDims);
-}
-__host__ __device__ __forceinline__ int value_offset_in_page(int token, int dim, int D) {
+__host__ __device__ __forceinline__ int row_offset_in_page(int token, int dim, int D) {
     return token * D + dim;
+}
+__host__ __device__ __forceinline__ int index_offset_in_page(int token, int dim) {
+    return (dim / kSlabDims) * (kBlockTokens * kSlabDims) + token * kSlabDims + (dim % kSlabDims);
 }
 
 // ---------------------------------------------------------------------------

@@ -28,8 +28,10 @@ loki_status check_cache(const loki_cache* c) {
     if (c->dtype != LOKI_F32 && c->dtype != LOKI_BF16) return LOKI_ERR_INVALID_ARG;
     if (c->num_blocks < 0 || c->num_kv_heads < 1 || c->head_dim < 1) return LOKI_ERR_INVALID_ARG;
     if (c->head_dim != 64 && c->head_dim != 128) return LOKI_ERR_UNSUPPORTED;
-    if (c->num_blocks > 0 && (!c->k_cache || !c->v_cache)) return LOKI_ERR_INVALID_ARG;
-    if (!aligned16(c->k_cache) || !aligned16(c->v_cache)) return LOKI_ERR_INVALID_ARG;
+    if (c->index_dims < kSlabDims || c->index_dims > c->head_dim || c->index_dims % kSlabDims != 0)
+        return LOKI_ERR_INVALID_ARG;
+    if (c->num_blocks > 0 && (!c->k_cache || !c->v_cache || !c->k_index)) return LOKI_ERR_INVALID_ARG;
+    if (!aligned16(c->k_cache) || !aligned16(c->v_cache) || !aligned16(c->k_index)) return LOKI_ERR_INVALID_ARG;
     return LOKI_OK;
 }
 
@@ -92,36 +94,6 @@ DeviceInfo device_info() {
     return di;
 }
 
-void sparse_layout(SparseParams& p, int D, int G, size_t esize) {
-    auto align = [](int x) { return (x + 127) & ~127; };
-    int off = 0;
-    p.off_keys = off;
-    off = align(off + std::max(p.cta_tokens * 4, D * D * 4));
-    p.off_ring = off;
-    off = align(off + kWarps * kRingBytesPerWarp);
-    p.off_list = off;
-    off = align(off + p.cta_tokens * 2);
-    p.off_qf = off;
-    off = align(off + G * D * 4);
-    p.off_qhat = off;
-    off = align(off + G * D * 4);
-    p.off_qs = off;
-    off = align(off + D * 4);
-    p.off_tbl = off;
-    off = align(off + (p.cta_tokens / kBlockTokens) * 4);
-    p.off_hist = off;
-    off = align(off + 2 * kHistBins * 4);
-    p.off_bars = off;
-    off = align(off + (kWarps * kMaxSlots + 1) * 8);
-    p.off_part = off;
-    off = align(off + G * (D + 2) * 4);
-    p.off_misc = off;
-    off = align(off + 64 * 4);
-    p.smem_bytes = off;
-    p.slot_bytes = p.r * kBlockTokens * (int)esize;
-    p.slots = std::min(kMaxSlots, std::max(1, kRingBytesPerWarp / p.slot_bytes));
-}
-
 // Whether at least one cluster of this shape can be resident on the device,
 // cached per kernel instantiation, cluster size and shared-memory size.
 template <typename K>
@@ -141,14 +113,97 @@ bool cluster_fits(K kern, const cudaLaunchConfig_t& cfg, std::map<std::pair<int,
     return fits;
 }
 
+// Shared-memory layout of one CTA for C CTAs per (sequence, kv head), with a
+// key-index ring of ring_per_warp bytes per warp.
+template <typename T, int D, int G>
+void sparse_layout(SparseParams& p, int max_seq_len, int ring_per_warp) {
+    using Geom = SparseGeom<T, D, G>;
+    auto align = [](int x) { return (x + 127) & ~127; };
+    const int nblk = (max_seq_len + kBlockTokens - 1) / kBlockTokens;
+    p.cta_tokens = std::max(1, (nblk + p.C - 1) / p.C) * kBlockTokens;
+    p.slot_bytes = p.r * kBlockTokens * (int)sizeof(T);
+    p.slots = std::min(kMaxSlots, std::max(1, ring_per_warp / p.slot_bytes));
+    p.ring_bytes_per_warp = p.slots * p.slot_bytes;
+    const int list_bytes = align(p.cta_tokens * 2);
+    int ring_bytes = align(kWarps * p.ring_bytes_per_warp);
+    if (ring_bytes < list_bytes + 8 * 1024) ring_bytes = list_bytes + 8 * 1024;
+    p.cand_cap = (ring_bytes - list_bytes) / 8;
+    int keys_bytes = align(std::max(p.cta_tokens * 4, Geom::QSCRATCH_BYTES));
+    // the gather stages rows in keys + ring minus the list; the warp partials
+    // of the merge go to keys + ring
+    const int staged = std::max(Geom::STAGE_BYTES + list_bytes, Geom::WPART_BYTES);
+    if (keys_bytes + ring_bytes < staged) keys_bytes = align(staged - ring_bytes);
+    int off = 0;
+    p.off_keys = off;
+    p.keys_bytes = keys_bytes;
+    off += keys_bytes;
+    p.off_ring = off;
+    p.ring_bytes = ring_bytes;
+    off += ring_bytes;
+    p.off_list = p.off_ring + ring_bytes - list_bytes;
+    p.off_qf = off;  // merge weights
+    off = align(off + G * kWarps * 4);
+    p.off_qhat = off;
+    off = align(off + G * D * 4);
+    p.off_qs = off;
+    off = align(off + D * 4);
+    p.off_tbl = off;
+    off = align(off + (p.cta_tokens / kBlockTokens) * 4);
+    p.off_hist = off;
+    off = align(off + 2 * kHistBins * 4);
+    p.off_bars = off;
+    off = align(off + kWarps * kMaxSlots * 8);
+    p.off_part = off;
+    off = align(off + G * (D + 2) * 4);
+    p.off_misc = off;
+    off = align(off + 128 * 4);
+    p.smem_bytes = off;
+}
+
+// The layout with the deepest key-index ring that fits in shared memory.
+template <typename T, int D, int G>
+bool sparse_layout_fit(SparseParams& p, int max_seq_len, int smem_optin) {
+    for (int ring_per_warp : {8192, 6144, 4096, 2048}) {
+        sparse_layout<T, D, G>(p, max_seq_len, ring_per_warp);
+        if (p.smem_bytes <= smem_optin) return true;
+    }
+    return false;
+}
+
+// Cluster size: enough CTAs that each holds at most kCtaTokenCap tokens and
+// the layout fits in shared memory, then as many as still fit every cluster
+// on the GPU at once (one CTA per SM), keeping at least 512 tokens per CTA.
+template <typename T, int D, int G>
+int choose_cluster(SparseParams& p, int max_seq_len, int pairs, int sms, int smem_optin) {
+    const int nblk = (max_seq_len + kBlockTokens - 1) / kBlockTokens;
+    const int cap_blocks = kCtaTokenCap / kBlockTokens;
+    int C = std::max(1, (nblk + cap_blocks - 1) / cap_blocks);
+    for (;; ++C) {
+        if (C > 16) return -1;
+        p.C = C;
+        if (sparse_layout_fit<T, D, G>(p, max_seq_len, smem_optin)) break;
+    }
+    for (int cand = C + 1; cand <= 16; ++cand) {
+        if ((int64_t)pairs * cand > sms) break;
+        if (nblk / cand < 32) break;
+        C = cand;
+    }
+    p.C = C;
+    sparse_layout_fit<T, D, G>(p, max_seq_len, smem_optin);
+    return C;
+}
+
 template <typename T, int D, int G>
 struct SparseLaunch {
-    static loki_status run(SparseParams p, int pairs, cudaStream_t stream) {
+    static loki_status run(SparseParams p, int pairs, int max_seq_len, const DeviceInfo& di,
+                           cudaStream_t stream) {
+        if (choose_cluster<T, D, G>(p, max_seq_len, pairs, di.sms, di.max_smem_optin) < 1)
+            return LOKI_ERR_UNSUPPORTED;
         auto kern = sparse_decode_kernel<T, D, G>;
         static std::once_flag once;
         static cudaError_t attr_err = cudaSuccess;
         std::call_once(once, [&] {
-            attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+            attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, di.max_smem_optin);
             if (attr_err == cudaSuccess)
                 attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         });
@@ -174,22 +229,6 @@ struct SparseLaunch {
     }
 };
 
-// Cluster size: enough CTAs that each holds at most kCtaTokenCap tokens, then
-// as many as still fit every cluster on the GPU at once (one CTA per SM),
-// keeping at least 512 tokens per CTA.
-int choose_cluster(int max_seq_len, int pairs, int sms) {
-    const int nblk = (max_seq_len + kBlockTokens - 1) / kBlockTokens;
-    const int cap_blocks = kCtaTokenCap / kBlockTokens;
-    int C = std::max(1, (nblk + cap_blocks - 1) / cap_blocks);
-    if (C > 16) return -1;
-    for (int cand = C + 1; cand <= 16; ++cand) {
-        if ((int64_t)pairs * cand > sms) break;
-        if (nblk / cand < 32) break;
-        C = cand;
-    }
-    return C;
-}
-
 }  // namespace
 
 extern "C" {
@@ -198,6 +237,14 @@ size_t loki_cache_bytes(int32_t num_blocks, int32_t num_kv_heads, int32_t head_d
     if (num_blocks < 0 || num_kv_heads < 1 || (head_dim != 64 && head_dim != 128)) return 0;
     if (dtype != LOKI_F32 && dtype != LOKI_BF16) return 0;
     return (size_t)num_blocks * num_kv_heads * kBlockTokens * head_dim * elem_size(dtype);
+}
+
+size_t loki_index_bytes(int32_t num_blocks, int32_t num_kv_heads, int32_t index_dims, loki_dtype dtype) {
+    if (num_blocks < 0 || num_kv_heads < 1 || index_dims < kSlabDims || index_dims > 128 ||
+        index_dims % kSlabDims != 0)
+        return 0;
+    if (dtype != LOKI_F32 && dtype != LOKI_BF16) return 0;
+    return (size_t)num_blocks * num_kv_heads * kBlockTokens * index_dims * elem_size(dtype);
 }
 
 int32_t loki_abi_version(void) { return LOKI_ABI_VERSION; }
@@ -236,6 +283,8 @@ loki_status loki_prefill_cache(const loki_cache* cache, const loki_batch* batch,
     PrefillParams p;
     p.k_cache = cache->k_cache;
     p.v_cache = cache->v_cache;
+    p.k_index = cache->k_index;
+    p.index_dims = cache->index_dims;
     p.block_table = batch->block_table;
     p.seq_lens = batch->seq_lens;
     p.k_rot = k_rot;
@@ -267,10 +316,13 @@ loki_status loki_append_keys(const loki_cache* cache, const loki_batch* batch, c
     if ((st = check_batch(batch)) != LOKI_OK) return st;
     if (batch->batch == 0) return LOKI_OK;
     if (!k_new || !v_new) return LOKI_ERR_INVALID_ARG;
+    if (P && !aligned16(P)) return LOKI_ERR_INVALID_ARG;
     if ((int64_t)batch->batch * cache->num_kv_heads > INT32_MAX / 2) return LOKI_ERR_UNSUPPORTED;
     AppendParams p;
     p.k_cache = cache->k_cache;
     p.v_cache = cache->v_cache;
+    p.k_index = cache->k_index;
+    p.index_dims = cache->index_dims;
     p.block_table = batch->block_table;
     p.seq_lens = batch->seq_lens;
     p.k_new = k_new;
@@ -284,11 +336,11 @@ loki_status loki_append_keys(const loki_cache* cache, const loki_batch* batch, c
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int D = cache->head_dim;
     if (cache->dtype == LOKI_BF16) {
-        if (D == 64) append_kernel<__nv_bfloat16, 64><<<grid, 64, 0, s>>>(p);
-        else append_kernel<__nv_bfloat16, 128><<<grid, 128, 0, s>>>(p);
+        if (D == 64) append_kernel<__nv_bfloat16, 64><<<grid, 256, 0, s>>>(p);
+        else append_kernel<__nv_bfloat16, 128><<<grid, 256, 0, s>>>(p);
     } else {
-        if (D == 64) append_kernel<float, 64><<<grid, 64, 0, s>>>(p);
-        else append_kernel<float, 128><<<grid, 128, 0, s>>>(p);
+        if (D == 64) append_kernel<float, 64><<<grid, 256, 0, s>>>(p);
+        else append_kernel<float, 128><<<grid, 256, 0, s>>>(p);
     }
     return launch_status();
 }
@@ -329,20 +381,20 @@ loki_status loki_decode_attention(const loki_cache* cache, const loki_batch* bat
     if ((int64_t)k + recent_window > INT32_MAX / 2) return LOKI_ERR_INVALID_ARG;
     if (batch->batch == 0) return LOKI_OK;
     if (!q || !P || !out) return LOKI_ERR_INVALID_ARG;
-    if (!aligned16(P)) return LOKI_ERR_INVALID_ARG;
+    if (!aligned16(P) || !aligned16(q)) return LOKI_ERR_INVALID_ARG;
     const int G = num_q_heads / Hkv;
     if (G != 1 && G != 2 && G != 4 && G != 8) return LOKI_ERR_UNSUPPORTED;
     if (r % kSlabDims != 0) return LOKI_ERR_UNSUPPORTED;
+    if (r > cache->index_dims) return LOKI_ERR_INVALID_ARG;
     const int pairs = batch->batch * Hkv;
     if ((int64_t)batch->batch * Hkv > 65535) return LOKI_ERR_UNSUPPORTED;
     if (batch->max_seq_len > loki_decode_max_seq_len(D, cache->dtype)) return LOKI_ERR_UNSUPPORTED;
 
     const DeviceInfo di = device_info();
-    const int C = choose_cluster(batch->max_seq_len, pairs, di.sms);
-    if (C < 1) return LOKI_ERR_UNSUPPORTED;
     SparseParams p;
     p.k_cache = cache->k_cache;
     p.v_cache = cache->v_cache;
+    p.k_index = cache->k_index;
     p.block_table = batch->block_table;
     p.seq_lens = batch->seq_lens;
     p.k_per_seq = k_per_seq;
@@ -354,18 +406,15 @@ loki_status loki_decode_attention(const loki_cache* cache, const loki_batch* bat
     p.Hkv = Hkv;
     p.max_blocks = batch->max_blocks_per_seq;
     p.max_seq_len = batch->max_seq_len;
+    p.index_dims = cache->index_dims;
     p.r = r;
     p.k = k;
     p.W = recent_window;
     p.group_max = group_reduce == LOKI_GROUP_MAX ? 1 : 0;
     const double sc = scale == 0.f ? 1.0 / std::sqrt((double)D) : (double)scale;
     p.scale_log2 = (float)(sc * kLog2e);
-    p.C = C;
-    const int nblk = (batch->max_seq_len + kBlockTokens - 1) / kBlockTokens;
-    p.cta_tokens = std::max(1, (nblk + C - 1) / C) * kBlockTokens;
-    sparse_layout(p, D, G, elem_size(cache->dtype));
-    if (p.smem_bytes > di.max_smem_optin) return LOKI_ERR_UNSUPPORTED;
-    return dispatch_tdg<SparseLaunch>(cache->dtype, D, G, p, pairs, reinterpret_cast<cudaStream_t>(stream));
+    return dispatch_tdg<SparseLaunch>(cache->dtype, D, G, p, pairs, (int)batch->max_seq_len, di,
+                                      reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -2,28 +2,29 @@
 // (sequence, kv head). The sequence's tokens are split into C contiguous
 // ranges of whole 16-token blocks, one per CTA, and every phase stays on chip:
 //
-//  1. prologue: P[h] arrives in shared memory by one bulk async copy (TMA
-//     engine); q_hat_j = q_j P[h] for the group's G query heads (AQUA page,
-//     appendix step 1: project the query with P). The key stream of phase 2
-//     is already in flight meanwhile.
+//  1. prologue: the key-index stream of phase 2 starts at once; meanwhile
+//     q_hat_j = q_j P[h] for the group's G query heads (AQUA page, appendix on
+//     complexity, step 1), register-blocked over (row group, column quad) of P.
 //  2. rank-r scoring (AQUA page, related work on LoKi: slice the leading
 //     dimensions after projection; Loki page, abstract: scores in the
 //     low-dimensional space). Each warp owns a private ring of bulk-copy
-//     slots; a slot receives the leading r/16 key slabs of one block, one
-//     contiguous run of r*16 elements. Scores become order-preserving uint32
-//     keys in shared memory; the histogram of their top 11 bits is built on
-//     the fly.
+//     slots (TMA engine, non-tensor form); a slot receives the leading r
+//     index dims of one 16-token block, one contiguous run of r*16 elements.
+//     Scores become order-preserving uint32 keys in shared memory; the
+//     histogram of their top 11 bits is built on the fly (one atomic per
+//     distinct bin per warp).
 //  3. top-k (Loki page, abstract: rank and select tokens): an exact radix
-//     select with digits of 11, 11 and 10 bits. After each digit the CTAs
-//     of the cluster sum their histograms through distributed shared memory,
-//     so every CTA finds the same boundary digit. The result is the k-th
-//     largest key tau and the number `need` of keys equal to tau to keep;
-//     those go to the lowest token indices (ties to the lower index), CTA by
-//     CTA in rank order. The recent window (aitopics page, LRQK abstract) is
-//     appended. Kept tokens become an ascending list of local indices.
+//     select with digits of 11, 11 and 10 bits. After each digit the CTAs of
+//     the cluster sum their histograms through distributed shared memory, so
+//     every CTA finds the same boundary digit. The result is the k-th largest
+//     key tau and the number of keys equal to tau to keep; those go to the
+//     lowest token indices (ties to the lower index), CTA by CTA in rank
+//     order. The recent window (aitopics page, LRQK abstract) is appended.
+//     Kept tokens become an ascending list of local indices.
 //  4. exact attention over the kept tokens (AQUA page, decode-step equations
-//     (3)-(5)) by AttnCore, each warp on its share of the list, loads of the
-//     next chunk in flight while the current one is consumed.
+//     (3)-(5)): each warp stages chunks of key rows and value rows into
+//     shared memory with cp.async (the next chunk in flight while the current
+//     one is consumed) and runs AttnCore on them.
 //  5. the warps' partials merge per CTA, then rank 0 merges the CTAs'
 //     partials through distributed shared memory and writes the output.
 #pragma once
@@ -36,16 +37,26 @@ namespace loki {
 
 namespace cg = cooperative_groups;
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kRingBytesPerWarp = 8192;
 constexpr int kMaxSlots = 16;
 constexpr int kHistBins = 2048;  // 11-bit digits (10 in the last pass)
 constexpr int kCtaTokenCap = 16384;
+// Scoring loop tuning: blocks per warp iteration, and whether the top-digit
+// histogram aggregates equal bins of a warp (match) or adds one by one.
+#ifndef LOKI_SCORE_BLOCKS
+#define LOKI_SCORE_BLOCKS 1
+#endif
+#ifndef LOKI_SCORE_HIST_MATCH
+#define LOKI_SCORE_HIST_MATCH 0
+#endif
+constexpr int kScoreBlocks = LOKI_SCORE_BLOCKS;
+constexpr bool kScoreHistMatch = LOKI_SCORE_HIST_MATCH != 0;
 
 struct SparseParams {
     const void* k_cache;
     const void* v_cache;
+    const void* k_index;
     const int32_t* block_table;
     const int32_t* seq_lens;
     const int32_t* k_per_seq;
@@ -53,24 +64,66 @@ struct SparseParams {
     const float* P;
     float* out;
     int32_t* sel;
-    int num_blocks, Hkv, max_blocks, max_seq_len;
+    int num_blocks, Hkv, max_blocks, max_seq_len, index_dims;
     int r, k, W, group_max;
     float scale_log2;
     int C;           // CTAs per (sequence, kv head), = cluster size
     int cta_tokens;  // token capacity of one CTA, multiple of 16
     int slots;       // ring slots per warp
-    int slot_bytes;  // bytes of one block's leading r dims
-    // shared-memory layout, byte offsets
-    int off_keys, off_ring, off_list, off_qf, off_qhat, off_qs, off_tbl, off_hist, off_bars, off_part,
-        off_misc, smem_bytes;
+    int slot_bytes;  // bytes of one block's leading r index dims
+    int ring_bytes_per_warp;
+    int cand_cap;    // entries of the boundary-candidate buffer (head of the ring region)
+    // shared-memory layout, byte offsets. keys and ring are adjacent: after the
+    // scoring the ring region holds the candidate buffer (head) and the kept
+    // list (tail), and the gather stages rows across keys + ring minus list.
+    int off_keys, keys_bytes, off_ring, ring_bytes, off_list, off_qf, off_qhat, off_qs, off_tbl, off_hist,
+        off_bars, off_part, off_misc, smem_bytes;
 };
+
+#ifndef LOKI_GATHER_CHUNK
+#define LOKI_GATHER_CHUNK 8
+#endif
+template <typename T, int D, int G>
+struct SparseGeom {
+    using Core = AttnCore<T, D, G, (LOKI_GATHER_CHUNK * G > 32 ? 32 / G : LOKI_GATHER_CHUNK)>;
+    static constexpr int NCH = Core::NCH;
+    static constexpr int TB = 2 * D * (int)sizeof(T);  // key row + value row bytes
+    static constexpr int CHUNK_BYTES = NCH * TB;
+    static constexpr int GS_FIT = (160 * 1024) / (kWarps * CHUNK_BYTES);
+    static constexpr int GS = GS_FIT < 1 ? 1 : (GS_FIT > 8 ? 8 : GS_FIT);  // staged chunks per warp
+    static constexpr int STAGE_BYTES = kWarps * GS * CHUNK_BYTES;
+    static constexpr int WPART_BYTES = kWarps * G * (D + 2) * 4;
+    static constexpr int QSCRATCH_BYTES = (2048 / D) * G * D * 4;  // row groups x G x D floats
+};
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, bool valid) {
+    const int n = valid ? 16 : 0;  // 0: nothing is read, the 16 bytes are zero-filled
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc), "r"(n)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Exclusive prefix sum over the lanes of a warp.
+__device__ __forceinline__ int warp_exclusive_scan(int v, int lane) {
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, x, o);
+        if (lane >= o) x += y;
+    }
+    return x - v;
+}
 
 // Exclusive suffix sum over the block: returns sum of v over threads > tid.
 __device__ __forceinline__ uint32_t block_suffix_exclusive(uint32_t v, uint32_t* wsum, int lane, int warp) {
     uint32_t x = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        uint32_t y = __shfl_down_sync(kFull, x, o);
+        const uint32_t y = __shfl_down_sync(kFull, x, o);
         if (lane + o < 32) x += y;
     }
     if (lane == 0) wsum[warp] = x;
@@ -83,8 +136,11 @@ __device__ __forceinline__ uint32_t block_suffix_exclusive(uint32_t v, uint32_t*
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const SparseParams p) {
-    using Core = AttnCore<T, D, G>;
-    constexpr int NCH = Core::NCH;
+    using Geom = SparseGeom<T, D, G>;
+    using Core = typename Geom::Core;
+    constexpr int NCH = Geom::NCH;
+    constexpr int TB = Geom::TB;
+    constexpr int GS = Geom::GS;
     extern __shared__ __align__(128) unsigned char smem[];
     cg::cluster_group cluster = cg::this_cluster();
 
@@ -96,11 +152,12 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     const int Hq = p.Hkv * G;
 
     uint32_t* keys = reinterpret_cast<uint32_t*>(smem + p.off_keys);
-    float* Ps = reinterpret_cast<float*>(smem + p.off_keys);  // P[h] staging, before keys exist
+    float* qscratch = reinterpret_cast<float*>(smem + p.off_keys);  // prologue only
+    unsigned char* stage = smem + p.off_keys;                        // gather only (keys + ring)
+    float* wpart = reinterpret_cast<float*>(smem + p.off_keys);     // after the gather
     unsigned char* ring = smem + p.off_ring;
-    float* wpart = reinterpret_cast<float*>(smem + p.off_ring);  // warp partials, after scoring
     uint16_t* list = reinterpret_cast<uint16_t*>(smem + p.off_list);
-    float* qf = reinterpret_cast<float*>(smem + p.off_qf);
+    float* wts = reinterpret_cast<float*>(smem + p.off_qf);         // merge weights [G][kWarps]
     float* qhat = reinterpret_cast<float*>(smem + p.off_qhat);
     float* qs = reinterpret_cast<float*>(smem + p.off_qs);
     int32_t* tbl = reinterpret_cast<int32_t*>(smem + p.off_tbl);
@@ -108,8 +165,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bars);
     float* part = reinterpret_cast<float*>(smem + p.off_part);
     int32_t* misc = reinterpret_cast<int32_t*>(smem + p.off_misc);
-    // misc: [0] boundary digit, [1] count above it, [8..15] warp sums,
-    //       [16..23] warp gt counts, [24..31] warp eq counts, [32] list length
+    // misc: [0] boundary digit, [1] count above it, [8..23] warp sums,
+    //       [32..47] warp kept counts, [48..63] warp equal counts, [64] list
+    //       length, [66] candidate count, [80..95] warp counts above digit 0
 
     // ---- sequence geometry (identical in every CTA of the cluster) ----
     int L = p.seq_lens[b];
@@ -137,147 +195,261 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     const int n_cand_loc = max(0, min(ncand - t0, n_loc));
     const int nblk_score = (n_cand_loc + kBlockTokens - 1) / kBlockTokens;
 
-    // ---- 1. prologue ----
+    // ---- 1. prologue: every global load is issued before the first barrier ----
     const int S = p.slots;
-    uint64_t* pbar = bars + kWarps * kMaxSlots;
+    // block-table entries of this warp's blocks jb = warp + it * kWarps:
+    // lane l holds those of it = l and it = l + 32 (at most 64 per warp)
+    const int32_t* trow = p.block_table + (int64_t)b * p.max_blocks + blk0;
+    int tb0 = 0, tb1 = 0;
+    {
+        const int j0 = warp + lane * kWarps, j1 = warp + (lane + 32) * kWarps;
+        if (j0 < nblk_loc) tb0 = trow[j0];
+        if (j1 < nblk_loc) tb1 = trow[j1];
+    }
+    constexpr int NQ = D / 4;             // q_hat: thread (row group rg, column quad cq)
+    constexpr int NRG = kThreads / NQ;
+    constexpr int RPG = D / NRG;
+    const int cq = tid % NQ, rg = tid / NQ;
+    float4 pv[RPG];
+    {
+        const float* Ph = p.P + (int64_t)h * D * D;
+#pragma unroll
+        for (int i = 0; i < RPG; ++i) pv[i] = *reinterpret_cast<const float4*>(Ph + (rg * RPG + i) * D + 4 * cq);
+    }
+    const T* qg = reinterpret_cast<const T*>(p.q) + ((int64_t)b * Hq + h * G) * D;
+    typename Vec<T, RPG>::raw_t qraw[G];
+#pragma unroll
+    for (int j = 0; j < G; ++j) qraw[j] = Vec<T, RPG>::load(qg + j * D + rg * RPG);
+
     if (tid == 0) {
-        for (int i = 0; i < kWarps * kMaxSlots + 1; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < kWarps * kMaxSlots; ++i) mbar_init(&bars[i], 1);
         fence_mbarrier_init();
     }
     for (int i = tid; i < 2 * kHistBins; i += kThreads) hist[i] = 0;
-    for (int jb = tid; jb < nblk_loc; jb += kThreads) {
-        int pb = p.block_table[(int64_t)b * p.max_blocks + blk0 + jb];
+    auto checked = [&](int pb) {
         if (pb < 0 || pb >= p.num_blocks) {
             flag_error(LOKI_DEVERR_BLOCK_ID);
-            pb = 0;
+            return 0;
         }
-        tbl[jb] = pb;
+        return pb;
+    };
+    tb0 = checked(tb0);
+    tb1 = checked(tb1);
+    {
+        const int j0 = warp + lane * kWarps, j1 = warp + (lane + 32) * kWarps;
+        if (j0 < nblk_loc) tbl[j0] = tb0;
+        if (j1 < nblk_loc) tbl[j1] = tb1;
     }
-    const T* qg = reinterpret_cast<const T*>(p.q) + ((int64_t)b * Hq + h * G) * D;
-    for (int i = tid; i < G * D; i += kThreads) qf[i] = Elem<T>::to_f(qg[i]);
     __syncthreads();
 
-    if (tid == 0) {
-        mbar_arrive_expect_tx(pbar, D * D * 4);
-        bulk_copy_g2s(Ps, p.P + (int64_t)h * D * D, D * D * 4, pbar);
-    }
-    unsigned char* wring = ring + warp * kRingBytesPerWarp;
+    unsigned char* wring = ring + warp * p.ring_bytes_per_warp;
     uint64_t* wbar = bars + warp * kMaxSlots;
     const int my_blocks = nblk_score > warp ? (nblk_score - warp + kWarps - 1) / kWarps : 0;
-    const unsigned char* kbytes = reinterpret_cast<const unsigned char*>(p.k_cache);
-    auto issue = [&](int it) {
-        const int jb = warp + it * kWarps;
+    const unsigned char* xbytes = reinterpret_cast<const unsigned char*>(p.k_index);
+    auto issue = [&](int it, int pb) {  // lane 0 only
         const int slot = it % S;
-        const unsigned char* src = kbytes + page_offset(tbl[jb], h, p.Hkv, D) * (int64_t)sizeof(T);
+        const unsigned char* src = xbytes + page_offset(pb, h, p.Hkv, p.index_dims) * (int64_t)sizeof(T);
         mbar_arrive_expect_tx(&wbar[slot], (uint32_t)p.slot_bytes);
         bulk_copy_g2s(wring + slot * p.slot_bytes, src, (uint32_t)p.slot_bytes, &wbar[slot]);
     };
-    if (lane == 0) {
+    auto entry = [&](int it) {  // all lanes: block of this warp's iteration it
+        const int v0 = __shfl_sync(kFull, tb0, it & 31);
+        const int v1 = __shfl_sync(kFull, tb1, it & 31);
+        return it < 32 ? v0 : v1;
+    };
+    {
         const int first = my_blocks < S ? my_blocks : S;
-        for (int it = 0; it < first; ++it) issue(it);
-    }
-
-    const bool okP = mbar_wait_bounded(pbar, 0);
-    for (int o = tid; o < G * D; o += kThreads) {
-        const int j = o / D, c = o - j * D;
-        float a = 0.f;
-#pragma unroll 8
-        for (int i = 0; i < D; ++i) a = fmaf(qf[j * D + i], Ps[i * D + c], a);
-        qhat[o] = okP ? a : 0.f;
-    }
-    __syncthreads();
-    if (!p.group_max) {
-        for (int c = tid; c < p.r; c += kThreads) {
-            float s = 0.f;
-            for (int j = 0; j < G; ++j) s += qhat[j * D + c];
-            qs[c] = s;
+        for (int it = 0; it < first; ++it) {
+            const int pb = entry(it);
+            if (lane == 0) issue(it, pb);
         }
     }
-    __syncthreads();
+
+    {   // q_hat = q P[h]: each thread sums its RPG rows for its 4 columns
+        float qv[G][RPG];
+#pragma unroll
+        for (int j = 0; j < G; ++j) Vec<T, RPG>::to_float(qraw[j], qv[j]);
+        float a[G][4];
+#pragma unroll
+        for (int j = 0; j < G; ++j) a[j][0] = a[j][1] = a[j][2] = a[j][3] = 0.f;
+#pragma unroll
+        for (int i = 0; i < RPG; ++i) {
+#pragma unroll
+            for (int j = 0; j < G; ++j) {
+                const float x = qv[j][i];
+                a[j][0] = fmaf(x, pv[i].x, a[j][0]);
+                a[j][1] = fmaf(x, pv[i].y, a[j][1]);
+                a[j][2] = fmaf(x, pv[i].z, a[j][2]);
+                a[j][3] = fmaf(x, pv[i].w, a[j][3]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < G; ++j)
+            *reinterpret_cast<float4*>(qscratch + (rg * G + j) * D + 4 * cq) =
+                make_float4(a[j][0], a[j][1], a[j][2], a[j][3]);
+        __syncthreads();
+        for (int o = tid; o < G * D; o += kThreads) {
+            float s = 0.f;
+            for (int g = 0; g < NRG; ++g) s += qscratch[g * G * D + o];
+            qhat[o] = s;
+        }
+        __syncthreads();
+        if (!p.group_max) {
+            for (int c = tid; c < p.r; c += kThreads) {
+                float s = 0.f;
+                for (int j = 0; j < G; ++j) s += qhat[j * D + c];
+                qs[c] = s;
+            }
+        }
+        __syncthreads();
+    }
 
     // ---- 2. rank-r scoring ----
+    // A warp takes kScoreBlocks blocks per iteration: their slots are read into
+    // registers and handed back to the bulk-copy engine before the arithmetic,
+    // and the blocks' dot products run as independent chains.
     {
-        const int R16 = p.r / kSlabDims;
-        const int tok = lane >> 1, half = lane & 1;
         bool failed = false;
-        for (int it = 0; it < my_blocks; ++it) {
-            const int slot = it % S;
-            const uint32_t parity = (uint32_t)(it / S) & 1u;
-            if (!failed) failed = __any_sync(kFull, !mbar_wait_bounded(&wbar[slot], parity));
-            const T* sl = reinterpret_cast<const T*>(wring + slot * p.slot_bytes);
-            float s;
-            if (!p.group_max) {
-                float a = 0.f;
-                for (int sb = 0; sb < R16; ++sb) {
-                    float kf[8];
-                    Vec<T, 8>::to_float(Vec<T, 8>::load(sl + sb * 256 + tok * 16 + half * 8), kf);
-                    const float* qq = qs + sb * 16 + half * 8;
+        // RMAX: compile-time bound on the slabs per block; R16 <= RMAX at run time
+        auto body = [&](auto rmax_tag) {
+            constexpr int RMAX = decltype(rmax_tag)::value;
+            const int R16 = p.r / kSlabDims;
+            constexpr int NB = kScoreBlocks;
+            using V8 = Vec<T, 8>;
+            const int tok = lane >> 1, half = lane & 1;
+            for (int it = 0; it < my_blocks; it += NB) {
+                typename V8::raw_t raw[NB][RMAX];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) a = fmaf(qq[i], kf[i], a);
-                }
-                s = a + __shfl_xor_sync(kFull, a, 1);
-            } else {
-                float ag[G];
+                for (int u = 0; u < NB; ++u) {
+                    if (it + u < my_blocks) {
+                        const int slot = (it + u) % S;
+                        const uint32_t parity = (uint32_t)((it + u) / S) & 1u;
+                        if (!failed) failed = __any_sync(kFull, !mbar_wait_bounded(&wbar[slot], parity));
+                        const T* sl = reinterpret_cast<const T*>(wring + slot * p.slot_bytes);
 #pragma unroll
-                for (int j = 0; j < G; ++j) ag[j] = 0.f;
-                for (int sb = 0; sb < R16; ++sb) {
-                    float kf[8];
-                    Vec<T, 8>::to_float(Vec<T, 8>::load(sl + sb * 256 + tok * 16 + half * 8), kf);
-#pragma unroll
-                    for (int j = 0; j < G; ++j) {
-                        const float* qq = qhat + j * D + sb * 16 + half * 8;
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) ag[j] = fmaf(qq[i], kf[i], ag[j]);
+                        for (int sb = 0; sb < RMAX; ++sb)
+                            if (sb < R16) raw[u][sb] = V8::load(sl + sb * 256 + tok * 16 + half * 8);
                     }
                 }
-                s = -INFINITY;
+                __syncwarp();
 #pragma unroll
-                for (int j = 0; j < G; ++j) s = fmaxf(s, ag[j] + __shfl_xor_sync(kFull, ag[j], 1));
+                for (int u = 0; u < NB; ++u) {
+                    if (it + u + S < my_blocks) {
+                        const int pb = entry(it + u + S);
+                        if (lane == 0) issue(it + u + S, pb);
+                    }
+                }
+                float sc[NB];
+                if (!p.group_max) {
+#pragma unroll
+                    for (int u = 0; u < NB; ++u) {
+                        float a = 0.f;
+#pragma unroll
+                        for (int sb = 0; sb < RMAX; ++sb) {
+                            if (sb >= R16) break;
+                            float kf[8];
+                            V8::to_float(raw[u][sb], kf);
+                            const float4 q0 = *reinterpret_cast<const float4*>(qs + sb * 16 + half * 8);
+                            const float4 q1 = *reinterpret_cast<const float4*>(qs + sb * 16 + half * 8 + 4);
+                            a = fmaf(q0.x, kf[0], a);
+                            a = fmaf(q0.y, kf[1], a);
+                            a = fmaf(q0.z, kf[2], a);
+                            a = fmaf(q0.w, kf[3], a);
+                            a = fmaf(q1.x, kf[4], a);
+                            a = fmaf(q1.y, kf[5], a);
+                            a = fmaf(q1.z, kf[6], a);
+                            a = fmaf(q1.w, kf[7], a);
+                        }
+                        sc[u] = a;
+                    }
+#pragma unroll
+                    for (int u = 0; u < NB; ++u) sc[u] += __shfl_xor_sync(kFull, sc[u], 1);
+                } else {
+#pragma unroll
+                    for (int u = 0; u < NB; ++u) {
+                        float ag[G];
+#pragma unroll
+                        for (int j = 0; j < G; ++j) ag[j] = 0.f;
+#pragma unroll
+                        for (int sb = 0; sb < RMAX; ++sb) {
+                            if (sb >= R16) break;
+                            float kf[8];
+                            V8::to_float(raw[u][sb], kf);
+#pragma unroll
+                            for (int j = 0; j < G; ++j) {
+                                const float* qq = qhat + j * D + sb * 16 + half * 8;
+#pragma unroll
+                                for (int i = 0; i < 8; ++i) ag[j] = fmaf(qq[i], kf[i], ag[j]);
+                            }
+                        }
+                        float m = -INFINITY;
+#pragma unroll
+                        for (int j = 0; j < G; ++j) m = fmaxf(m, ag[j] + __shfl_xor_sync(kFull, ag[j], 1));
+                        sc[u] = m;
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < NB; ++u) {
+                    const int li = (warp + (it + u) * kWarps) * kBlockTokens + tok;
+                    const bool valid = half == 0 && it + u < my_blocks && li < n_cand_loc;
+                    const uint32_t key = score_key(sc[u]);
+                    if (valid) keys[li] = key;
+                    const unsigned bin = key >> 21;
+                    if constexpr (kScoreHistMatch) {
+                        const unsigned vmask = __ballot_sync(kFull, valid);
+                        if (valid) {
+                            const unsigned peers = __match_any_sync(vmask, bin);
+                            if ((peers & ((1u << lane) - 1u)) == 0) atomicAdd(&hist[bin], (unsigned)__popc(peers));
+                        }
+                    } else {
+                        if (valid) atomicAdd(&hist[bin], 1u);
+                    }
+                }
             }
-            const int li = (warp + it * kWarps) * kBlockTokens + tok;
-            if (half == 0 && li < n_cand_loc) {
-                const uint32_t key = score_key(s);
-                keys[li] = key;
-                atomicAdd(&hist[key >> 21], 1u);
-            }
-            __syncwarp();
-            if (lane == 0 && it + S < my_blocks) {
-                fence_proxy_async_smem();
-                issue(it + S);
-            }
-        }
+        };
+        if (p.r <= 2 * kSlabDims)
+            body(std::integral_constant<int, 2>{});
+        else
+            body(std::integral_constant<int, D / kSlabDims>{});
     }
     __syncthreads();
 
     // ---- 3. top-k over the cluster ----
-    // mode 0: keep every candidate, 1: keep none, 2: threshold tau / quota
+    // mode 0: keep every candidate, 1: keep none, 2: threshold tau / quota.
+    // Warp w owns the contiguous key range [lo, hi) in every scan below.
     const int mode = keff >= ncand ? 0 : (keff == 0 ? 1 : 2);
+    const int per_warp = (((n_cand_loc + kWarps - 1) / kWarps) + 127) & ~127;
+    const int lo = min(warp * per_warp, n_cand_loc);
+    const int hi = min(lo + per_warp, n_cand_loc);
+    const uint4* k4 = reinterpret_cast<const uint4*>(keys);
+    uint2* cand = reinterpret_cast<uint2*>(ring);  // (key, local index) of boundary-bin keys
     uint32_t tau = 0;
     int quota = 0;
+    bool counted = false;  // per-warp kept / equal counts already in misc[32..63]
     if (mode == 2) {
-        uint32_t prefix = 0, pmask = 0;
-        int krem = keff;
-        for (int pass = 0; pass < 3; ++pass) {
-            const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-            const int nbins = pass == 2 ? 1024 : 2048;
-            uint32_t* hcur = hist + (pass & 1) * kHistBins;
-            if (pass > 0) {
-                for (int i = tid; i < n_cand_loc; i += kThreads) {
-                    const uint32_t key = keys[i];
-                    if ((key & pmask) == prefix) atomicAdd(&hcur[(key >> shift) & (nbins - 1)], 1u);
-                }
-            }
+        // Sum the cluster's histograms (buffer hcur) and find the digit where
+        // the count from the top reaches krem; returns (digit, count above it).
+        auto boundary = [&](const uint32_t* hcur, int nbins, int krem) {
             __syncthreads();
             cluster.sync();
-            const int bpt = nbins / kThreads;  // 8 or 4 bins per thread
-            uint32_t hv[8];
-            uint32_t tsum = 0;
-            for (int j = 0; j < bpt; ++j) {
-                uint32_t s = 0;
-                for (int c = 0; c < p.C; ++c) s += cluster.map_shared_rank(hcur, c)[tid * bpt + j];
-                hv[j] = s;
-                tsum += s;
+            const int bpt = nbins / kThreads;  // 4 or 2 bins per thread
+            uint32_t hv[4] = {0u, 0u, 0u, 0u};
+            if (bpt == 4) {
+                for (int c = 0; c < p.C; ++c) {
+                    const uint4 v = reinterpret_cast<const uint4*>(cluster.map_shared_rank(hcur, c))[tid];
+                    hv[0] += v.x;
+                    hv[1] += v.y;
+                    hv[2] += v.z;
+                    hv[3] += v.w;
+                }
+            } else {
+                for (int c = 0; c < p.C; ++c) {
+                    const uint2 v = reinterpret_cast<const uint2*>(cluster.map_shared_rank(hcur, c))[tid];
+                    hv[0] += v.x;
+                    hv[1] += v.y;
+                }
             }
+            const uint32_t tsum = hv[0] + hv[1] + hv[2] + hv[3];
             uint32_t run = block_suffix_exclusive(tsum, reinterpret_cast<uint32_t*>(misc + 8), lane, warp);
             for (int j = bpt - 1; j >= 0; --j) {
                 if (run < (uint32_t)krem && run + hv[j] >= (uint32_t)krem) {
@@ -287,83 +459,180 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
                 run += hv[j];
             }
             __syncthreads();
-            const int beta = misc[0];
-            krem -= misc[1];
-            prefix |= (uint32_t)beta << shift;
-            pmask |= (uint32_t)(nbins - 1) << shift;
-            if (pass < 2) {
-                uint32_t* hnext = hist + ((pass + 1) & 1) * kHistBins;
-                for (int i = tid; i < kHistBins; i += kThreads) hnext[i] = 0;
+            return make_int2(misc[0], misc[1]);
+        };
+        // digit 0 (top 11 bits): its histogram was built while scoring
+        const int2 d0 = boundary(hist, 2048, keff);
+        const uint32_t beta0 = (uint32_t)d0.x;
+        int krem = keff - d0.y;
+        // digit 1: one scan of the keys counts the keys above the boundary
+        // bin per warp and copies the boundary bin's keys to the candidate
+        // buffer (unless there are too many: then later passes rescan keys)
+        const bool use_buf = (int)hist[beta0] <= p.cand_cap;
+        uint32_t* h1 = hist + kHistBins;
+        if (tid == 0) misc[66] = 0;
+        __syncthreads();
+        {
+            int gt0 = 0;
+            for (int base = lo; base < hi; base += 128) {
+                const int i0 = base + lane * 4;
+                const uint4 v = i0 < hi ? k4[i0 / 4] : make_uint4(0u, 0u, 0u, 0u);
+                const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
+                bool isc[4];
+                int nc = 0;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const bool in = i0 + j < hi;
+                    const uint32_t dg = kk[j] >> 21;
+                    gt0 += in && dg > beta0;
+                    isc[j] = in && dg == beta0;
+                    nc += isc[j];
+                    if (isc[j]) atomicAdd(&h1[(kk[j] >> 10) & 2047u], 1u);
+                }
+                if (use_buf) {
+                    const unsigned any = __ballot_sync(kFull, nc > 0);
+                    if (any) {
+                        const int pre = warp_exclusive_scan(nc, lane);
+                        const int tot = __shfl_sync(kFull, pre + nc, 31);
+                        int at = 0;
+                        if (lane == 0) at = atomicAdd(&misc[66], tot);
+                        at = __shfl_sync(kFull, at, 0) + pre;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            if (isc[j]) cand[at++] = make_uint2(kk[j], (uint32_t)(i0 + j));
+                    }
+                }
             }
-            __syncthreads();
+            gt0 = __reduce_add_sync(kFull, gt0);
+            if (lane == 0) misc[80 + warp] = gt0;
         }
-        tau = prefix;
-        // keys equal to tau: the last pass counted them per CTA in bin (tau & 1023)
+        const int2 d1 = boundary(h1, 2048, krem);
+        const uint32_t beta1 = (uint32_t)d1.x;
+        krem -= d1.y;
+        // digit 2 (last 10 bits), over the candidates only
+        for (int i = tid; i < kHistBins; i += kThreads) hist[i] = 0;  // readers of digit 0 are done
+        __syncthreads();
+        const uint32_t pre22 = (beta0 << 21) | (beta1 << 10);
+        const int ncb = misc[66];
+        if (use_buf) {
+            for (int i = tid; i < ncb; i += kThreads) {
+                const uint32_t kk = cand[i].x;
+                if ((kk & 0xFFFFFC00u) == pre22) atomicAdd(&hist[kk & 1023u], 1u);
+            }
+        } else {
+            const int n4 = (n_cand_loc + 3) / 4;
+            for (int qd = tid; qd < n4; qd += kThreads) {
+                const uint4 v = k4[qd];
+                const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (4 * qd + j < n_cand_loc && (kk[j] & 0xFFFFFC00u) == pre22) atomicAdd(&hist[kk[j] & 1023u], 1u);
+            }
+        }
+        const int2 d2 = boundary(hist, 1024, krem);
+        tau = pre22 | (uint32_t)d2.x;
+        krem -= d2.y;
+        // keys equal to tau: the last histogram counted them per CTA in bin (tau & 1023)
         int eq_before = 0;
         for (int c = 0; c < crank; ++c) eq_before += (int)cluster.map_shared_rank(hist, c)[tau & 1023u];
         const int eq_mine = (int)hist[tau & 1023u];
         quota = min(max(krem - eq_before, 0), eq_mine);
+        // per-warp kept / equal counts from the candidates
+        if (use_buf) {
+            if (tid < 2 * kWarps) misc[32 + tid] = 0;
+            __syncthreads();
+            for (int i = tid; i < ncb; i += kThreads) {
+                const uint2 e = cand[i];
+                const int w = (int)e.y / per_warp;
+                if (e.x > tau) atomicAdd(&misc[32 + w], 1);
+                else if (e.x == tau) atomicAdd(&misc[48 + w], 1);
+            }
+            __syncthreads();
+            if (tid < kWarps) misc[32 + tid] += misc[80 + tid];
+            counted = true;
+        }
     }
 
     // ---- compaction of the kept local tokens into `list`, ascending ----
     {
-        const int chunk = (((n_cand_loc + kWarps - 1) / kWarps) + 31) & ~31;
-        const int lo = warp * chunk;
-        const int hi = min(lo + chunk, n_cand_loc);
-        const unsigned lt_mask = (1u << lane) - 1u;
-        int cnt_gt = 0, cnt_eq = 0;
-        for (int base = lo; base < hi; base += 32) {
-            const int i = base + lane;
-            const bool in = i < hi;
-            const uint32_t key = in ? keys[i] : 0u;
-            const bool gt = in && (mode == 0 || (mode == 2 && key > tau));
-            const bool eq = in && mode == 2 && key == tau;
-            cnt_gt += __popc(__ballot_sync(kFull, gt));
-            cnt_eq += __popc(__ballot_sync(kFull, eq));
-        }
-        if (lane == 0) {
-            misc[16 + warp] = cnt_gt;
-            misc[24 + warp] = cnt_eq;
+        auto classify = [&](int i0, bool (&gt)[4], bool (&eq)[4]) {
+            const uint4 v = i0 < hi ? k4[i0 / 4] : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const bool in = i0 + j < hi;
+                gt[j] = in && (mode == 0 || (mode == 2 && kk[j] > tau));
+                eq[j] = in && mode == 2 && kk[j] == tau;
+            }
+        };
+        if (!counted) {
+            int cgt = 0, ceq = 0;
+            for (int base = lo; base < hi; base += 128) {
+                bool gt[4], eq[4];
+                classify(base + lane * 4, gt, eq);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    cgt += gt[j];
+                    ceq += eq[j];
+                }
+            }
+            cgt = __reduce_add_sync(kFull, cgt);
+            ceq = __reduce_add_sync(kFull, ceq);
+            __syncthreads();
+            if (lane == 0) {
+                misc[32 + warp] = cgt;
+                misc[48 + warp] = ceq;
+            }
         }
         __syncthreads();
         // warp w keeps all its keys above tau and the equal ones whose rank
         // among the CTA's equal keys (in index order) is below the quota
         int eq_base = 0, out_base = 0, total = 0, eb = 0;
         for (int w = 0; w < kWarps; ++w) {
-            const int take = min(max(quota - eb, 0), misc[24 + w]);
+            const int take = min(max(quota - eb, 0), misc[48 + w]);
             if (w < warp) {
-                out_base += misc[16 + w] + take;
-                eq_base += misc[24 + w];
+                out_base += misc[32 + w] + take;
+                eq_base += misc[48 + w];
             }
-            total += misc[16 + w] + take;
-            eb += misc[24 + w];
+            total += misc[32 + w] + take;
+            eb += misc[48 + w];
         }
         int run_eq = eq_base, run_out = out_base;
-        for (int base = lo; base < hi; base += 32) {
-            const int i = base + lane;
-            const bool in = i < hi;
-            const uint32_t key = in ? keys[i] : 0u;
-            const bool gt = in && (mode == 0 || (mode == 2 && key > tau));
-            const bool eq = in && mode == 2 && key == tau;
-            const unsigned beq = __ballot_sync(kFull, eq);
-            const bool take = gt || (eq && run_eq + __popc(beq & lt_mask) < quota);
-            const unsigned bt = __ballot_sync(kFull, take);
-            if (take) list[run_out + __popc(bt & lt_mask)] = (uint16_t)i;
-            run_eq += __popc(beq);
-            run_out += __popc(bt);
+        for (int base = lo; base < hi; base += 128) {
+            const int i0 = base + lane * 4;
+            bool gt[4], eq[4];
+            classify(i0, gt, eq);
+            const int neq = eq[0] + eq[1] + eq[2] + eq[3];
+            const int eq_pre = warp_exclusive_scan(neq, lane);
+            int er = run_eq + eq_pre;
+            bool take[4];
+            int nsel = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                take[j] = gt[j] || (eq[j] && er < quota);
+                er += eq[j];
+                nsel += take[j];
+            }
+            const int sel_pre = warp_exclusive_scan(nsel, lane);
+            int pos = run_out + sel_pre;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (take[j]) list[pos++] = (uint16_t)(i0 + j);
+            run_eq += __shfl_sync(kFull, eq_pre + neq, 31);
+            run_out += __shfl_sync(kFull, sel_pre + nsel, 31);
         }
         for (int i = tid; i < n_loc - n_cand_loc; i += kThreads) list[total + i] = (uint16_t)(n_cand_loc + i);
-        if (tid == 0) misc[32] = total + (n_loc - n_cand_loc);
+        if (tid == 0) misc[64] = total + (n_loc - n_cand_loc);
         __syncthreads();
     }
-    const int n_list = misc[32];
+    const int n_list = misc[64];
 
     // ---- optional export of the kept set ----
     if (p.sel) {
         cluster.sync();
         int before = 0, all = 0;
         for (int c = 0; c < p.C; ++c) {
-            const int nc = cluster.map_shared_rank(misc, c)[32];
+            const int nc = cluster.map_shared_rank(misc, c)[64];
             if (c < crank) before += nc;
             all += nc;
         }
@@ -376,52 +645,81 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
 
     // ---- 4. exact attention over the kept tokens ----
     {
-        const T* kc = reinterpret_cast<const T*>(p.k_cache);
-        const T* vc = reinterpret_cast<const T*>(p.v_cache);
-        Core core;
-        core.init(qhat, p.scale_log2, lane);
-        typename Core::raw_t kA[NCH], vA[NCH], kB[NCH], vB[NCH];
-        uint32_t validA = 0, validB = 0;
+        const unsigned char* kbytes = reinterpret_cast<const unsigned char*>(p.k_cache);
+        const unsigned char* vbytes = reinterpret_cast<const unsigned char*>(p.v_cache);
+        constexpr int PIECES = TB / 16;
+        constexpr int ROWB = D * (int)sizeof(T);
+        unsigned char* wst = stage + warp * GS * Geom::CHUNK_BYTES;
         const int nchunks = (n_list + NCH - 1) / NCH;
-        auto load = [&](typename Core::raw_t (&kr)[NCH], typename Core::raw_t (&vr)[NCH], uint32_t& valid,
-                        int ch) {
-            valid = 0;
-#pragma unroll
-            for (int n = 0; n < NCH; ++n) {
-                const int idx = ch * NCH + n;
-                if (idx < n_list) {
-                    const int li = list[idx];
-                    const int64_t page = page_offset(tbl[li >> 4], h, p.Hkv, D);
-                    kr[n] = Core::V::load(Core::key_ptr(kc, page, li & 15, lane));
-                    vr[n] = Core::V::load(Core::val_ptr(vc, page, li & 15, lane));
-                    valid |= 1u << n;
-                } else {
-                    kr[n] = Core::zero_raw();
-                    vr[n] = Core::zero_raw();
+        const int my_n = nchunks > warp ? (nchunks - warp + kWarps - 1) / kWarps : 0;
+        auto fetch = [&](int m) {
+            if (m < my_n) {
+                unsigned char* dst = wst + (m % GS) * Geom::CHUNK_BYTES;
+                const int ch = warp + m * kWarps;
+                for (int pc = lane; pc < NCH * PIECES; pc += 32) {
+                    const int n = pc / PIECES, o = (pc - n * PIECES) * 16;
+                    const int idx = ch * NCH + n;
+                    const bool ok = idx < n_list;
+                    const unsigned char* src = kbytes;
+                    if (ok) {
+                        const int li = list[idx];
+                        const int64_t at = page_offset(tbl[li >> 4], h, p.Hkv, D) * (int64_t)sizeof(T) +
+                                           (int64_t)(li & 15) * ROWB;
+                        src = o < ROWB ? kbytes + at + o : vbytes + at + (o - ROWB);
+                    }
+                    cp_async16(dst + n * TB + o, src, ok);
                 }
             }
+            cp_async_commit();
         };
-        int ch = warp;
-        if (ch < nchunks) load(kA, vA, validA, ch);
-        for (; ch < nchunks; ch += 2 * kWarps) {
-            if (ch + kWarps < nchunks) load(kB, vB, validB, ch + kWarps);
-            core.consume(kA, vA, validA, lane);
-            if (ch + kWarps >= nchunks) break;
-            if (ch + 2 * kWarps < nchunks) load(kA, vA, validA, ch + 2 * kWarps);
-            core.consume(kB, vB, validB, lane);
+        Core core;
+        core.init(qhat, p.scale_log2, lane);
+        for (int m = 0; m < GS - 1; ++m) fetch(m);
+        for (int m = 0; m < my_n; ++m) {
+            fetch(m + GS - 1);
+            cp_async_wait<GS - 1>();
+            __syncwarp();
+            const unsigned char* src = wst + (m % GS) * Geom::CHUNK_BYTES;
+            typename Core::raw_t kr[NCH], vr[NCH];
+            uint32_t valid = 0;
+#pragma unroll
+            for (int n = 0; n < NCH; ++n) {
+                kr[n] = Core::V::load(reinterpret_cast<const T*>(src + n * TB) + lane * Core::DPL);
+                vr[n] = Core::V::load(reinterpret_cast<const T*>(src + n * TB + ROWB) + lane * Core::DPL);
+                if ((warp + m * kWarps) * NCH + n < n_list) valid |= 1u << n;
+            }
+            core.consume(kr, vr, valid, lane);
+            __syncwarp();
         }
+        cp_async_wait<0>();
+        __syncthreads();  // every warp is done with the staging area
         core.store_partial(wpart + warp * G * (D + 2), lane);
     }
     __syncthreads();
 
     // ---- 5. merge: warps -> CTA partial -> cluster rank 0 -> out ----
-    for (int o = tid; o < G * D; o += kThreads) {
-        const int j = o / D, c = o - j * D;
-        const Merged mg = merge_partials<D>(wpart, kWarps, G * (D + 2), j, c);
-        part[j * (D + 2) + c] = mg.o;
-        if (c == 0) {
-            part[j * (D + 2) + D] = mg.m;
-            part[j * (D + 2) + D + 1] = mg.l;
+    {
+        if (tid < G) {
+            const int j = tid;
+            float M = -INFINITY;
+            for (int w = 0; w < kWarps; ++w) M = fmaxf(M, wpart[w * G * (D + 2) + j * (D + 2) + D]);
+            float lsum = 0.f;
+            for (int w = 0; w < kWarps; ++w) {
+                const float mw = wpart[w * G * (D + 2) + j * (D + 2) + D];
+                const float wt = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+                wts[j * kWarps + w] = wt;
+                lsum = fmaf(wt, wpart[w * G * (D + 2) + j * (D + 2) + D + 1], lsum);
+            }
+            part[j * (D + 2) + D] = M;
+            part[j * (D + 2) + D + 1] = lsum;
+        }
+        __syncthreads();
+        for (int o = tid; o < G * D; o += kThreads) {
+            const int j = o / D, c = o - j * D;
+            float a = 0.f;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) a = fmaf(wts[j * kWarps + w], wpart[w * G * (D + 2) + j * (D + 2) + c], a);
+            part[j * (D + 2) + c] = a;
         }
     }
     cluster.sync();

@@ -37,9 +37,9 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 
 class loki_cache(ctypes.Structure):
-    _fields_ = [("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+    _fields_ = [("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p), ("k_index", ctypes.c_void_p),
                 ("num_blocks", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
-                ("head_dim", ctypes.c_int32), ("dtype", ctypes.c_int)]
+                ("head_dim", ctypes.c_int32), ("index_dims", ctypes.c_int32), ("dtype", ctypes.c_int)]
 
 
 class loki_batch(ctypes.Structure):
@@ -56,6 +56,7 @@ _B = ctypes.POINTER(loki_batch)
 
 _SIGS = {
     "loki_cache_bytes": (_SZ, [_I32, _I32, _I32, ctypes.c_int]),
+    "loki_index_bytes": (_SZ, [_I32, _I32, _I32, ctypes.c_int]),
     "loki_prefill_cache": (ctypes.c_int, [_C, _B, _P, _P, _I32, _P]),
     "loki_append_keys": (ctypes.c_int, [_C, _B, _P, _P, _P, _P]),
     "loki_decode_workspace_bytes": (_SZ, [_C, _B, _I32, _I32, _I32]),
@@ -106,18 +107,22 @@ def dtype_code(dt) -> int:
 # --------------------------------------------------------------------------
 
 class Cache:
-    """Owns a k/v cache pair (torch uint8 buffers) and its loki_cache struct."""
+    """Owns the key, value and key-index buffers (torch uint8) of a paged
+    cache and its loki_cache struct."""
 
-    def __init__(self, num_blocks, num_kv_heads, head_dim, dtype, device="cuda"):
+    def __init__(self, num_blocks, num_kv_heads, head_dim, dtype, device="cuda", index_dims=64):
         code = dtype_code(dtype)
         nbytes = loki_cache_bytes(num_blocks, num_kv_heads, head_dim, code)
-        if nbytes == 0 and num_blocks > 0:
+        ibytes = loki_index_bytes(num_blocks, num_kv_heads, index_dims, code)
+        if (nbytes == 0 or ibytes == 0) and num_blocks > 0:
             raise ValueError("invalid cache shape")
         self.dtype = dtype
+        self.index_dims = index_dims
         self.k = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
         self.v = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
-        self.struct = loki_cache(self.k.data_ptr(), self.v.data_ptr(), num_blocks, num_kv_heads,
-                                 head_dim, code)
+        self.x = torch.empty(max(ibytes, 16), dtype=torch.uint8, device=device)
+        self.struct = loki_cache(self.k.data_ptr(), self.v.data_ptr(), self.x.data_ptr(), num_blocks,
+                                 num_kv_heads, head_dim, index_dims, code)
 
 
 class Batch:
@@ -140,6 +145,10 @@ class Batch:
 
 def loki_cache_bytes(num_blocks, num_kv_heads, head_dim, dtype_code_):
     return _lib.loki_cache_bytes(num_blocks, num_kv_heads, head_dim, dtype_code_)
+
+
+def loki_index_bytes(num_blocks, num_kv_heads, index_dims, dtype_code_):
+    return _lib.loki_index_bytes(num_blocks, num_kv_heads, index_dims, dtype_code_)
 
 
 def loki_prefill_cache(cache, batch, k_rot, v, max_len=None, stream=None):

@@ -19,10 +19,13 @@ def tol_for(spec):
 class Device:
     """A workload's cache and inputs on the GPU."""
 
-    def __init__(self, wl, loki, device="cuda", max_seq_len=None):
+    def __init__(self, wl, loki, device="cuda", max_seq_len=None, index_dims=None):
         s = wl.spec
         self.wl, self.loki = wl, loki
-        self.cache = loki.Cache(wl.num_blocks, s.num_kv_heads, s.head_dim, synth.torch_dtype(s.dtype), device)
+        if index_dims is None:
+            index_dims = max(s.r, min(64, s.head_dim))
+        self.cache = loki.Cache(wl.num_blocks, s.num_kv_heads, s.head_dim, synth.torch_dtype(s.dtype), device,
+                                index_dims=index_dims)
         self.batch = loki.Batch(wl.block_table.to(device), wl.seq_lens.to(device),
                                 max_seq_len if max_seq_len is not None else s.max_seq_len)
         self.q = wl.q.to(device)

@@ -36,13 +36,19 @@ def test_library_exports_every_declared_symbol(loki):
     for name in declared_symbols():
         assert hasattr(lib, name), name
     assert sorted(loki.EXPORTED) == declared_symbols()
-    assert loki.loki_abi_version() == 1
+    assert loki.loki_abi_version() == 2
 
 
 def test_status_strings(loki):
     for s in range(5):
         assert loki.loki_status_string(s)
     assert loki.loki_status_string(99) == "unknown status"
+
+
+def test_index_bytes(loki):
+    assert loki.loki_index_bytes(10, 8, 32, loki.LOKI_BF16) == 10 * 8 * 16 * 32 * 2
+    assert loki.loki_index_bytes(10, 8, 24, loki.LOKI_BF16) == 0
+    assert loki.loki_index_bytes(10, 8, 0, loki.LOKI_F32) == 0
 
 
 def test_cache_bytes(loki):
@@ -56,8 +62,8 @@ def test_cache_bytes(loki):
 FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
 
 
-def structs(loki, *, D=128, Hkv=8, dtype=1, B=2, max_blocks=4, max_len=64, blocks=8):
-    c = loki.loki_cache(FAKE, FAKE, blocks, Hkv, D, dtype)
+def structs(loki, *, D=128, Hkv=8, dtype=1, B=2, max_blocks=4, max_len=64, blocks=8, index_dims=32):
+    c = loki.loki_cache(FAKE, FAKE, FAKE, blocks, Hkv, D, index_dims, dtype)
     b = loki.loki_batch(FAKE, FAKE, B, max_blocks, max_len)
     return c, b
 
@@ -73,7 +79,7 @@ def decode(loki, c, b, Hq=32, r=32, k=8, W=0, group=0, scale=0.0, q=FAKE, P=FAKE
     (dict(W=-2), 1),
     (dict(r=0), 1),
     (dict(r=129), 1),
-    (dict(r=40), 2),                # not a multiple of 16
+    (dict(r=24), 2),                # not a multiple of 16
     (dict(Hq=30), 1),               # not a multiple of Hkv
     (dict(Hq=24), 2),               # group 3
     (dict(Hq=128), 2),              # group 16
@@ -83,7 +89,8 @@ def decode(loki, c, b, Hq=32, r=32, k=8, W=0, group=0, scale=0.0, q=FAKE, P=FAKE
     (dict(q=None), 1),
     (dict(P=None), 1),
     (dict(out=None), 1),
-    (dict(P=FAKE + 4), 1),          # P must be 16-byte aligned (bulk copy source)
+    (dict(P=FAKE + 4), 1),          # P must be 16-byte aligned (vector loads)
+    (dict(q=FAKE + 8), 1),          # q must be 16-byte aligned (vector loads)
 ])
 def test_decode_rejects(loki, kw, status):
     c, b = structs(loki)
@@ -99,11 +106,18 @@ def test_decode_rejects_bad_shapes(loki):
     assert decode(loki, c, b) == 2         # above the fused kernel's capacity
     c, b = structs(loki, B=-1)
     assert decode(loki, c, b) == 1
-    c = loki.loki_cache(FAKE + 8, FAKE, 8, 8, 128, 1)
+    c = loki.loki_cache(FAKE + 8, FAKE, FAKE, 8, 8, 128, 32, 1)
     _, b = structs(loki)
     assert decode(loki, c, b) == 1         # misaligned cache
-    c = loki.loki_cache(FAKE, FAKE, 8, 8, 128, 7)
+    c = loki.loki_cache(FAKE, FAKE, FAKE + 4, 8, 8, 128, 32, 1)
+    assert decode(loki, c, b) == 1         # misaligned index
+    c = loki.loki_cache(FAKE, FAKE, FAKE, 8, 8, 128, 32, 7)
     assert decode(loki, c, b) == 1         # unknown dtype
+    for bad_index in (0, 8, 24, 144):
+        c = loki.loki_cache(FAKE, FAKE, FAKE, 8, 8, 128, bad_index, 1)
+        assert decode(loki, c, b) == 1, bad_index
+    c, b = structs(loki, index_dims=32)
+    assert decode(loki, c, b, r=48) == 1   # r above the index dims
     assert loki.raw().loki_decode_attention(None, ctypes.byref(b), FAKE, 32, FAKE, 32, 8, None, 0, 0, 0.0,
                                             FAKE, None, None, 0, None) == 1
 

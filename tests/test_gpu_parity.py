@@ -168,20 +168,23 @@ def test_repeat_calls_identical(cuda_lib):
 # ---------------------------------------------------------------------------
 
 def read_pair(dev, b, h, L):
-    """Reads keys and values of one pair back through the documented cache
-    layout: block p of head h at element (p * Hkv + h) * 16 * D; keys as
-    [D/16 slabs][16 tokens][16 dims], values as [16 tokens][D]."""
+    """Reads keys, values and the key index of one pair back through the
+    documented layout: block p of head h at element (p * Hkv + h) * 16 * D in
+    the key and value caches ([16 tokens][D] each) and at (p * Hkv + h) * 16 * I
+    in the key index ([I/16 slabs][16 tokens][16 dims])."""
     s = dev.wl.spec
     dt = synth.torch_dtype(s.dtype)
-    D, Hkv = s.head_dim, s.num_kv_heads
-    kc = dev.cache.k.view(dt).view(-1, Hkv, D // 16, 16, 16)
+    D, Hkv, I = s.head_dim, s.num_kv_heads, dev.cache.index_dims
+    kc = dev.cache.k.view(dt).view(-1, Hkv, 16, D)
     vc = dev.cache.v.view(dt).view(-1, Hkv, 16, D)
+    xc = dev.cache.x.view(dt).view(-1, Hkv, I // 16, 16, 16)
     tbl = dev.wl.block_table[b]
     nblk = (L + 15) // 16
     blocks = tbl[:nblk].long().to(kc.device)
-    K = kc[blocks, h].permute(0, 2, 1, 3).reshape(nblk * 16, D)[:L]
+    K = kc[blocks, h].reshape(nblk * 16, D)[:L]
     V = vc[blocks, h].reshape(nblk * 16, D)[:L]
-    return K.cpu(), V.cpu()
+    X = xc[blocks, h].permute(0, 2, 1, 3).reshape(nblk * 16, I)[:L]
+    return K.cpu(), V.cpu(), X.cpu()
 
 
 def test_prefill_layout(cuda_lib):
@@ -190,8 +193,9 @@ def test_prefill_layout(cuda_lib):
     dev = harness.Device(wl, cuda_lib)
     for b, L in enumerate(s.seq_lens):
         for h in range(2):
-            K, V = read_pair(dev, b, h, L)
+            K, V, X = read_pair(dev, b, h, L)
             assert torch.equal(K, wl.Kt[b, h, :L]) and torch.equal(V, wl.V[b, h, :L])
+            assert torch.equal(X, wl.Kt[b, h, :L, :dev.cache.index_dims])
 
 
 @pytest.mark.parametrize("dtype,D", [("bf16", 128), ("f32", 64), ("bf16", 64)])
@@ -208,7 +212,8 @@ def test_append_matches_oracle(cuda_lib, dtype, D):
     assert cuda_lib.loki_device_error() == 0
     for b, L in enumerate(lens.tolist()):
         for h in range(s.num_kv_heads):
-            K, V = read_pair(dev, b, h, L)
+            K, V, X = read_pair(dev, b, h, L)
+            assert torch.equal(X, K[:, :dev.cache.index_dims])
             assert torch.equal(V[L - 1], v_new[b, h])
             if L > 1:
                 assert torch.equal(K[: L - 1], wl.Kt[b, h, : L - 1])
