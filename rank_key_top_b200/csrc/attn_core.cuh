@@ -148,3 +148,180 @@ __device__ __forceinline__ Merged merge_partials(const float* src, int n, int st
 }
 
 }  // namespace loki
+
+namespace loki {
+
+// ---------------------------------------------------------------------------
+// Tensor-core variant for bf16 caches: the same exact attention (AQUA page,
+// decode-step equations (3)-(5)) with the two contractions of a chunk of 8
+// staged tokens on warp-level MMA (m16n8k16, bf16 inputs, fp32 accumulate):
+//   logits  S[8 tok x 8 col] = K[8 tok x D] . Qt[D x 8 col]
+//   output  Ot[D x 8 col]  += Vt[D x 8 tok] . Pt[8 tok x 8 col]
+// Column n of Qt / Pt is head n/2, part n%2: each fp32 query value (and each
+// softmax weight) is split into a bf16 high part and a bf16 remainder, so the
+// products keep about 16 significant bits and the accumulation is fp32. With
+// G = 8 a second group of 8 columns carries heads 4..7. Rows 8..15 of each
+// m16 tile are unused (8 tokens per chunk).
+//
+// Lane l = 4g + t then owns, after the logits MMA, token g's logit for head
+// t (and t + 4), and after the output MMA, head t's output for dims
+// {16m + g, 16m + g + 8 : m < D/16}: the running max and the rescale of a
+// lane's accumulators concern its own head only.
+//
+// Staging layout of one chunk (written by cp.async): 8 key rows then 8 value
+// rows of D bf16 each; the 16-byte piece c of row r sits at piece c ^ (r & 7)
+// so that every ldmatrix below is free of bank conflicts.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mma_16816_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldmatrix_x2(uint32_t& r0, uint32_t& r1, const void* row_ptr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+                 : "=r"(r0), "=r"(r1)
+                 : "r"(smem_u32(row_ptr)));
+}
+__device__ __forceinline__ void ldmatrix_x2_trans(uint32_t& r0, uint32_t& r1, const void* row_ptr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
+                 : "=r"(r0), "=r"(r1)
+                 : "r"(smem_u32(row_ptr)));
+}
+// bf16 pair {lo16 = a, hi16 = b}
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+    const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(a));
+    const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(b));
+    return lo | (hi << 16);
+}
+// high (part 0) or remainder (part 1) of x in bf16
+__device__ __forceinline__ float split_part(float x, int part) {
+    const float h = __bfloat162float(__float2bfloat16_rn(x));
+    return part ? x - h : h;
+}
+
+template <int D, int G>
+struct MmaAttnCore {
+    static constexpr int NCH = 8;              // tokens per chunk
+    static constexpr int KS = D / 16;          // k-steps of the logits MMA, m-tiles of the output MMA
+    static constexpr int NG = G > 4 ? 2 : 1;   // column groups of 8 (4 heads each)
+    static constexpr int ROWB = D * 2;         // bytes of one staged row
+    static constexpr int CHUNK_BYTES = 2 * NCH * ROWB;
+
+    uint32_t qb[NG][KS][2];   // Qt fragments (scale * log2(e) folded in)
+    float acc[NG][KS][4];     // Ot accumulators
+    float m[NG];              // running max of this lane's head (per column group)
+    float l[NG];              // this lane's running sum of weights (its token g)
+
+    // byte offset of piece c of staged row r (key rows: kv = 0, value rows: kv = 1)
+    static __device__ __forceinline__ int staged_offset(int kv, int r, int c) {
+        return kv * NCH * ROWB + r * ROWB + ((c ^ (r & 7)) << 4);
+    }
+
+    __device__ __forceinline__ void init(const float* qhat, float scale_log2, int lane) {
+        const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+        for (int ng = 0; ng < NG; ++ng) {
+            const int head = ng * 4 + (g >> 1);
+            const int part = g & 1;
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                float v[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int d = ks * 16 + 2 * t + (e & 1) + (e >> 1) * 8;
+                    v[e] = head < G ? split_part(qhat[head * D + d] * scale_log2, part) : 0.f;
+                }
+                qb[ng][ks][0] = pack_bf16(v[0], v[1]);
+                qb[ng][ks][1] = pack_bf16(v[2], v[3]);
+            }
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks)
+                acc[ng][ks][0] = acc[ng][ks][1] = acc[ng][ks][2] = acc[ng][ks][3] = 0.f;
+            m[ng] = -INFINITY;
+            l[ng] = 0.f;
+        }
+    }
+
+    // One staged chunk; token n is present iff bit n of `valid` (absent rows
+    // are zero-filled by the staging copy).
+    __device__ __forceinline__ void consume(const unsigned char* chunk, uint32_t valid, int lane) {
+        const int g = lane >> 2, t = lane & 3;
+        // ldmatrix row addresses: lanes 0-7 rows 0-7 of piece 2s, lanes 8-15 of piece 2s+1
+        const int lr = lane & 7, lh = (lane >> 3) & 1;
+        float z[NG];
+#pragma unroll
+        for (int ng = 0; ng < NG; ++ng) {
+            float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                uint32_t a0, a2;
+                ldmatrix_x2(a0, a2, chunk + staged_offset(0, lr, 2 * ks + lh));
+                mma_16816_bf16(s, a0, 0u, a2, 0u, qb[ng][ks][0], qb[ng][ks][1]);
+            }
+            z[ng] = s[0] + s[1];  // token g, head 4 ng + t: high part + remainder
+        }
+        const bool ok = (valid >> g) & 1u;
+        float p[NG], alpha[NG];
+#pragma unroll
+        for (int ng = 0; ng < NG; ++ng) {
+            const float zz = ok ? z[ng] : -INFINITY;
+            float cm = zz;
+            cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 4));
+            cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 8));
+            cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 16));
+            const float m_new = fmaxf(m[ng], cm);
+            alpha[ng] = (m_new == -INFINITY) ? 1.f : exp2f(m[ng] - m_new);
+            p[ng] = ok ? exp2f(zz - m_new) : 0.f;
+            m[ng] = m_new;
+            l[ng] = l[ng] * alpha[ng] + p[ng];
+        }
+        // Pt fragments: lane needs weights of tokens 2t, 2t+1 for column g
+#pragma unroll
+        for (int ng = 0; ng < NG; ++ng) {
+            const int src = (g >> 1);
+            const float pa = __shfl_sync(kFull, p[ng], 4 * (2 * t) + src);
+            const float pb = __shfl_sync(kFull, p[ng], 4 * (2 * t + 1) + src);
+            const uint32_t b0 = pack_bf16(split_part(pa, g & 1), split_part(pb, g & 1));
+            const bool rescale = __any_sync(kFull, alpha[ng] != 1.f);
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
+                if (rescale) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[ng][mt][e] *= alpha[ng];
+                }
+                uint32_t a0, a1;
+                ldmatrix_x2_trans(a0, a1, chunk + staged_offset(1, lr, 2 * mt + lh));
+                mma_16816_bf16(acc[ng][mt], a0, a1, 0u, 0u, b0, 0u);
+            }
+        }
+    }
+
+    // This warp's partial (o[D], m, l per head) to dst[G][D + 2].
+    __device__ __forceinline__ void store_partial(float* dst, int lane) {
+        const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+        for (int ng = 0; ng < NG; ++ng) {
+            const int head = ng * 4 + t;
+            float lt = l[ng];
+            lt += __shfl_xor_sync(kFull, lt, 4);
+            lt += __shfl_xor_sync(kFull, lt, 8);
+            lt += __shfl_xor_sync(kFull, lt, 16);
+            if (head < G) {
+#pragma unroll
+                for (int mt = 0; mt < KS; ++mt) {
+                    dst[head * (D + 2) + mt * 16 + g] = acc[ng][mt][0] + acc[ng][mt][1];
+                    dst[head * (D + 2) + mt * 16 + g + 8] = acc[ng][mt][2] + acc[ng][mt][3];
+                }
+                if (g == 0) {
+                    dst[head * (D + 2) + D] = m[ng];
+                    dst[head * (D + 2) + D + 1] = lt;
+                }
+            }
+        }
+    }
+};
+
+}  // namespace loki

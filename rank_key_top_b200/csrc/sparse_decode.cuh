@@ -31,6 +31,8 @@
 
 #include <cooperative_groups.h>
 
+#include <type_traits>
+
 #include "attn_core.cuh"
 
 namespace loki {
@@ -85,8 +87,11 @@ struct SparseParams {
 #endif
 template <typename T, int D, int G>
 struct SparseGeom {
+    // bf16 caches: tensor-core attention on 8-token chunks; fp32: CUDA cores
+    static constexpr bool MMA = std::is_same<T, __nv_bfloat16>::value;
     using Core = AttnCore<T, D, G, (LOKI_GATHER_CHUNK * G > 32 ? 32 / G : LOKI_GATHER_CHUNK)>;
-    static constexpr int NCH = Core::NCH;
+    using MCore = MmaAttnCore<D, G>;
+    static constexpr int NCH = MMA ? MCore::NCH : Core::NCH;
     static constexpr int TB = 2 * D * (int)sizeof(T);  // key row + value row bytes
     static constexpr int CHUNK_BYTES = NCH * TB;
     static constexpr int GS_FIT = (160 * 1024) / (kWarps * CHUNK_BYTES);
@@ -647,53 +652,73 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     {
         const unsigned char* kbytes = reinterpret_cast<const unsigned char*>(p.k_cache);
         const unsigned char* vbytes = reinterpret_cast<const unsigned char*>(p.v_cache);
-        constexpr int PIECES = TB / 16;
         constexpr int ROWB = D * (int)sizeof(T);
+        constexpr int PIECES = TB / 16;  // 16-byte pieces of one token (key row + value row)
         unsigned char* wst = stage + warp * GS * Geom::CHUNK_BYTES;
         const int nchunks = (n_list + NCH - 1) / NCH;
         const int my_n = nchunks > warp ? (nchunks - warp + kWarps - 1) / kWarps : 0;
+        // stage chunk m of this warp (tokens list[ch*NCH .. ch*NCH+NCH)) into slot m % GS
         auto fetch = [&](int m) {
             if (m < my_n) {
                 unsigned char* dst = wst + (m % GS) * Geom::CHUNK_BYTES;
                 const int ch = warp + m * kWarps;
                 for (int pc = lane; pc < NCH * PIECES; pc += 32) {
-                    const int n = pc / PIECES, o = (pc - n * PIECES) * 16;
+                    const int n = pc / PIECES, w = pc - n * PIECES;
+                    const int kv = w >= PIECES / 2, c = w - kv * (PIECES / 2);
                     const int idx = ch * NCH + n;
                     const bool ok = idx < n_list;
                     const unsigned char* src = kbytes;
                     if (ok) {
                         const int li = list[idx];
                         const int64_t at = page_offset(tbl[li >> 4], h, p.Hkv, D) * (int64_t)sizeof(T) +
-                                           (int64_t)(li & 15) * ROWB;
-                        src = o < ROWB ? kbytes + at + o : vbytes + at + (o - ROWB);
+                                           (int64_t)(li & 15) * ROWB + c * 16;
+                        src = (kv ? vbytes : kbytes) + at;
                     }
-                    cp_async16(dst + n * TB + o, src, ok);
+                    int off;
+                    if constexpr (Geom::MMA) off = Geom::MCore::staged_offset(kv, n, c);
+                    else off = n * TB + kv * ROWB + c * 16;
+                    cp_async16(dst + off, src, ok);
                 }
             }
             cp_async_commit();
         };
-        Core core;
-        core.init(qhat, p.scale_log2, lane);
-        for (int m = 0; m < GS - 1; ++m) fetch(m);
-        for (int m = 0; m < my_n; ++m) {
-            fetch(m + GS - 1);
-            cp_async_wait<GS - 1>();
-            __syncwarp();
-            const unsigned char* src = wst + (m % GS) * Geom::CHUNK_BYTES;
-            typename Core::raw_t kr[NCH], vr[NCH];
-            uint32_t valid = 0;
+        auto run = [&](auto& core) {
+            for (int m = 0; m < GS - 1; ++m) fetch(m);
+            for (int m = 0; m < my_n; ++m) {
+                fetch(m + GS - 1);
+                cp_async_wait<GS - 1>();
+                __syncwarp();
+                const unsigned char* src = wst + (m % GS) * Geom::CHUNK_BYTES;
+                uint32_t valid = 0;
 #pragma unroll
-            for (int n = 0; n < NCH; ++n) {
-                kr[n] = Core::V::load(reinterpret_cast<const T*>(src + n * TB) + lane * Core::DPL);
-                vr[n] = Core::V::load(reinterpret_cast<const T*>(src + n * TB + ROWB) + lane * Core::DPL);
-                if ((warp + m * kWarps) * NCH + n < n_list) valid |= 1u << n;
+                for (int n = 0; n < NCH; ++n)
+                    if ((warp + m * kWarps) * NCH + n < n_list) valid |= 1u << n;
+                if constexpr (Geom::MMA) {
+                    core.consume(src, valid, lane);
+                } else {
+                    typename Core::raw_t kr[NCH], vr[NCH];
+#pragma unroll
+                    for (int n = 0; n < NCH; ++n) {
+                        kr[n] = Core::V::load(reinterpret_cast<const T*>(src + n * TB) + lane * Core::DPL);
+                        vr[n] = Core::V::load(reinterpret_cast<const T*>(src + n * TB + ROWB) + lane * Core::DPL);
+                    }
+                    core.consume(kr, vr, valid, lane);
+                }
+                __syncwarp();
             }
-            core.consume(kr, vr, valid, lane);
-            __syncwarp();
+            cp_async_wait<0>();
+            __syncthreads();  // every warp is done with the staging area
+            core.store_partial(wpart + warp * G * (D + 2), lane);
+        };
+        if constexpr (Geom::MMA) {
+            typename Geom::MCore core;
+            core.init(qhat, p.scale_log2, lane);
+            run(core);
+        } else {
+            Core core;
+            core.init(qhat, p.scale_log2, lane);
+            run(core);
         }
-        cp_async_wait<0>();
-        __syncthreads();  // every warp is done with the staging area
-        core.store_partial(wpart + warp * G * (D + 2), lane);
     }
     __syncthreads();
 
