@@ -215,6 +215,33 @@ LOKI_API loki_status loki_dense_attention(const loki_cache* cache, const loki_ba
                                  float scale, float* out, void* workspace,
                                  size_t workspace_bytes, loki_stream_t stream);
 
+/* Size of the scratch array built into the library for
+ * loki_dense_attention_static (16 MiB). */
+#define LOKI_DENSE_STATIC_SCRATCH_BYTES (16u << 20)
+
+/* loki_dense_attention for callers that cannot allocate device memory: a
+ * serving engine that hands all device memory to its own arena at start-up,
+ * a plugin host that exposes no allocator, or code that must not call
+ * cudaMalloc because it can synchronise the device. This is an addition of
+ * the library, not a step of the method, so no page has a counterpart.
+ *
+ * Same arguments and result as loki_dense_attention, without the workspace:
+ * the split partials go to a scratch array inside the library
+ * (LOKI_DENSE_STATIC_SCRATCH_BYTES; every GPU that loads the library holds it
+ * until the process exits). The call allocates nothing.
+ *  - Sizes whose loki_dense_workspace_bytes exceeds the array are rejected
+ *    with LOKI_ERR_WORKSPACE before anything is launched.
+ *  - The first call on a device looks up the array's device address (once per
+ *    device, with that device current); make that first call before any
+ *    stream capture on the device.
+ *  - All calls on a device share the one array, which keeps the last call's
+ *    contents (every value a call reads it writes first, so nothing needs
+ *    clearing). Calls whose executions overlap on the GPU (different streams
+ *    without ordering) race on the array and must not be issued that way. */
+LOKI_API loki_status loki_dense_attention_static(const loki_cache* cache, const loki_batch* batch,
+                                                 const void* q, int32_t num_q_heads, const float* P,
+                                                 float scale, float* out, loki_stream_t stream);
+
 /* Reads (and with clear != 0 resets) the device error word of the current
  * device: an OR of LOKI_DEVERR_* bits set by kernels since the last clear.
  * Synchronises the device. */

@@ -488,3 +488,50 @@ loki_status loki_dense_attention(const loki_cache* cache, const loki_batch* batc
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Dense decode attention with the library's own scratch, for callers that
+// cannot allocate device memory. The scratch is a file-scope device array, so
+// every GPU that loads the library holds LOKI_DENSE_STATIC_SCRATCH_BYTES of
+// it until the process exits; all calls on a device share it.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_dense_static_scratch[LOKI_DENSE_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of the static scratch on the current device. In host code
+// the array's name is only a host-side stand-in, so the address is taken
+// once per device with cudaGetSymbolAddress (with that device current).
+loki_status static_scratch_address(void** out) {
+    static std::mutex mu;
+    static std::map<int, void*> addr;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LOKI_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = addr.find(dev);
+    if (it == addr.end()) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_dense_static_scratch) != cudaSuccess || ptr == nullptr) {
+            cudaGetLastError();
+            return LOKI_ERR_CUDA;
+        }
+        it = addr.emplace(dev, ptr).first;
+    }
+    *out = it->second;
+    return LOKI_OK;
+}
+
+}  // namespace
+
+extern "C" loki_status loki_dense_attention_static(const loki_cache* cache, const loki_batch* batch, const void* q,
+                                                   int32_t num_q_heads, const float* P, float scale, float* out,
+                                                   loki_stream_t stream) {
+    void* scratch = nullptr;
+    loki_status st = static_scratch_address(&scratch);
+    if (st != LOKI_OK) return st;
+    if (check_cache(cache) == LOKI_OK && check_batch(batch) == LOKI_OK && num_q_heads >= 1 &&
+        loki_dense_workspace_bytes(cache, batch, num_q_heads) > (size_t)LOKI_DENSE_STATIC_SCRATCH_BYTES)
+        return LOKI_ERR_WORKSPACE;  // these sizes need more scratch than the built-in array holds
+    return loki_dense_attention(cache, batch, q, num_q_heads, P, scale, out, scratch,
+                                (size_t)LOKI_DENSE_STATIC_SCRATCH_BYTES, stream);
+}

@@ -29,6 +29,8 @@ LOKI_DEVERR_BLOCK_ID = 0x2
 LOKI_DEVERR_K = 0x4
 LOKI_DEVERR_TIMEOUT = 0x8
 
+LOKI_DENSE_STATIC_SCRATCH_BYTES = 16 << 20
+
 BLOCK_TOKENS = 16
 
 if not os.path.exists(LIB_PATH):
@@ -65,6 +67,7 @@ _SIGS = {
     "loki_decode_max_seq_len": (_I32, [_I32, ctypes.c_int]),
     "loki_dense_workspace_bytes": (_SZ, [_C, _B, _I32]),
     "loki_dense_attention": (ctypes.c_int, [_C, _B, _P, _I32, _P, ctypes.c_float, _P, _P, _SZ, _P]),
+    "loki_dense_attention_static": (ctypes.c_int, [_C, _B, _P, _I32, _P, ctypes.c_float, _P, _P]),
     "loki_device_error": (ctypes.c_int, [_I32, ctypes.POINTER(ctypes.c_uint32)]),
     "loki_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "loki_abi_version": (_I32, []),
@@ -193,6 +196,13 @@ def loki_dense_attention(cache, batch, q, P, out, workspace, scale=0.0, stream=N
     _check("loki_dense_attention", _lib.loki_dense_attention(
         ctypes.byref(cache.struct), ctypes.byref(batch.struct), _ptr(q), q.shape[1], _ptr(P), scale,
         _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def loki_dense_attention_static(cache, batch, q, P, out, scale=0.0, stream=None):
+    """Dense attention with the library's built-in scratch (no workspace)."""
+    _check("loki_dense_attention_static", _lib.loki_dense_attention_static(
+        ctypes.byref(cache.struct), ctypes.byref(batch.struct), _ptr(q), q.shape[1], _ptr(P), scale,
+        _ptr(out), _stream(stream)))
 
 
 def loki_device_error(clear=True):
