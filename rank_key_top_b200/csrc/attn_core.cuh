@@ -190,6 +190,12 @@ __device__ __forceinline__ void ldmatrix_x2_trans(uint32_t& r0, uint32_t& r1, co
                  : "=r"(r0), "=r"(r1)
                  : "r"(smem_u32(row_ptr)));
 }
+__device__ __forceinline__ void ldmatrix_x4(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3,
+                                            const void* row_ptr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(smem_u32(row_ptr)));
+}
 // bf16 pair {lo16 = a, hi16 = b}
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(a));

@@ -124,6 +124,7 @@ __device__ __forceinline__ int warp_exclusive_scan(int v, int lane) {
 }
 
 // Exclusive suffix sum over the block: returns sum of v over threads > tid.
+// wsum: 2 * kWarps words of shared scratch.
 __device__ __forceinline__ uint32_t block_suffix_exclusive(uint32_t v, uint32_t* wsum, int lane, int warp) {
     uint32_t x = v;
 #pragma unroll
@@ -131,12 +132,20 @@ __device__ __forceinline__ uint32_t block_suffix_exclusive(uint32_t v, uint32_t*
         const uint32_t y = __shfl_down_sync(kFull, x, o);
         if (lane + o < 32) x += y;
     }
-    if (lane == 0) wsum[warp] = x;
+    if (lane == 0) wsum[warp] = x;  // warp total
     __syncthreads();
-    uint32_t other = 0;
-    for (int w = warp + 1; w < kWarps; ++w) other += wsum[w];
+    if (warp == 0) {  // suffix over the warp totals, excluding the warp itself
+        uint32_t t = lane < kWarps ? wsum[lane] : 0u;
+        uint32_t s = t;
+#pragma unroll
+        for (int o = 1; o < kWarps; o <<= 1) {
+            const uint32_t y = __shfl_down_sync(kFull, s, o);
+            if (lane + o < kWarps) s += y;
+        }
+        if (lane < kWarps) wsum[kWarps + lane] = s - t;
+    }
     __syncthreads();
-    return x - v + other;
+    return x - v + wsum[kWarps + warp];
 }
 
 template <typename T, int D, int G>
@@ -170,9 +179,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bars);
     float* part = reinterpret_cast<float*>(smem + p.off_part);
     int32_t* misc = reinterpret_cast<int32_t*>(smem + p.off_misc);
-    // misc: [0] boundary digit, [1] count above it, [8..23] warp sums,
-    //       [32..47] warp kept counts, [48..63] warp equal counts, [64] list
-    //       length, [66] candidate count, [80..95] warp counts above digit 0
+    // misc: [0] boundary digit, [1] count above it, [8..39] suffix-sum scratch,
+    //       [40..55] warp kept counts, [56..71] warp equal counts, [72] list length
 
     // ---- sequence geometry (identical in every CTA of the cluster) ----
     int L = p.seq_lens[b];
@@ -226,11 +234,15 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
 #pragma unroll
     for (int j = 0; j < G; ++j) qraw[j] = Vec<T, RPG>::load(qg + j * D + rg * RPG);
 
-    if (tid == 0) {
-        for (int i = 0; i < kWarps * kMaxSlots; ++i) mbar_init(&bars[i], 1);
+    // each warp owns its ring's barriers: it starts its key-index stream as
+    // soon as its block-table entries arrive, before any CTA-wide barrier
+    unsigned char* wring = ring + warp * p.ring_bytes_per_warp;
+    uint64_t* wbar = bars + warp * kMaxSlots;
+    if (lane == 0) {
+        for (int i = 0; i < kMaxSlots; ++i) mbar_init(&wbar[i], 1);
         fence_mbarrier_init();
     }
-    for (int i = tid; i < 2 * kHistBins; i += kThreads) hist[i] = 0;
+    __syncwarp();
     auto checked = [&](int pb) {
         if (pb < 0 || pb >= p.num_blocks) {
             flag_error(LOKI_DEVERR_BLOCK_ID);
@@ -240,15 +252,6 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     };
     tb0 = checked(tb0);
     tb1 = checked(tb1);
-    {
-        const int j0 = warp + lane * kWarps, j1 = warp + (lane + 32) * kWarps;
-        if (j0 < nblk_loc) tbl[j0] = tb0;
-        if (j1 < nblk_loc) tbl[j1] = tb1;
-    }
-    __syncthreads();
-
-    unsigned char* wring = ring + warp * p.ring_bytes_per_warp;
-    uint64_t* wbar = bars + warp * kMaxSlots;
     const int my_blocks = nblk_score > warp ? (nblk_score - warp + kWarps - 1) / kWarps : 0;
     const unsigned char* xbytes = reinterpret_cast<const unsigned char*>(p.k_index);
     auto issue = [&](int it, int pb) {  // lane 0 only
@@ -269,6 +272,13 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
             if (lane == 0) issue(it, pb);
         }
     }
+    for (int i = tid; i < 2 * kHistBins; i += kThreads) hist[i] = 0;
+    {
+        const int j0 = warp + lane * kWarps, j1 = warp + (lane + 32) * kWarps;
+        if (j0 < nblk_loc) tbl[j0] = tb0;
+        if (j1 < nblk_loc) tbl[j1] = tb1;
+    }
+    __syncthreads();
 
     {   // q_hat = q P[h]: each thread sums its RPG rows for its 4 columns
         float qv[G][RPG];
@@ -310,12 +320,94 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     }
 
     // ---- 2. rank-r scoring ----
-    // A warp takes kScoreBlocks blocks per iteration: their slots are read into
-    // registers and handed back to the bulk-copy engine before the arithmetic,
-    // and the blocks' dot products run as independent chains.
+    // A warp takes one block per iteration: its slot is read into registers and
+    // handed back to the bulk-copy engine before the arithmetic. bf16 index:
+    // the 16 x 16 tile of each slab (16 tokens x 16 dims) times a fragment whose
+    // columns hold the score vector split into bf16 high part and remainder
+    // (SUM: the summed query in columns 0, 1; MAX: q_hat_j in columns 2j, 2j+1,
+    // a second column group for heads 4..7), on warp-level MMA with fp32
+    // accumulation. fp32 index: CUDA-core dot products.
     {
         bool failed = false;
-        // RMAX: compile-time bound on the slabs per block; R16 <= RMAX at run time
+        auto mma_body = [&](auto rmax_tag) {
+            constexpr int RMAX = decltype(rmax_tag)::value;
+            constexpr int SG = G > 4 ? 2 : 1;
+            const int R16 = p.r / kSlabDims;
+            const int g = lane >> 2, t = lane & 3;
+            const int ngroups = p.group_max ? SG : 1;
+            uint32_t qb[SG][RMAX][2];
+#pragma unroll
+            for (int ng = 0; ng < SG; ++ng)
+#pragma unroll
+                for (int sb = 0; sb < RMAX; ++sb) {
+                    float v[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int d = sb * 16 + 2 * t + (e & 1) + (e >> 1) * 8;
+                        float x = 0.f;
+                        if (sb < R16) {
+                            if (!p.group_max) {
+                                x = (ng == 0 && g < 2) ? split_part(qs[d], g & 1) : 0.f;
+                            } else {
+                                const int head = ng * 4 + (g >> 1);
+                                x = head < G ? split_part(qhat[head * D + d], g & 1) : 0.f;
+                            }
+                        }
+                        v[e] = x;
+                    }
+                    qb[ng][sb][0] = pack_bf16(v[0], v[1]);
+                    qb[ng][sb][1] = pack_bf16(v[2], v[3]);
+                }
+            const int arow = (lane & 7) + 8 * ((lane >> 3) & 1), ahalf = lane >> 4;
+            for (int it = 0; it < my_blocks; ++it) {
+                const int slot = it % S;
+                const uint32_t parity = (uint32_t)(it / S) & 1u;
+                if (!failed) failed = __any_sync(kFull, !mbar_wait_bounded(&wbar[slot], parity));
+                const unsigned char* sl = wring + slot * p.slot_bytes;
+                uint32_t a[RMAX][4];
+#pragma unroll
+                for (int sb = 0; sb < RMAX; ++sb)
+                    if (sb < R16) ldmatrix_x4(a[sb][0], a[sb][1], a[sb][2], a[sb][3], sl + sb * 512 + arow * 32 + ahalf * 16);
+                __syncwarp();
+                if (it + S < my_blocks) {
+                    const int pb = entry(it + S);
+                    if (lane == 0) issue(it + S, pb);
+                }
+                float sc0 = -INFINITY, sc1 = -INFINITY;  // tokens g and g + 8
+#pragma unroll
+                for (int ng = 0; ng < SG; ++ng) {
+                    if (ng < ngroups) {
+                        float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                        for (int sb = 0; sb < RMAX; ++sb)
+                            if (sb < R16) mma_16816_bf16(c, a[sb][0], a[sb][1], a[sb][2], a[sb][3], qb[ng][sb][0], qb[ng][sb][1]);
+                        float h0 = c[0] + c[1], h1 = c[2] + c[3];  // column pair t: head 4 ng + t (MAX) / qs (SUM, t = 0)
+                        if (p.group_max) {
+                            if (ng * 4 + t >= G) h0 = h1 = -INFINITY;
+                            h0 = fmaxf(h0, __shfl_xor_sync(kFull, h0, 1));
+                            h0 = fmaxf(h0, __shfl_xor_sync(kFull, h0, 2));
+                            h1 = fmaxf(h1, __shfl_xor_sync(kFull, h1, 1));
+                            h1 = fmaxf(h1, __shfl_xor_sync(kFull, h1, 2));
+                        }
+                        sc0 = fmaxf(sc0, h0);
+                        sc1 = fmaxf(sc1, h1);
+                    }
+                }
+                if (t == 0) {
+                    const int base = (warp + it * kWarps) * kBlockTokens;
+                    if (base + g < n_cand_loc) {
+                        const uint32_t key = score_key(sc0);
+                        keys[base + g] = key;
+                        atomicAdd(&hist[key >> 21], 1u);
+                    }
+                    if (base + g + 8 < n_cand_loc) {
+                        const uint32_t key = score_key(sc1);
+                        keys[base + g + 8] = key;
+                        atomicAdd(&hist[key >> 21], 1u);
+                    }
+                }
+            }
+        };
         auto body = [&](auto rmax_tag) {
             constexpr int RMAX = decltype(rmax_tag)::value;
             const int R16 = p.r / kSlabDims;
@@ -412,25 +504,37 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
                 }
             }
         };
-        if (p.r <= 2 * kSlabDims)
-            body(std::integral_constant<int, 2>{});
-        else
-            body(std::integral_constant<int, D / kSlabDims>{});
+        if constexpr (Geom::MMA) {
+            if (p.r <= 2 * kSlabDims)
+                mma_body(std::integral_constant<int, 2>{});
+            else
+                mma_body(std::integral_constant<int, D / kSlabDims>{});
+        } else {
+            if (p.r <= 2 * kSlabDims)
+                body(std::integral_constant<int, 2>{});
+            else
+                body(std::integral_constant<int, D / kSlabDims>{});
+        }
     }
     __syncthreads();
 
     // ---- 3. top-k over the cluster ----
     // mode 0: keep every candidate, 1: keep none, 2: threshold tau / quota.
-    // Warp w owns the contiguous key range [lo, hi) in every scan below.
+    // From here on lane l of warp w holds the keys w*32*KPL + 32 m + l (m < KPL)
+    // in registers, KPL = ceil(cta_tokens / threads) <= 32: every pass below
+    // reads registers, and the kept list comes out in index order.
     const int mode = keff >= ncand ? 0 : (keff == 0 ? 1 : 2);
-    const int per_warp = (((n_cand_loc + kWarps - 1) / kWarps) + 127) & ~127;
-    const int lo = min(warp * per_warp, n_cand_loc);
-    const int hi = min(lo + per_warp, n_cand_loc);
-    const uint4* k4 = reinterpret_cast<const uint4*>(keys);
-    uint2* cand = reinterpret_cast<uint2*>(ring);  // (key, local index) of boundary-bin keys
+    const int KPL = (p.cta_tokens + kThreads - 1) / kThreads;
+    const int wbase = warp * 32 * KPL;
+    uint32_t kr[32];
+#pragma unroll
+    for (int m = 0; m < 32; ++m) {
+        const int i = wbase + 32 * m + lane;
+        kr[m] = (m < KPL && i < n_cand_loc) ? keys[i] : 0u;
+    }
+    auto valid_at = [&](int m) { return m < KPL && wbase + 32 * m + lane < n_cand_loc; };
     uint32_t tau = 0;
     int quota = 0;
-    bool counted = false;  // per-warp kept / equal counts already in misc[32..63]
     if (mode == 2) {
         // Sum the cluster's histograms (buffer hcur) and find the digit where
         // the count from the top reaches krem; returns (digit, count above it).
@@ -470,70 +574,21 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
         const int2 d0 = boundary(hist, 2048, keff);
         const uint32_t beta0 = (uint32_t)d0.x;
         int krem = keff - d0.y;
-        // digit 1: one scan of the keys counts the keys above the boundary
-        // bin per warp and copies the boundary bin's keys to the candidate
-        // buffer (unless there are too many: then later passes rescan keys)
-        const bool use_buf = (int)hist[beta0] <= p.cand_cap;
+        // digit 1 (next 11 bits) over the keys in the boundary bin
         uint32_t* h1 = hist + kHistBins;
-        if (tid == 0) misc[66] = 0;
-        __syncthreads();
-        {
-            int gt0 = 0;
-            for (int base = lo; base < hi; base += 128) {
-                const int i0 = base + lane * 4;
-                const uint4 v = i0 < hi ? k4[i0 / 4] : make_uint4(0u, 0u, 0u, 0u);
-                const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
-                bool isc[4];
-                int nc = 0;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const bool in = i0 + j < hi;
-                    const uint32_t dg = kk[j] >> 21;
-                    gt0 += in && dg > beta0;
-                    isc[j] = in && dg == beta0;
-                    nc += isc[j];
-                    if (isc[j]) atomicAdd(&h1[(kk[j] >> 10) & 2047u], 1u);
-                }
-                if (use_buf) {
-                    const unsigned any = __ballot_sync(kFull, nc > 0);
-                    if (any) {
-                        const int pre = warp_exclusive_scan(nc, lane);
-                        const int tot = __shfl_sync(kFull, pre + nc, 31);
-                        int at = 0;
-                        if (lane == 0) at = atomicAdd(&misc[66], tot);
-                        at = __shfl_sync(kFull, at, 0) + pre;
-#pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            if (isc[j]) cand[at++] = make_uint2(kk[j], (uint32_t)(i0 + j));
-                    }
-                }
-            }
-            gt0 = __reduce_add_sync(kFull, gt0);
-            if (lane == 0) misc[80 + warp] = gt0;
-        }
+        for (int m = 0; m < 32; ++m)
+            if (valid_at(m) && (kr[m] >> 21) == beta0) atomicAdd(&h1[(kr[m] >> 10) & 2047u], 1u);
         const int2 d1 = boundary(h1, 2048, krem);
         const uint32_t beta1 = (uint32_t)d1.x;
         krem -= d1.y;
-        // digit 2 (last 10 bits), over the candidates only
-        for (int i = tid; i < kHistBins; i += kThreads) hist[i] = 0;  // readers of digit 0 are done
+        // digit 2 (last 10 bits) into buffer 0, whose readers are all done
+        for (int i = tid; i < kHistBins; i += kThreads) hist[i] = 0;
         __syncthreads();
         const uint32_t pre22 = (beta0 << 21) | (beta1 << 10);
-        const int ncb = misc[66];
-        if (use_buf) {
-            for (int i = tid; i < ncb; i += kThreads) {
-                const uint32_t kk = cand[i].x;
-                if ((kk & 0xFFFFFC00u) == pre22) atomicAdd(&hist[kk & 1023u], 1u);
-            }
-        } else {
-            const int n4 = (n_cand_loc + 3) / 4;
-            for (int qd = tid; qd < n4; qd += kThreads) {
-                const uint4 v = k4[qd];
-                const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    if (4 * qd + j < n_cand_loc && (kk[j] & 0xFFFFFC00u) == pre22) atomicAdd(&hist[kk[j] & 1023u], 1u);
-            }
-        }
+        for (int m = 0; m < 32; ++m)
+            if (valid_at(m) && (kr[m] & 0xFFFFFC00u) == pre22) atomicAdd(&hist[kr[m] & 1023u], 1u);
         const int2 d2 = boundary(hist, 1024, krem);
         tau = pre22 | (uint32_t)d2.x;
         krem -= d2.y;
@@ -542,51 +597,34 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
         for (int c = 0; c < crank; ++c) eq_before += (int)cluster.map_shared_rank(hist, c)[tau & 1023u];
         const int eq_mine = (int)hist[tau & 1023u];
         quota = min(max(krem - eq_before, 0), eq_mine);
-        // per-warp kept / equal counts from the candidates
-        if (use_buf) {
-            if (tid < 2 * kWarps) misc[32 + tid] = 0;
-            __syncthreads();
-            for (int i = tid; i < ncb; i += kThreads) {
-                const uint2 e = cand[i];
-                const int w = (int)e.y / per_warp;
-                if (e.x > tau) atomicAdd(&misc[32 + w], 1);
-                else if (e.x == tau) atomicAdd(&misc[48 + w], 1);
-            }
-            __syncthreads();
-            if (tid < kWarps) misc[32 + tid] += misc[80 + tid];
-            counted = true;
-        }
     }
 
     // ---- compaction of the kept local tokens into `list`, ascending ----
+    // Bit m of a lane's masks marks its key m (index wbase + 32 m + lane). 32
+    // ballots transpose the masks, so that lane r holds row r (keys wbase +
+    // 32 r + b, b = 0..31); rows in lane order, bits in order, are index order.
     {
-        auto classify = [&](int i0, bool (&gt)[4], bool (&eq)[4]) {
-            const uint4 v = i0 < hi ? k4[i0 / 4] : make_uint4(0u, 0u, 0u, 0u);
-            const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
+        uint32_t gtm = 0u, eqm = 0u;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const bool in = i0 + j < hi;
-                gt[j] = in && (mode == 0 || (mode == 2 && kk[j] > tau));
-                eq[j] = in && mode == 2 && kk[j] == tau;
-            }
-        };
-        if (!counted) {
-            int cgt = 0, ceq = 0;
-            for (int base = lo; base < hi; base += 128) {
-                bool gt[4], eq[4];
-                classify(base + lane * 4, gt, eq);
+        for (int m = 0; m < 32; ++m) {
+            const bool v = valid_at(m);
+            gtm |= (uint32_t)(v && (mode == 0 || (mode == 2 && kr[m] > tau))) << m;
+            eqm |= (uint32_t)(v && mode == 2 && kr[m] == tau) << m;
+        }
+        const int ngt = __reduce_add_sync(kFull, __popc(gtm));
+        const int neq = __reduce_add_sync(kFull, __popc(eqm));
+        if (lane == 0) {
+            misc[40 + warp] = ngt;
+            misc[56 + warp] = neq;
+        }
+        uint32_t rowgt = 0u, roweq = 0u;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    cgt += gt[j];
-                    ceq += eq[j];
-                }
-            }
-            cgt = __reduce_add_sync(kFull, cgt);
-            ceq = __reduce_add_sync(kFull, ceq);
-            __syncthreads();
-            if (lane == 0) {
-                misc[32 + warp] = cgt;
-                misc[48 + warp] = ceq;
+        for (int m = 0; m < 32; ++m) {
+            const uint32_t bg = __ballot_sync(kFull, (gtm >> m) & 1u);
+            const uint32_t be = __ballot_sync(kFull, (eqm >> m) & 1u);
+            if (lane == m) {
+                rowgt = bg;
+                roweq = be;
             }
         }
         __syncthreads();
@@ -594,50 +632,34 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
         // among the CTA's equal keys (in index order) is below the quota
         int eq_base = 0, out_base = 0, total = 0, eb = 0;
         for (int w = 0; w < kWarps; ++w) {
-            const int take = min(max(quota - eb, 0), misc[48 + w]);
+            const int take = min(max(quota - eb, 0), misc[56 + w]);
             if (w < warp) {
-                out_base += misc[32 + w] + take;
-                eq_base += misc[48 + w];
+                out_base += misc[40 + w] + take;
+                eq_base += misc[56 + w];
             }
-            total += misc[32 + w] + take;
-            eb += misc[48 + w];
+            total += misc[40 + w] + take;
+            eb += misc[56 + w];
         }
-        int run_eq = eq_base, run_out = out_base;
-        for (int base = lo; base < hi; base += 128) {
-            const int i0 = base + lane * 4;
-            bool gt[4], eq[4];
-            classify(i0, gt, eq);
-            const int neq = eq[0] + eq[1] + eq[2] + eq[3];
-            const int eq_pre = warp_exclusive_scan(neq, lane);
-            int er = run_eq + eq_pre;
-            bool take[4];
-            int nsel = 0;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                take[j] = gt[j] || (eq[j] && er < quota);
-                er += eq[j];
-                nsel += take[j];
-            }
-            const int sel_pre = warp_exclusive_scan(nsel, lane);
-            int pos = run_out + sel_pre;
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (take[j]) list[pos++] = (uint16_t)(i0 + j);
-            run_eq += __shfl_sync(kFull, eq_pre + neq, 31);
-            run_out += __shfl_sync(kFull, sel_pre + nsel, 31);
+        uint32_t rowtake = rowgt;
+        {
+            int r = eq_base + warp_exclusive_scan(__popc(roweq), lane);
+            for (uint32_t e = roweq; e; e &= e - 1u, ++r)
+                if (r < quota) rowtake |= e & (0u - e);
         }
+        int pos = out_base + warp_exclusive_scan(__popc(rowtake), lane);
+        for (uint32_t t = rowtake; t; t &= t - 1u) list[pos++] = (uint16_t)(wbase + 32 * lane + (__ffs(t) - 1));
         for (int i = tid; i < n_loc - n_cand_loc; i += kThreads) list[total + i] = (uint16_t)(n_cand_loc + i);
-        if (tid == 0) misc[64] = total + (n_loc - n_cand_loc);
+        if (tid == 0) misc[72] = total + (n_loc - n_cand_loc);
         __syncthreads();
     }
-    const int n_list = misc[64];
+    const int n_list = misc[72];
 
     // ---- optional export of the kept set ----
     if (p.sel) {
         cluster.sync();
         int before = 0, all = 0;
         for (int c = 0; c < p.C; ++c) {
-            const int nc = cluster.map_shared_rank(misc, c)[64];
+            const int nc = cluster.map_shared_rank(misc, c)[72];
             if (c < crank) before += nc;
             all += nc;
         }
