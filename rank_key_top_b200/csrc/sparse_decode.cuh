@@ -148,6 +148,41 @@ __device__ __forceinline__ uint32_t block_suffix_exclusive(uint32_t v, uint32_t*
     return x - v + wsum[kWarps + warp];
 }
 
+// One digit of the cluster-wide radix select. Sums the cluster's histograms
+// hcur[0 .. nbins) (nbins <= 4 * kThreads, a multiple of 4) through distributed
+// shared memory and finds the digit where the count of keys from the top
+// reaches krem. Returns (digit, count above it) in every thread. Called by all
+// threads of every CTA of the cluster; not inlined, so the three digits share
+// one copy of the code.
+__device__ __noinline__ int2 radix_boundary(const uint32_t* hcur, int nbins, int krem, int32_t* misc, int C) {
+    cg::cluster_group cluster = cg::this_cluster();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __syncthreads();
+    cluster.sync();
+    uint32_t hv[4] = {0u, 0u, 0u, 0u};  // bins 4 tid .. 4 tid + 3
+    if (4 * tid < nbins) {
+        for (int c = 0; c < C; ++c) {
+            const uint4 v = reinterpret_cast<const uint4*>(cluster.map_shared_rank(hcur, c))[tid];
+            hv[0] += v.x;
+            hv[1] += v.y;
+            hv[2] += v.z;
+            hv[3] += v.w;
+        }
+    }
+    const uint32_t tsum = hv[0] + hv[1] + hv[2] + hv[3];
+    uint32_t run = block_suffix_exclusive(tsum, reinterpret_cast<uint32_t*>(misc + 8), lane, warp);
+#pragma unroll
+    for (int j = 3; j >= 0; --j) {
+        if (run < (uint32_t)krem && run + hv[j] >= (uint32_t)krem) {
+            misc[0] = 4 * tid + j;
+            misc[1] = (int)run;
+        }
+        run += hv[j];
+    }
+    __syncthreads();
+    return make_int2(misc[0], misc[1]);
+}
+
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const SparseParams p) {
     using Geom = SparseGeom<T, D, G>;
@@ -520,76 +555,37 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
 
     // ---- 3. top-k over the cluster ----
     // mode 0: keep every candidate, 1: keep none, 2: threshold tau / quota.
-    // From here on lane l of warp w holds the keys w*32*KPL + 32 m + l (m < KPL)
-    // in registers, KPL = ceil(cta_tokens / threads) <= 32: every pass below
-    // reads registers, and the kept list comes out in index order.
+    // Phases 3 and 5 run once per launch, so their instructions are fetched
+    // cold every time: they are written as rolled loops over the keys in
+    // shared memory, and the boundary search exists once (radix_boundary).
     const int mode = keff >= ncand ? 0 : (keff == 0 ? 1 : 2);
-    const int KPL = (p.cta_tokens + kThreads - 1) / kThreads;
-    const int wbase = warp * 32 * KPL;
-    uint32_t kr[32];
-#pragma unroll
-    for (int m = 0; m < 32; ++m) {
-        const int i = wbase + 32 * m + lane;
-        kr[m] = (m < KPL && i < n_cand_loc) ? keys[i] : 0u;
-    }
-    auto valid_at = [&](int m) { return m < KPL && wbase + 32 * m + lane < n_cand_loc; };
     uint32_t tau = 0;
     int quota = 0;
     if (mode == 2) {
-        // Sum the cluster's histograms (buffer hcur) and find the digit where
-        // the count from the top reaches krem; returns (digit, count above it).
-        auto boundary = [&](const uint32_t* hcur, int nbins, int krem) {
-            __syncthreads();
-            cluster.sync();
-            const int bpt = nbins / kThreads;  // 4 or 2 bins per thread
-            uint32_t hv[4] = {0u, 0u, 0u, 0u};
-            if (bpt == 4) {
-                for (int c = 0; c < p.C; ++c) {
-                    const uint4 v = reinterpret_cast<const uint4*>(cluster.map_shared_rank(hcur, c))[tid];
-                    hv[0] += v.x;
-                    hv[1] += v.y;
-                    hv[2] += v.z;
-                    hv[3] += v.w;
-                }
-            } else {
-                for (int c = 0; c < p.C; ++c) {
-                    const uint2 v = reinterpret_cast<const uint2*>(cluster.map_shared_rank(hcur, c))[tid];
-                    hv[0] += v.x;
-                    hv[1] += v.y;
-                }
-            }
-            const uint32_t tsum = hv[0] + hv[1] + hv[2] + hv[3];
-            uint32_t run = block_suffix_exclusive(tsum, reinterpret_cast<uint32_t*>(misc + 8), lane, warp);
-            for (int j = bpt - 1; j >= 0; --j) {
-                if (run < (uint32_t)krem && run + hv[j] >= (uint32_t)krem) {
-                    misc[0] = tid * bpt + j;
-                    misc[1] = (int)run;
-                }
-                run += hv[j];
-            }
-            __syncthreads();
-            return make_int2(misc[0], misc[1]);
-        };
         // digit 0 (top 11 bits): its histogram was built while scoring
-        const int2 d0 = boundary(hist, 2048, keff);
+        const int2 d0 = radix_boundary(hist, 2048, keff, misc, p.C);
         const uint32_t beta0 = (uint32_t)d0.x;
         int krem = keff - d0.y;
         // digit 1 (next 11 bits) over the keys in the boundary bin
         uint32_t* h1 = hist + kHistBins;
-#pragma unroll
-        for (int m = 0; m < 32; ++m)
-            if (valid_at(m) && (kr[m] >> 21) == beta0) atomicAdd(&h1[(kr[m] >> 10) & 2047u], 1u);
-        const int2 d1 = boundary(h1, 2048, krem);
-        const uint32_t beta1 = (uint32_t)d1.x;
+#pragma unroll 4
+        for (int i = tid; i < n_cand_loc; i += kThreads) {
+            const uint32_t x = keys[i];
+            if ((x >> 21) == beta0) atomicAdd(&h1[(x >> 10) & 2047u], 1u);
+        }
+        const int2 d1 = radix_boundary(h1, 2048, krem, misc, p.C);
         krem -= d1.y;
-        // digit 2 (last 10 bits) into buffer 0, whose readers are all done
+        // digit 2 (last 10 bits) into buffer 0: every CTA of the cluster has
+        // read it, the cluster barrier of the previous search orders that
         for (int i = tid; i < kHistBins; i += kThreads) hist[i] = 0;
         __syncthreads();
-        const uint32_t pre22 = (beta0 << 21) | (beta1 << 10);
-#pragma unroll
-        for (int m = 0; m < 32; ++m)
-            if (valid_at(m) && (kr[m] & 0xFFFFFC00u) == pre22) atomicAdd(&hist[kr[m] & 1023u], 1u);
-        const int2 d2 = boundary(hist, 1024, krem);
+        const uint32_t pre22 = (beta0 << 21) | ((uint32_t)d1.x << 10);
+#pragma unroll 4
+        for (int i = tid; i < n_cand_loc; i += kThreads) {
+            const uint32_t x = keys[i];
+            if ((x & 0xFFFFFC00u) == pre22) atomicAdd(&hist[x & 1023u], 1u);
+        }
+        const int2 d2 = radix_boundary(hist, 1024, krem, misc, p.C);
         tau = pre22 | (uint32_t)d2.x;
         krem -= d2.y;
         // keys equal to tau: the last histogram counted them per CTA in bin (tau & 1023)
@@ -600,32 +596,35 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     }
 
     // ---- compaction of the kept local tokens into `list`, ascending ----
-    // Bit m of a lane's masks marks its key m (index wbase + 32 m + lane). 32
-    // ballots transpose the masks, so that lane r holds row r (keys wbase +
-    // 32 r + b, b = 0..31); rows in lane order, bits in order, are index order.
+    // Thread (warp w, lane l) owns row 32 w + l: keys 32 (32 w + l) .. + 31,
+    // read as 8 vectors in a lane-rotated order (conflict-free). Rows in lane
+    // order, bits in order, are index order. The keys region is a multiple of
+    // 32 keys, so a row that starts below n_cand_loc is inside it.
     {
-        uint32_t gtm = 0u, eqm = 0u;
+        const int row0 = 32 * (32 * warp + lane);
+        uint32_t rowgt = 0u, roweq = 0u;
+        if (mode != 1 && row0 < n_cand_loc) {
+            const uint4* kv = reinterpret_cast<const uint4*>(keys + row0);
+            const int nv = n_cand_loc - row0;  // valid keys in this row (may exceed 32)
+#pragma unroll 1
+            for (int j = 0; j < 8; ++j) {
+                const int c = (j + lane) & 7;
+                const uint4 v = kv[c];
+                const uint32_t x[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int m = 0; m < 32; ++m) {
-            const bool v = valid_at(m);
-            gtm |= (uint32_t)(v && (mode == 0 || (mode == 2 && kr[m] > tau))) << m;
-            eqm |= (uint32_t)(v && mode == 2 && kr[m] == tau) << m;
+                for (int e = 0; e < 4; ++e) {
+                    const int bit = 4 * c + e;
+                    const bool ok = bit < nv;
+                    rowgt |= (uint32_t)(ok && (mode == 0 || x[e] > tau)) << bit;
+                    roweq |= (uint32_t)(ok && mode == 2 && x[e] == tau) << bit;
+                }
+            }
         }
-        const int ngt = __reduce_add_sync(kFull, __popc(gtm));
-        const int neq = __reduce_add_sync(kFull, __popc(eqm));
+        const int ngt = __reduce_add_sync(kFull, __popc(rowgt));
+        const int neq = __reduce_add_sync(kFull, __popc(roweq));
         if (lane == 0) {
             misc[40 + warp] = ngt;
             misc[56 + warp] = neq;
-        }
-        uint32_t rowgt = 0u, roweq = 0u;
-#pragma unroll
-        for (int m = 0; m < 32; ++m) {
-            const uint32_t bg = __ballot_sync(kFull, (gtm >> m) & 1u);
-            const uint32_t be = __ballot_sync(kFull, (eqm >> m) & 1u);
-            if (lane == m) {
-                rowgt = bg;
-                roweq = be;
-            }
         }
         __syncthreads();
         // warp w keeps all its keys above tau and the equal ones whose rank
@@ -647,7 +646,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
                 if (r < quota) rowtake |= e & (0u - e);
         }
         int pos = out_base + warp_exclusive_scan(__popc(rowtake), lane);
-        for (uint32_t t = rowtake; t; t &= t - 1u) list[pos++] = (uint16_t)(wbase + 32 * lane + (__ffs(t) - 1));
+        for (uint32_t t = rowtake; t; t &= t - 1u) list[pos++] = (uint16_t)(row0 + (__ffs(t) - 1));
         for (int i = tid; i < n_loc - n_cand_loc; i += kThreads) list[total + i] = (uint16_t)(n_cand_loc + i);
         if (tid == 0) misc[72] = total + (n_loc - n_cand_loc);
         __syncthreads();
