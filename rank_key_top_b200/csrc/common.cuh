@@ -1,7 +1,7 @@
 // Device-side helpers shared by the libloki kernels: cache layout, typed
-// loads, order-preserving score keys, mbarrier + bulk-copy (TMA) wrappers and
-// the device error word. Included once, by loki.cu, so that every kernel and
-// the error word live in one translation unit.
+// loads, order-preserving score keys, warp helpers and the device error
+// word. Included once, by loki.cu, so that every kernel and the error word
+// live in one translation unit.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -118,61 +118,10 @@ __device__ __forceinline__ uint32_t score_key(float s) {
 }
 
 // ---------------------------------------------------------------------------
-// mbarrier and bulk async copy (TMA engine, non-tensor form) wrappers.
+// Shared-memory addresses.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void fence_mbarrier_init() {
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
-
-// Bulk copy global -> this CTA's shared memory, completing on `bar`.
-// dst, src 16-byte aligned; bytes a multiple of 16.
-__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded wait for phase `parity` of `bar`. Gives up after kWaitLimit polls
-// (each poll may suspend the thread for a while in hardware), sets
-// LOKI_DEVERR_TIMEOUT and returns false; the caller then treats the data as
-// absent and keeps going so that every barrier of the CTA is still reached.
-constexpr uint32_t kWaitLimit = 1u << 22;
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kWaitLimit; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
-    flag_error(LOKI_DEVERR_TIMEOUT);
-    return false;
 }
 
 // ---------------------------------------------------------------------------

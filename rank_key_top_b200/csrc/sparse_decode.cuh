@@ -44,16 +44,6 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kMaxSlots = 16;
 constexpr int kHistBins = 2048;  // 11-bit digits (10 in the last pass)
 constexpr int kCtaTokenCap = 16384;
-// Scoring loop tuning: blocks per warp iteration, and whether the top-digit
-// histogram aggregates equal bins of a warp (match) or adds one by one.
-#ifndef LOKI_SCORE_BLOCKS
-#define LOKI_SCORE_BLOCKS 1
-#endif
-#ifndef LOKI_SCORE_HIST_MATCH
-#define LOKI_SCORE_HIST_MATCH 0
-#endif
-constexpr int kScoreBlocks = LOKI_SCORE_BLOCKS;
-constexpr bool kScoreHistMatch = LOKI_SCORE_HIST_MATCH != 0;
 
 struct SparseParams {
     const void* k_cache;
@@ -79,7 +69,7 @@ struct SparseParams {
     // scoring the ring region holds the candidate buffer (head) and the kept
     // list (tail), and the gather stages rows across keys + ring minus list.
     int off_keys, keys_bytes, off_ring, ring_bytes, off_list, off_qf, off_qhat, off_qs, off_tbl, off_hist,
-        off_bars, off_part, off_misc, smem_bytes;
+        off_part, off_misc, smem_bytes;
 };
 
 #ifndef LOKI_GATHER_CHUNK
@@ -110,6 +100,27 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+// cp.async.wait_group with a run-time count n in [0, 15]
+__device__ __forceinline__ void cp_async_wait_n(int n) {
+    switch (n) {
+        case 0: cp_async_wait<0>(); break;
+        case 1: cp_async_wait<1>(); break;
+        case 2: cp_async_wait<2>(); break;
+        case 3: cp_async_wait<3>(); break;
+        case 4: cp_async_wait<4>(); break;
+        case 5: cp_async_wait<5>(); break;
+        case 6: cp_async_wait<6>(); break;
+        case 7: cp_async_wait<7>(); break;
+        case 8: cp_async_wait<8>(); break;
+        case 9: cp_async_wait<9>(); break;
+        case 10: cp_async_wait<10>(); break;
+        case 11: cp_async_wait<11>(); break;
+        case 12: cp_async_wait<12>(); break;
+        case 13: cp_async_wait<13>(); break;
+        case 14: cp_async_wait<14>(); break;
+        default: cp_async_wait<15>(); break;
+    }
 }
 
 // Exclusive prefix sum over the lanes of a warp.
@@ -211,7 +222,6 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     float* qs = reinterpret_cast<float*>(smem + p.off_qs);
     int32_t* tbl = reinterpret_cast<int32_t*>(smem + p.off_tbl);
     uint32_t* hist = reinterpret_cast<uint32_t*>(smem + p.off_hist);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bars);
     float* part = reinterpret_cast<float*>(smem + p.off_part);
     int32_t* misc = reinterpret_cast<int32_t*>(smem + p.off_misc);
     // misc: [0] boundary digit, [1] count above it, [8..39] suffix-sum scratch,
@@ -269,15 +279,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
 #pragma unroll
     for (int j = 0; j < G; ++j) qraw[j] = Vec<T, RPG>::load(qg + j * D + rg * RPG);
 
-    // each warp owns its ring's barriers: it starts its key-index stream as
-    // soon as its block-table entries arrive, before any CTA-wide barrier
+    // each warp starts its key-index stream as soon as its block-table
+    // entries arrive, before any CTA-wide barrier
     unsigned char* wring = ring + warp * p.ring_bytes_per_warp;
-    uint64_t* wbar = bars + warp * kMaxSlots;
-    if (lane == 0) {
-        for (int i = 0; i < kMaxSlots; ++i) mbar_init(&wbar[i], 1);
-        fence_mbarrier_init();
-    }
-    __syncwarp();
     auto checked = [&](int pb) {
         if (pb < 0 || pb >= p.num_blocks) {
             flag_error(LOKI_DEVERR_BLOCK_ID);
@@ -289,24 +293,25 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     tb1 = checked(tb1);
     const int my_blocks = nblk_score > warp ? (nblk_score - warp + kWarps - 1) / kWarps : 0;
     const unsigned char* xbytes = reinterpret_cast<const unsigned char*>(p.k_index);
-    auto issue = [&](int it, int pb) {  // lane 0 only
-        const int slot = it % S;
-        const unsigned char* src = xbytes + page_offset(pb, h, p.Hkv, p.index_dims) * (int64_t)sizeof(T);
-        mbar_arrive_expect_tx(&wbar[slot], (uint32_t)p.slot_bytes);
-        bulk_copy_g2s(wring + slot * p.slot_bytes, src, (uint32_t)p.slot_bytes, &wbar[slot]);
-    };
     auto entry = [&](int it) {  // all lanes: block of this warp's iteration it
         const int v0 = __shfl_sync(kFull, tb0, it & 31);
         const int v1 = __shfl_sync(kFull, tb1, it & 31);
         return it < 32 ? v0 : v1;
     };
-    {
-        const int first = my_blocks < S ? my_blocks : S;
-        for (int it = 0; it < first; ++it) {
+    // Ring of S slots per warp: every lane copies 16-byte pieces of a block
+    // with cp.async (pieces lane, lane + 32, ...), one commit group per
+    // iteration (empty past the warp's last block), so that waiting for block
+    // it is cp.async.wait_group S - 1.
+    auto refill = [&](int it) {  // all lanes; slot it % S is free
+        if (it < my_blocks) {
             const int pb = entry(it);
-            if (lane == 0) issue(it, pb);
+            const unsigned char* src = xbytes + page_offset(pb, h, p.Hkv, p.index_dims) * (int64_t)sizeof(T);
+            unsigned char* dst = wring + (it % S) * p.slot_bytes;
+            for (int o = lane * 16; o < p.slot_bytes; o += 32 * 16) cp_async16(dst + o, src + o, true);
         }
-    }
+        cp_async_commit();
+    };
+    for (int it = 0; it < S; ++it) refill(it);
     for (int i = tid; i < 2 * kHistBins; i += kThreads) hist[i] = 0;
     {
         const int j0 = warp + lane * kWarps, j1 = warp + (lane + 32) * kWarps;
@@ -363,7 +368,10 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     // a second column group for heads 4..7), on warp-level MMA with fp32
     // accumulation. fp32 index: CUDA-core dot products.
     {
-        bool failed = false;
+        auto wait_slot = [&]() {  // all lanes: the oldest slot in flight has landed
+            cp_async_wait_n(S - 1);
+            __syncwarp();
+        };
         auto mma_body = [&](auto rmax_tag) {
             constexpr int RMAX = decltype(rmax_tag)::value;
             constexpr int SG = G > 4 ? 2 : 1;
@@ -395,19 +403,14 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
                 }
             const int arow = (lane & 7) + 8 * ((lane >> 3) & 1), ahalf = lane >> 4;
             for (int it = 0; it < my_blocks; ++it) {
-                const int slot = it % S;
-                const uint32_t parity = (uint32_t)(it / S) & 1u;
-                if (!failed) failed = __any_sync(kFull, !mbar_wait_bounded(&wbar[slot], parity));
-                const unsigned char* sl = wring + slot * p.slot_bytes;
+                wait_slot();
+                const unsigned char* sl = wring + (it % S) * p.slot_bytes;
                 uint32_t a[RMAX][4];
 #pragma unroll
                 for (int sb = 0; sb < RMAX; ++sb)
                     if (sb < R16) ldmatrix_x4(a[sb][0], a[sb][1], a[sb][2], a[sb][3], sl + sb * 512 + arow * 32 + ahalf * 16);
                 __syncwarp();
-                if (it + S < my_blocks) {
-                    const int pb = entry(it + S);
-                    if (lane == 0) issue(it + S, pb);
-                }
+                refill(it + S);
                 float sc0 = -INFINITY, sc1 = -INFINITY;  // tokens g and g + 8
 #pragma unroll
                 for (int ng = 0; ng < SG; ++ng) {
@@ -446,96 +449,63 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
         auto body = [&](auto rmax_tag) {
             constexpr int RMAX = decltype(rmax_tag)::value;
             const int R16 = p.r / kSlabDims;
-            constexpr int NB = kScoreBlocks;
             using V8 = Vec<T, 8>;
             const int tok = lane >> 1, half = lane & 1;
-            for (int it = 0; it < my_blocks; it += NB) {
-                typename V8::raw_t raw[NB][RMAX];
+            for (int it = 0; it < my_blocks; ++it) {
+                wait_slot();
+                const T* sl = reinterpret_cast<const T*>(wring + (it % S) * p.slot_bytes);
+                typename V8::raw_t raw[RMAX];
 #pragma unroll
-                for (int u = 0; u < NB; ++u) {
-                    if (it + u < my_blocks) {
-                        const int slot = (it + u) % S;
-                        const uint32_t parity = (uint32_t)((it + u) / S) & 1u;
-                        if (!failed) failed = __any_sync(kFull, !mbar_wait_bounded(&wbar[slot], parity));
-                        const T* sl = reinterpret_cast<const T*>(wring + slot * p.slot_bytes);
-#pragma unroll
-                        for (int sb = 0; sb < RMAX; ++sb)
-                            if (sb < R16) raw[u][sb] = V8::load(sl + sb * 256 + tok * 16 + half * 8);
-                    }
-                }
+                for (int sb = 0; sb < RMAX; ++sb)
+                    if (sb < R16) raw[sb] = V8::load(sl + sb * 256 + tok * 16 + half * 8);
                 __syncwarp();
-#pragma unroll
-                for (int u = 0; u < NB; ++u) {
-                    if (it + u + S < my_blocks) {
-                        const int pb = entry(it + u + S);
-                        if (lane == 0) issue(it + u + S, pb);
-                    }
-                }
-                float sc[NB];
+                refill(it + S);
+                float sc;
                 if (!p.group_max) {
+                    float a = 0.f;
 #pragma unroll
-                    for (int u = 0; u < NB; ++u) {
-                        float a = 0.f;
-#pragma unroll
-                        for (int sb = 0; sb < RMAX; ++sb) {
-                            if (sb >= R16) break;
-                            float kf[8];
-                            V8::to_float(raw[u][sb], kf);
-                            const float4 q0 = *reinterpret_cast<const float4*>(qs + sb * 16 + half * 8);
-                            const float4 q1 = *reinterpret_cast<const float4*>(qs + sb * 16 + half * 8 + 4);
-                            a = fmaf(q0.x, kf[0], a);
-                            a = fmaf(q0.y, kf[1], a);
-                            a = fmaf(q0.z, kf[2], a);
-                            a = fmaf(q0.w, kf[3], a);
-                            a = fmaf(q1.x, kf[4], a);
-                            a = fmaf(q1.y, kf[5], a);
-                            a = fmaf(q1.z, kf[6], a);
-                            a = fmaf(q1.w, kf[7], a);
-                        }
-                        sc[u] = a;
+                    for (int sb = 0; sb < RMAX; ++sb) {
+                        if (sb >= R16) break;
+                        float kf[8];
+                        V8::to_float(raw[sb], kf);
+                        const float4 q0 = *reinterpret_cast<const float4*>(qs + sb * 16 + half * 8);
+                        const float4 q1 = *reinterpret_cast<const float4*>(qs + sb * 16 + half * 8 + 4);
+                        a = fmaf(q0.x, kf[0], a);
+                        a = fmaf(q0.y, kf[1], a);
+                        a = fmaf(q0.z, kf[2], a);
+                        a = fmaf(q0.w, kf[3], a);
+                        a = fmaf(q1.x, kf[4], a);
+                        a = fmaf(q1.y, kf[5], a);
+                        a = fmaf(q1.z, kf[6], a);
+                        a = fmaf(q1.w, kf[7], a);
                     }
-#pragma unroll
-                    for (int u = 0; u < NB; ++u) sc[u] += __shfl_xor_sync(kFull, sc[u], 1);
+                    sc = a + __shfl_xor_sync(kFull, a, 1);
                 } else {
+                    float ag[G];
 #pragma unroll
-                    for (int u = 0; u < NB; ++u) {
-                        float ag[G];
+                    for (int j = 0; j < G; ++j) ag[j] = 0.f;
 #pragma unroll
-                        for (int j = 0; j < G; ++j) ag[j] = 0.f;
+                    for (int sb = 0; sb < RMAX; ++sb) {
+                        if (sb >= R16) break;
+                        float kf[8];
+                        V8::to_float(raw[sb], kf);
 #pragma unroll
-                        for (int sb = 0; sb < RMAX; ++sb) {
-                            if (sb >= R16) break;
-                            float kf[8];
-                            V8::to_float(raw[u][sb], kf);
+                        for (int j = 0; j < G; ++j) {
+                            const float* qq = qhat + j * D + sb * 16 + half * 8;
 #pragma unroll
-                            for (int j = 0; j < G; ++j) {
-                                const float* qq = qhat + j * D + sb * 16 + half * 8;
-#pragma unroll
-                                for (int i = 0; i < 8; ++i) ag[j] = fmaf(qq[i], kf[i], ag[j]);
-                            }
+                            for (int i = 0; i < 8; ++i) ag[j] = fmaf(qq[i], kf[i], ag[j]);
                         }
-                        float m = -INFINITY;
-#pragma unroll
-                        for (int j = 0; j < G; ++j) m = fmaxf(m, ag[j] + __shfl_xor_sync(kFull, ag[j], 1));
-                        sc[u] = m;
                     }
+                    float m = -INFINITY;
+#pragma unroll
+                    for (int j = 0; j < G; ++j) m = fmaxf(m, ag[j] + __shfl_xor_sync(kFull, ag[j], 1));
+                    sc = m;
                 }
-#pragma unroll
-                for (int u = 0; u < NB; ++u) {
-                    const int li = (warp + (it + u) * kWarps) * kBlockTokens + tok;
-                    const bool valid = half == 0 && it + u < my_blocks && li < n_cand_loc;
-                    const uint32_t key = score_key(sc[u]);
-                    if (valid) keys[li] = key;
-                    const unsigned bin = key >> 21;
-                    if constexpr (kScoreHistMatch) {
-                        const unsigned vmask = __ballot_sync(kFull, valid);
-                        if (valid) {
-                            const unsigned peers = __match_any_sync(vmask, bin);
-                            if ((peers & ((1u << lane) - 1u)) == 0) atomicAdd(&hist[bin], (unsigned)__popc(peers));
-                        }
-                    } else {
-                        if (valid) atomicAdd(&hist[bin], 1u);
-                    }
+                const int li = (warp + it * kWarps) * kBlockTokens + tok;
+                if (half == 0 && li < n_cand_loc) {
+                    const uint32_t key = score_key(sc);
+                    keys[li] = key;
+                    atomicAdd(&hist[key >> 21], 1u);
                 }
             }
         };
@@ -551,6 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
                 body(std::integral_constant<int, D / kSlabDims>{});
         }
     }
+    cp_async_wait<0>();  // the empty trailing groups
     __syncthreads();
 
     // ---- 3. top-k over the cluster ----
