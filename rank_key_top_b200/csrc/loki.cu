@@ -151,8 +151,8 @@ void sparse_layout(SparseParams& p, int max_seq_len, int ring_per_warp) {
     off = align(off + (p.cta_tokens / kBlockTokens) * 4);
     p.off_hist = off;
     off = align(off + 2 * kHistBins * 4);
-    p.off_part = off;
-    off = align(off + G * (D + 2) * 4);
+    p.off_part = off;  // one partial slot per CTA of the cluster (used in rank 0)
+    off = align(off + p.C * G * (D + 2) * 4);
     p.off_misc = off;
     off = align(off + 128 * 4);
     p.smem_bytes = off;

@@ -25,8 +25,9 @@
 //     (3)-(5)): each warp stages chunks of key rows and value rows into
 //     shared memory with cp.async (the next chunk in flight while the current
 //     one is consumed) and runs AttnCore on them.
-//  5. the warps' partials merge per CTA, then rank 0 merges the CTAs'
-//     partials through distributed shared memory and writes the output.
+//  5. the warps' partials merge per CTA into a slot of rank 0's shared
+//     memory (distributed shared memory stores); after one cluster barrier
+//     rank 0 combines the slots and writes the output.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -227,7 +228,40 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     // misc: [0] boundary digit, [1] count above it, [8..39] suffix-sum scratch,
     //       [40..55] warp kept counts, [56..71] warp equal counts, [72] list length
 
-    // ---- sequence geometry (identical in every CTA of the cluster) ----
+    // ---- sequence geometry ----
+    // CTA crank owns the fixed token range [crank * cta_tokens, + cta_tokens)
+    // of its sequence, so its block-table loads need not wait for the length;
+    // one wave of clusters runs at once, so the launch takes as long as the
+    // longest sequence whatever the split of the shorter ones.
+    const int cta_blocks = p.cta_tokens / kBlockTokens;
+    const int blk0 = crank * cta_blocks;
+    const int t0 = blk0 * kBlockTokens;
+    // block-table entries of this warp's blocks jb = warp + it * kWarps:
+    // lane l holds those of it = l and it = l + 32 (at most 64 per warp);
+    // entries past the end of the sequence are loaded but never used
+    const int32_t* trow = p.block_table + (int64_t)b * p.max_blocks + blk0;
+    int tb0 = 0, tb1 = 0;
+    const int j0 = warp + lane * kWarps, j1 = warp + (lane + 32) * kWarps;
+    {
+        const int lim = min(cta_blocks, p.max_blocks - blk0);
+        if (j0 < lim) tb0 = trow[j0];
+        if (j1 < lim) tb1 = trow[j1];
+    }
+    // the prologue's P and q loads do not depend on the length either
+    constexpr int NQ = D / 4;             // q_hat: thread (row group rg, column quad cq)
+    constexpr int NRG = kThreads / NQ;
+    constexpr int RPG = D / NRG;
+    const int cq = tid % NQ, rg = tid / NQ;
+    float4 pv[RPG];
+    {
+        const float* Ph = p.P + (int64_t)h * D * D;
+#pragma unroll
+        for (int i = 0; i < RPG; ++i) pv[i] = *reinterpret_cast<const float4*>(Ph + (rg * RPG + i) * D + 4 * cq);
+    }
+    const T* qg = reinterpret_cast<const T*>(p.q) + ((int64_t)b * Hq + h * G) * D;
+    typename Vec<T, RPG>::raw_t qraw[G];
+#pragma unroll
+    for (int j = 0; j < G; ++j) qraw[j] = Vec<T, RPG>::load(qg + j * D + rg * RPG);
     int L = p.seq_lens[b];
     if (L < 0 || L > p.max_seq_len) {
         if (tid == 0 && crank == 0) flag_error(LOKI_DEVERR_SEQ_LEN);
@@ -244,40 +278,13 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
         }
     }
     const int keff = kb < ncand ? kb : ncand;
-    const int nblk = (L + kBlockTokens - 1) / kBlockTokens;
-    const int bpc = (nblk + p.C - 1) / p.C;
-    const int blk0 = crank * bpc;
-    const int t0 = blk0 * kBlockTokens;
-    const int n_loc = max(0, min(L - t0, bpc * kBlockTokens));
+    const int n_loc = max(0, min(L - t0, p.cta_tokens));
     const int nblk_loc = (n_loc + kBlockTokens - 1) / kBlockTokens;
     const int n_cand_loc = max(0, min(ncand - t0, n_loc));
     const int nblk_score = (n_cand_loc + kBlockTokens - 1) / kBlockTokens;
 
     // ---- 1. prologue: every global load is issued before the first barrier ----
     const int S = p.slots;
-    // block-table entries of this warp's blocks jb = warp + it * kWarps:
-    // lane l holds those of it = l and it = l + 32 (at most 64 per warp)
-    const int32_t* trow = p.block_table + (int64_t)b * p.max_blocks + blk0;
-    int tb0 = 0, tb1 = 0;
-    {
-        const int j0 = warp + lane * kWarps, j1 = warp + (lane + 32) * kWarps;
-        if (j0 < nblk_loc) tb0 = trow[j0];
-        if (j1 < nblk_loc) tb1 = trow[j1];
-    }
-    constexpr int NQ = D / 4;             // q_hat: thread (row group rg, column quad cq)
-    constexpr int NRG = kThreads / NQ;
-    constexpr int RPG = D / NRG;
-    const int cq = tid % NQ, rg = tid / NQ;
-    float4 pv[RPG];
-    {
-        const float* Ph = p.P + (int64_t)h * D * D;
-#pragma unroll
-        for (int i = 0; i < RPG; ++i) pv[i] = *reinterpret_cast<const float4*>(Ph + (rg * RPG + i) * D + 4 * cq);
-    }
-    const T* qg = reinterpret_cast<const T*>(p.q) + ((int64_t)b * Hq + h * G) * D;
-    typename Vec<T, RPG>::raw_t qraw[G];
-#pragma unroll
-    for (int j = 0; j < G; ++j) qraw[j] = Vec<T, RPG>::load(qg + j * D + rg * RPG);
 
     // each warp starts its key-index stream as soon as its block-table
     // entries arrive, before any CTA-wide barrier
@@ -289,8 +296,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
         }
         return pb;
     };
-    tb0 = checked(tb0);
-    tb1 = checked(tb1);
+    tb0 = j0 < nblk_loc ? checked(tb0) : 0;
+    tb1 = j1 < nblk_loc ? checked(tb1) : 0;
     const int my_blocks = nblk_score > warp ? (nblk_score - warp + kWarps - 1) / kWarps : 0;
     const unsigned char* xbytes = reinterpret_cast<const unsigned char*>(p.k_index);
     auto entry = [&](int it) {  // all lanes: block of this warp's iteration it
@@ -313,11 +320,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     };
     for (int it = 0; it < S; ++it) refill(it);
     for (int i = tid; i < 2 * kHistBins; i += kThreads) hist[i] = 0;
-    {
-        const int j0 = warp + lane * kWarps, j1 = warp + (lane + 32) * kWarps;
-        if (j0 < nblk_loc) tbl[j0] = tb0;
-        if (j1 < nblk_loc) tbl[j1] = tb1;
-    }
+    if (j0 < nblk_loc) tbl[j0] = tb0;
+    if (j1 < nblk_loc) tbl[j1] = tb1;
     __syncthreads();
 
     {   // q_hat = q P[h]: each thread sums its RPG rows for its 4 columns
@@ -714,29 +718,34 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     }
     __syncthreads();
 
-    // ---- 5. merge: warps -> CTA partial -> cluster rank 0 -> out ----
+    // ---- 5. merge: warps -> CTA partial in rank 0's shared memory -> out ----
+    // Every CTA writes its partial (per head: G x D numerators, running max,
+    // denominator) into slot crank of rank 0's `part`; one cluster barrier
+    // publishes them, and rank 0 combines the slots and writes the output.
+    // No CTA reads another's shared memory after that barrier, so the others
+    // may exit at once.
     {
-        if (tid < G) {
-            const int j = tid;
-            float M = -INFINITY;
-            for (int w = 0; w < kWarps; ++w) M = fmaxf(M, wpart[w * G * (D + 2) + j * (D + 2) + D]);
-            float lsum = 0.f;
-            for (int w = 0; w < kWarps; ++w) {
-                const float mw = wpart[w * G * (D + 2) + j * (D + 2) + D];
-                const float wt = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
-                wts[j * kWarps + w] = wt;
-                lsum = fmaf(wt, wpart[w * G * (D + 2) + j * (D + 2) + D + 1], lsum);
+        float* dst = cluster.map_shared_rank(part, 0) + crank * G * (D + 2);
+        if (warp < G) {  // warp j: head j's max and denominator over the CTA's warps
+            const int j = warp;
+            const float* wp = wpart + lane * G * (D + 2) + j * (D + 2);
+            const float mw = lane < kWarps ? wp[D] : -INFINITY;
+            const float M = warp_max_xor(mw, 0, 5);
+            const float wt = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+            const float l = warp_sum_xor(lane < kWarps ? wt * wp[D + 1] : 0.f, 0, 5);
+            if (lane < kWarps) wts[j * kWarps + lane] = wt;
+            if (lane == 0) {
+                dst[j * (D + 2) + D] = M;
+                dst[j * (D + 2) + D + 1] = l;
             }
-            part[j * (D + 2) + D] = M;
-            part[j * (D + 2) + D + 1] = lsum;
         }
         __syncthreads();
         for (int o = tid; o < G * D; o += kThreads) {
             const int j = o / D, c = o - j * D;
             float a = 0.f;
-#pragma unroll
+#pragma unroll 4
             for (int w = 0; w < kWarps; ++w) a = fmaf(wts[j * kWarps + w], wpart[w * G * (D + 2) + j * (D + 2) + c], a);
-            part[j * (D + 2) + c] = a;
+            dst[j * (D + 2) + c] = a;
         }
     }
     cluster.sync();
@@ -744,11 +753,11 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
         for (int o = tid; o < G * D; o += kThreads) {
             const int j = o / D, c = o - j * D;
             float M = -INFINITY;
-            for (int r = 0; r < p.C; ++r) M = fmaxf(M, cluster.map_shared_rank(part, r)[j * (D + 2) + D]);
+            for (int r = 0; r < p.C; ++r) M = fmaxf(M, part[(r * G + j) * (D + 2) + D]);
             float num = 0.f, den = 0.f;
             if (M != -INFINITY) {
                 for (int r = 0; r < p.C; ++r) {
-                    const float* pr = cluster.map_shared_rank(part, r) + j * (D + 2);
+                    const float* pr = part + (r * G + j) * (D + 2);
                     const float mr = pr[D];
                     if (mr == -INFINITY) continue;
                     const float w = exp2f(mr - M);
@@ -759,7 +768,6 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
             p.out[((int64_t)b * Hq + h * G + j) * D + c] = den > 0.f ? num / den : 0.f;
         }
     }
-    cluster.sync();
 }
 
 }  // namespace loki
