@@ -126,8 +126,10 @@ void sparse_layout(SparseParams& p, int max_seq_len, int ring_per_warp) {
     p.ring_bytes_per_warp = p.slots * p.slot_bytes;
     const int list_bytes = align(p.cta_tokens * 2);
     int ring_bytes = align(kWarps * p.ring_bytes_per_warp);
-    if (ring_bytes < list_bytes + 8 * 1024) ring_bytes = list_bytes + 8 * 1024;
-    p.cand_cap = (ring_bytes - list_bytes) / 8;
+    // after the scoring the ring region holds the select's candidate
+    // segments (head, up to one key per token) and the kept list (tail)
+    const int cand_bytes = align(p.cta_tokens * 4);
+    if (ring_bytes < list_bytes + cand_bytes) ring_bytes = list_bytes + cand_bytes;
     int keys_bytes = align(std::max(p.cta_tokens * 4, Geom::QSCRATCH_BYTES));
     // the gather stages rows in keys + ring minus the list; the warp partials
     // of the merge go to keys + ring

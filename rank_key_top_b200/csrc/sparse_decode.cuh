@@ -65,7 +65,6 @@ struct SparseParams {
     int slots;       // ring slots per warp
     int slot_bytes;  // bytes of one block's leading r index dims
     int ring_bytes_per_warp;
-    int cand_cap;    // entries of the boundary-candidate buffer (head of the ring region)
     // shared-memory layout, byte offsets. keys and ring are adjacent: after the
     // scoring the ring region holds the candidate buffer (head) and the kept
     // list (tail), and the gather stages rows across keys + ring minus list.
@@ -218,6 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     float* wpart = reinterpret_cast<float*>(smem + p.off_keys);     // after the gather
     unsigned char* ring = smem + p.off_ring;
     uint16_t* list = reinterpret_cast<uint16_t*>(smem + p.off_list);
+    uint32_t* cand = reinterpret_cast<uint32_t*>(ring);             // select only (ring head)
     float* wts = reinterpret_cast<float*>(smem + p.off_qf);         // merge weights [G][kWarps]
     float* qhat = reinterpret_cast<float*>(smem + p.off_qhat);
     float* qs = reinterpret_cast<float*>(smem + p.off_qs);
@@ -530,24 +530,63 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
 
     // ---- 3. top-k over the cluster ----
     // mode 0: keep every candidate, 1: keep none, 2: threshold tau / quota.
-    // Phases 3 and 5 run once per launch, so their instructions are fetched
-    // cold every time: they are written as rolled loops over the keys in
-    // shared memory, and the boundary search exists once (radix_boundary).
+    // Thread t owns row t of the keys (keys 32 t .. 32 t + 31, bit b of its
+    // masks = key 32 t + b); rows in thread order, bits in order, are token
+    // order. A full pass over the keys costs about a microsecond, so there is
+    // one: after digit 0 it marks the keys above the
+    // boundary bin (kept whatever tau is) and the keys inside it (the
+    // candidates, a few percent); digits 1 and 2 and the final comparison with
+    // tau look at the candidates only. The three digits share one copy of the
+    // boundary search (radix_boundary).
     const int mode = keff >= ncand ? 0 : (keff == 0 ? 1 : 2);
-    uint32_t tau = 0;
+    const int row0 = 32 * tid;
+    const int nv = n_cand_loc - row0;  // valid keys in this row (may exceed 32)
+    const uint32_t vmask = nv >= 32 ? kFull : (nv > 0 ? (1u << nv) - 1u : 0u);
+    uint32_t rowgt = mode == 0 ? vmask : 0u, roweq = 0u;
     int quota = 0;
     if (mode == 2) {
         // digit 0 (top 11 bits): its histogram was built while scoring
         const int2 d0 = radix_boundary(hist, 2048, keff, misc, p.C);
         const uint32_t beta0 = (uint32_t)d0.x;
         int krem = keff - d0.y;
-        // digit 1 (next 11 bits) over the keys in the boundary bin
-        uint32_t* h1 = hist + kHistBins;
-#pragma unroll 4
-        for (int i = tid; i < n_cand_loc; i += kThreads) {
-            const uint32_t x = keys[i];
-            if ((x >> 21) == beta0) atomicAdd(&h1[(x >> 10) & 2047u], 1u);
+        uint32_t rowcand = 0u;
+        if (nv > 0) {  // the keys region is a multiple of 32 keys
+            const uint4* kv = reinterpret_cast<const uint4*>(keys + row0);
+            uint4 v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = kv[j ^ (lane & 7)];  // XOR-rotated: conflict-free
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int c = j ^ (lane & 7);
+                const uint32_t x[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+                uint32_t g = 0u, e = 0u;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    g |= (uint32_t)((x[u] >> 21) > beta0) << u;
+                    e |= (uint32_t)((x[u] >> 21) == beta0) << u;
+                }
+                rowgt |= g << (4 * c);
+                rowcand |= e << (4 * c);
+            }
+            rowgt &= vmask;
+            rowcand &= vmask;
         }
+        // Each warp copies its candidates into its own segment of `cand` (lane
+        // offsets from a warp scan) and histograms that dense list: predicated
+        // shared atomics over all keys would be slow, since almost every
+        // warp-wide atomic would have a lane or two active.
+        uint32_t* wcand = cand + 1024 * warp;  // warp w's rows: keys [1024 w, 1024 w + 1024)
+        int nw;                                 // entries in wcand
+        {
+            const int cnt = __popc(rowcand);
+            int off = warp_exclusive_scan(cnt, lane);
+            nw = __shfl_sync(kFull, off + cnt, 31);
+            for (uint32_t t = rowcand; t; t &= t - 1u) wcand[off++] = keys[row0 + __ffs(t) - 1];
+            __syncwarp();
+        }
+        // digit 1 (next 11 bits)
+        uint32_t* h1 = hist + kHistBins;
+        for (int i = lane; i < nw; i += 32) atomicAdd(&h1[(wcand[i] >> 10) & 2047u], 1u);
         const int2 d1 = radix_boundary(h1, 2048, krem, misc, p.C);
         krem -= d1.y;
         // digit 2 (last 10 bits) into buffer 0: every CTA of the cluster has
@@ -555,46 +594,29 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
         for (int i = tid; i < kHistBins; i += kThreads) hist[i] = 0;
         __syncthreads();
         const uint32_t pre22 = (beta0 << 21) | ((uint32_t)d1.x << 10);
-#pragma unroll 4
-        for (int i = tid; i < n_cand_loc; i += kThreads) {
-            const uint32_t x = keys[i];
+        for (int i = lane; i < nw; i += 32) {
+            const uint32_t x = wcand[i];
             if ((x & 0xFFFFFC00u) == pre22) atomicAdd(&hist[x & 1023u], 1u);
         }
         const int2 d2 = radix_boundary(hist, 1024, krem, misc, p.C);
-        tau = pre22 | (uint32_t)d2.x;
+        const uint32_t tau = pre22 | (uint32_t)d2.x;
         krem -= d2.y;
         // keys equal to tau: the last histogram counted them per CTA in bin (tau & 1023)
         int eq_before = 0;
         for (int c = 0; c < crank; ++c) eq_before += (int)cluster.map_shared_rank(hist, c)[tau & 1023u];
         const int eq_mine = (int)hist[tau & 1023u];
         quota = min(max(krem - eq_before, 0), eq_mine);
+        // the candidates against tau
+        for (uint32_t t = rowcand; t; t &= t - 1u) {
+            const int bit = __ffs(t) - 1;
+            const uint32_t x = keys[row0 + bit];
+            rowgt |= (uint32_t)(x > tau) << bit;
+            roweq |= (uint32_t)(x == tau) << bit;
+        }
     }
 
     // ---- compaction of the kept local tokens into `list`, ascending ----
-    // Thread (warp w, lane l) owns row 32 w + l: keys 32 (32 w + l) .. + 31,
-    // read as 8 vectors in a lane-rotated order (conflict-free). Rows in lane
-    // order, bits in order, are index order. The keys region is a multiple of
-    // 32 keys, so a row that starts below n_cand_loc is inside it.
     {
-        const int row0 = 32 * (32 * warp + lane);
-        uint32_t rowgt = 0u, roweq = 0u;
-        if (mode != 1 && row0 < n_cand_loc) {
-            const uint4* kv = reinterpret_cast<const uint4*>(keys + row0);
-            const int nv = n_cand_loc - row0;  // valid keys in this row (may exceed 32)
-#pragma unroll 1
-            for (int j = 0; j < 8; ++j) {
-                const int c = (j + lane) & 7;
-                const uint4 v = kv[c];
-                const uint32_t x[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int bit = 4 * c + e;
-                    const bool ok = bit < nv;
-                    rowgt |= (uint32_t)(ok && (mode == 0 || x[e] > tau)) << bit;
-                    roweq |= (uint32_t)(ok && mode == 2 && x[e] == tau) << bit;
-                }
-            }
-        }
         const int ngt = __reduce_add_sync(kFull, __popc(rowgt));
         const int neq = __reduce_add_sync(kFull, __popc(roweq));
         if (lane == 0) {
