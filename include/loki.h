@@ -195,6 +195,25 @@ LOKI_API loki_status loki_decode_attention(const loki_cache* cache, const loki_b
                                   void* workspace, size_t workspace_bytes,
                                   loki_stream_t stream);
 
+/* One whole decode step: loki_append_keys(k_new, v_new, P) followed by
+ * loki_decode_attention(...) on the same stream, with the same arguments and
+ * the same results as those two calls (seq_lens already counts the new
+ * token). The attention kernel is launched as a programmatic dependent of the
+ * append kernel: it starts while the append runs and waits for it only
+ * before it first reads the appended token (before the exact attention when
+ * recent_window >= 1, before the scoring otherwise). Every argument is checked
+ * before anything is launched; an error launches nothing. This entry point has
+ * no counterpart in the pages: it packages their per-step cache update and
+ * attention as one call. */
+LOKI_API loki_status loki_decode_step(const loki_cache* cache, const loki_batch* batch,
+                             const void* k_new, const void* v_new,
+                             const void* q, int32_t num_q_heads, const float* P,
+                             int32_t r, int32_t k, const int32_t* k_per_seq,
+                             int32_t recent_window, loki_group_reduce group_reduce,
+                             float scale, float* out, int32_t* selected_idx,
+                             void* workspace, size_t workspace_bytes,
+                             loki_stream_t stream);
+
 /* Largest max_seq_len loki_decode_attention accepts for this cache shape. */
 LOKI_API int32_t loki_decode_max_seq_len(int32_t head_dim, loki_dtype dtype);
 

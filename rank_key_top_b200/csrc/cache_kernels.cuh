@@ -87,6 +87,9 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
     const int pair = blockIdx.x;
     const int b = pair / p.Hkv, h = pair - b * p.Hkv;
     const int tid = threadIdx.x;
+    // a decode launched as this kernel's programmatic dependent may start now:
+    // it waits for this grid before it reads the token written here
+    griddep_launch_dependents();
     int L = p.seq_lens[b];
     if (L < 0 || L > p.max_seq_len) {
         if (tid == 0) flag_error(LOKI_DEVERR_SEQ_LEN);

@@ -125,6 +125,18 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch. A kernel launched as a programmatic
+// dependent may start while the kernel before it in the stream still runs;
+// griddep_wait() returns once that kernel has completed and its writes are
+// visible (at once when there is no such dependency). griddep_launch_dependents()
+// lets the dependent of this kernel start launching.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // Warp helpers.
 // ---------------------------------------------------------------------------
 constexpr unsigned kFull = 0xffffffffu;

@@ -196,7 +196,7 @@ int choose_cluster(SparseParams& p, int max_seq_len, int pairs, int sms, int sme
 template <typename T, int D, int G>
 struct SparseLaunch {
     static loki_status run(SparseParams p, int pairs, int max_seq_len, const DeviceInfo& di,
-                           cudaStream_t stream) {
+                           cudaStream_t stream, bool programmatic) {
         if (choose_cluster<T, D, G>(p, max_seq_len, pairs, di.sms, di.max_smem_optin) < 1)
             return LOKI_ERR_UNSUPPORTED;
         auto kern = sparse_decode_kernel<T, D, G>;
@@ -213,13 +213,18 @@ struct SparseLaunch {
         cfg.blockDim = dim3(kThreads, 1, 1);
         cfg.dynamicSmemBytes = p.smem_bytes;
         cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = p.C;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
+        // programmatic dependent of the previous kernel in the stream (the
+        // step's append): the kernel calls griddep_wait() before it reads
+        // anything that kernel writes
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = programmatic ? 2 : 1;
         // a cluster that can never be resident is reported, not launched
         static std::map<std::pair<int, int>, bool> known;
         static std::mutex known_mu;
@@ -228,6 +233,106 @@ struct SparseLaunch {
         return launch_status();
     }
 };
+
+// Argument checks and launches shared by the entry points (the checks run on
+// the host before anything is launched).
+loki_status check_append(const loki_cache* cache, const loki_batch* batch, const void* k_new, const void* v_new,
+                         const float* P) {
+    loki_status st = check_cache(cache);
+    if (st != LOKI_OK) return st;
+    if ((st = check_batch(batch)) != LOKI_OK) return st;
+    if (batch->batch == 0) return LOKI_OK;
+    if (!k_new || !v_new) return LOKI_ERR_INVALID_ARG;
+    if (P && !aligned16(P)) return LOKI_ERR_INVALID_ARG;
+    if ((int64_t)batch->batch * cache->num_kv_heads > INT32_MAX / 2) return LOKI_ERR_UNSUPPORTED;
+    return LOKI_OK;
+}
+
+loki_status launch_append(const loki_cache* cache, const loki_batch* batch, const void* k_new, const void* v_new,
+                          const float* P, cudaStream_t s) {
+    AppendParams p;
+    p.k_cache = cache->k_cache;
+    p.v_cache = cache->v_cache;
+    p.k_index = cache->k_index;
+    p.index_dims = cache->index_dims;
+    p.block_table = batch->block_table;
+    p.seq_lens = batch->seq_lens;
+    p.k_new = k_new;
+    p.v_new = v_new;
+    p.P = P;
+    p.num_blocks = cache->num_blocks;
+    p.Hkv = cache->num_kv_heads;
+    p.max_blocks = batch->max_blocks_per_seq;
+    p.max_seq_len = batch->max_seq_len;
+    const int grid = batch->batch * cache->num_kv_heads;
+    const int D = cache->head_dim;
+    if (cache->dtype == LOKI_BF16) {
+        if (D == 64) append_kernel<__nv_bfloat16, 64><<<grid, 256, 0, s>>>(p);
+        else append_kernel<__nv_bfloat16, 128><<<grid, 256, 0, s>>>(p);
+    } else {
+        if (D == 64) append_kernel<float, 64><<<grid, 256, 0, s>>>(p);
+        else append_kernel<float, 128><<<grid, 256, 0, s>>>(p);
+    }
+    return launch_status();
+}
+
+loki_status check_decode(const loki_cache* cache, const loki_batch* batch, const void* q, int32_t num_q_heads,
+                         const float* P, int32_t r, int32_t k, int32_t recent_window,
+                         loki_group_reduce group_reduce, float scale, const float* out) {
+    loki_status st = check_cache(cache);
+    if (st != LOKI_OK) return st;
+    if ((st = check_batch(batch)) != LOKI_OK) return st;
+    const int Hkv = cache->num_kv_heads, D = cache->head_dim;
+    if (num_q_heads < 1 || num_q_heads % Hkv != 0) return LOKI_ERR_INVALID_ARG;
+    if (k < 0 || recent_window < 0 || (k == 0 && recent_window == 0)) return LOKI_ERR_INVALID_ARG;
+    if (r < 1 || r > D) return LOKI_ERR_INVALID_ARG;
+    if (group_reduce != LOKI_GROUP_SUM && group_reduce != LOKI_GROUP_MAX) return LOKI_ERR_INVALID_ARG;
+    if (!(scale >= 0.f) || std::isinf(scale)) return LOKI_ERR_INVALID_ARG;
+    if ((int64_t)k + recent_window > INT32_MAX / 2) return LOKI_ERR_INVALID_ARG;
+    if (batch->batch == 0) return LOKI_OK;
+    if (!q || !P || !out) return LOKI_ERR_INVALID_ARG;
+    if (!aligned16(P) || !aligned16(q)) return LOKI_ERR_INVALID_ARG;
+    const int G = num_q_heads / Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return LOKI_ERR_UNSUPPORTED;
+    if (r % kSlabDims != 0) return LOKI_ERR_UNSUPPORTED;
+    if (r > cache->index_dims) return LOKI_ERR_INVALID_ARG;
+    if ((int64_t)batch->batch * Hkv > 65535) return LOKI_ERR_UNSUPPORTED;
+    if (batch->max_seq_len > loki_decode_max_seq_len(D, cache->dtype)) return LOKI_ERR_UNSUPPORTED;
+    return LOKI_OK;
+}
+
+loki_status launch_decode(const loki_cache* cache, const loki_batch* batch, const void* q, int32_t num_q_heads,
+                          const float* P, int32_t r, int32_t k, const int32_t* k_per_seq, int32_t recent_window,
+                          loki_group_reduce group_reduce, float scale, float* out, int32_t* selected_idx,
+                          cudaStream_t s, bool programmatic) {
+    const int Hkv = cache->num_kv_heads, D = cache->head_dim;
+    const int G = num_q_heads / Hkv;
+    const int pairs = batch->batch * Hkv;
+    const DeviceInfo di = device_info();
+    SparseParams p;
+    p.k_cache = cache->k_cache;
+    p.v_cache = cache->v_cache;
+    p.k_index = cache->k_index;
+    p.block_table = batch->block_table;
+    p.seq_lens = batch->seq_lens;
+    p.k_per_seq = k_per_seq;
+    p.q = q;
+    p.P = P;
+    p.out = out;
+    p.sel = selected_idx;
+    p.num_blocks = cache->num_blocks;
+    p.Hkv = Hkv;
+    p.max_blocks = batch->max_blocks_per_seq;
+    p.max_seq_len = batch->max_seq_len;
+    p.index_dims = cache->index_dims;
+    p.r = r;
+    p.k = k;
+    p.W = recent_window;
+    p.group_max = group_reduce == LOKI_GROUP_MAX ? 1 : 0;
+    const double sc = scale == 0.f ? 1.0 / std::sqrt((double)D) : (double)scale;
+    p.scale_log2 = (float)(sc * kLog2e);
+    return dispatch_tdg<SparseLaunch>(cache->dtype, D, G, p, pairs, (int)batch->max_seq_len, di, s, programmatic);
+}
 
 }  // namespace
 
@@ -311,38 +416,9 @@ loki_status loki_prefill_cache(const loki_cache* cache, const loki_batch* batch,
 
 loki_status loki_append_keys(const loki_cache* cache, const loki_batch* batch, const void* k_new,
                              const void* v_new, const float* P, loki_stream_t stream) {
-    loki_status st = check_cache(cache);
-    if (st != LOKI_OK) return st;
-    if ((st = check_batch(batch)) != LOKI_OK) return st;
-    if (batch->batch == 0) return LOKI_OK;
-    if (!k_new || !v_new) return LOKI_ERR_INVALID_ARG;
-    if (P && !aligned16(P)) return LOKI_ERR_INVALID_ARG;
-    if ((int64_t)batch->batch * cache->num_kv_heads > INT32_MAX / 2) return LOKI_ERR_UNSUPPORTED;
-    AppendParams p;
-    p.k_cache = cache->k_cache;
-    p.v_cache = cache->v_cache;
-    p.k_index = cache->k_index;
-    p.index_dims = cache->index_dims;
-    p.block_table = batch->block_table;
-    p.seq_lens = batch->seq_lens;
-    p.k_new = k_new;
-    p.v_new = v_new;
-    p.P = P;
-    p.num_blocks = cache->num_blocks;
-    p.Hkv = cache->num_kv_heads;
-    p.max_blocks = batch->max_blocks_per_seq;
-    p.max_seq_len = batch->max_seq_len;
-    const int grid = batch->batch * cache->num_kv_heads;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const int D = cache->head_dim;
-    if (cache->dtype == LOKI_BF16) {
-        if (D == 64) append_kernel<__nv_bfloat16, 64><<<grid, 256, 0, s>>>(p);
-        else append_kernel<__nv_bfloat16, 128><<<grid, 256, 0, s>>>(p);
-    } else {
-        if (D == 64) append_kernel<float, 64><<<grid, 256, 0, s>>>(p);
-        else append_kernel<float, 128><<<grid, 256, 0, s>>>(p);
-    }
-    return launch_status();
+    const loki_status st = check_append(cache, batch, k_new, v_new, P);
+    if (st != LOKI_OK || batch->batch == 0) return st;
+    return launch_append(cache, batch, k_new, v_new, P, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int32_t loki_decode_max_seq_len(int32_t head_dim, loki_dtype dtype) {
@@ -369,52 +445,28 @@ loki_status loki_decode_attention(const loki_cache* cache, const loki_batch* bat
                                   loki_stream_t stream) {
     (void)workspace;
     (void)workspace_bytes;
-    loki_status st = check_cache(cache);
-    if (st != LOKI_OK) return st;
-    if ((st = check_batch(batch)) != LOKI_OK) return st;
-    const int Hkv = cache->num_kv_heads, D = cache->head_dim;
-    if (num_q_heads < 1 || num_q_heads % Hkv != 0) return LOKI_ERR_INVALID_ARG;
-    if (k < 0 || recent_window < 0 || (k == 0 && recent_window == 0)) return LOKI_ERR_INVALID_ARG;
-    if (r < 1 || r > D) return LOKI_ERR_INVALID_ARG;
-    if (group_reduce != LOKI_GROUP_SUM && group_reduce != LOKI_GROUP_MAX) return LOKI_ERR_INVALID_ARG;
-    if (!(scale >= 0.f) || std::isinf(scale)) return LOKI_ERR_INVALID_ARG;
-    if ((int64_t)k + recent_window > INT32_MAX / 2) return LOKI_ERR_INVALID_ARG;
-    if (batch->batch == 0) return LOKI_OK;
-    if (!q || !P || !out) return LOKI_ERR_INVALID_ARG;
-    if (!aligned16(P) || !aligned16(q)) return LOKI_ERR_INVALID_ARG;
-    const int G = num_q_heads / Hkv;
-    if (G != 1 && G != 2 && G != 4 && G != 8) return LOKI_ERR_UNSUPPORTED;
-    if (r % kSlabDims != 0) return LOKI_ERR_UNSUPPORTED;
-    if (r > cache->index_dims) return LOKI_ERR_INVALID_ARG;
-    const int pairs = batch->batch * Hkv;
-    if ((int64_t)batch->batch * Hkv > 65535) return LOKI_ERR_UNSUPPORTED;
-    if (batch->max_seq_len > loki_decode_max_seq_len(D, cache->dtype)) return LOKI_ERR_UNSUPPORTED;
+    const loki_status st = check_decode(cache, batch, q, num_q_heads, P, r, k, recent_window, group_reduce, scale,
+                                        out);
+    if (st != LOKI_OK || batch->batch == 0) return st;
+    return launch_decode(cache, batch, q, num_q_heads, P, r, k, k_per_seq, recent_window, group_reduce, scale, out,
+                         selected_idx, reinterpret_cast<cudaStream_t>(stream), false);
+}
 
-    const DeviceInfo di = device_info();
-    SparseParams p;
-    p.k_cache = cache->k_cache;
-    p.v_cache = cache->v_cache;
-    p.k_index = cache->k_index;
-    p.block_table = batch->block_table;
-    p.seq_lens = batch->seq_lens;
-    p.k_per_seq = k_per_seq;
-    p.q = q;
-    p.P = P;
-    p.out = out;
-    p.sel = selected_idx;
-    p.num_blocks = cache->num_blocks;
-    p.Hkv = Hkv;
-    p.max_blocks = batch->max_blocks_per_seq;
-    p.max_seq_len = batch->max_seq_len;
-    p.index_dims = cache->index_dims;
-    p.r = r;
-    p.k = k;
-    p.W = recent_window;
-    p.group_max = group_reduce == LOKI_GROUP_MAX ? 1 : 0;
-    const double sc = scale == 0.f ? 1.0 / std::sqrt((double)D) : (double)scale;
-    p.scale_log2 = (float)(sc * kLog2e);
-    return dispatch_tdg<SparseLaunch>(cache->dtype, D, G, p, pairs, (int)batch->max_seq_len, di,
-                                      reinterpret_cast<cudaStream_t>(stream));
+loki_status loki_decode_step(const loki_cache* cache, const loki_batch* batch, const void* k_new, const void* v_new,
+                             const void* q, int32_t num_q_heads, const float* P, int32_t r, int32_t k,
+                             const int32_t* k_per_seq, int32_t recent_window, loki_group_reduce group_reduce,
+                             float scale, float* out, int32_t* selected_idx, void* workspace,
+                             size_t workspace_bytes, loki_stream_t stream) {
+    (void)workspace;
+    (void)workspace_bytes;
+    loki_status st = check_append(cache, batch, k_new, v_new, P);
+    if (st != LOKI_OK) return st;
+    st = check_decode(cache, batch, q, num_q_heads, P, r, k, recent_window, group_reduce, scale, out);
+    if (st != LOKI_OK || batch->batch == 0) return st;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((st = launch_append(cache, batch, k_new, v_new, P, s)) != LOKI_OK) return st;
+    return launch_decode(cache, batch, q, num_q_heads, P, r, k, k_per_seq, recent_window, group_reduce, scale, out,
+                         selected_idx, s, true);
 }
 
 }  // extern "C"

@@ -318,6 +318,13 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
         }
         cp_async_commit();
     };
+    // Launched as the programmatic dependent of the step's append, the kernel
+    // must not read the appended token (position L - 1) before that grid is
+    // done. With a recent window the token is not a scoring candidate and is
+    // first read by the gather; without one the key index may hold it.
+    // (The scoring copies whole 16-token blocks: bytes of a token that is not
+    // a candidate may be read while being written; they are never used.)
+    if (p.W == 0) griddep_wait();
     for (int it = 0; it < S; ++it) refill(it);
     for (int i = tid; i < 2 * kHistBins; i += kThreads) hist[i] = 0;
     if (j0 < nblk_loc) tbl[j0] = tb0;
@@ -667,6 +674,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     }
 
     // ---- 4. exact attention over the kept tokens ----
+    griddep_wait();  // the appended token's key and value rows (no-op when already waited)
     {
         const unsigned char* kbytes = reinterpret_cast<const unsigned char*>(p.k_cache);
         const unsigned char* vbytes = reinterpret_cast<const unsigned char*>(p.v_cache);

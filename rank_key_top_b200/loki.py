@@ -64,6 +64,8 @@ _SIGS = {
     "loki_decode_workspace_bytes": (_SZ, [_C, _B, _I32, _I32, _I32]),
     "loki_decode_attention": (ctypes.c_int, [_C, _B, _P, _I32, _P, _I32, _I32, _P, _I32,
                                              ctypes.c_int, ctypes.c_float, _P, _P, _P, _SZ, _P]),
+    "loki_decode_step": (ctypes.c_int, [_C, _B, _P, _P, _P, _I32, _P, _I32, _I32, _P, _I32,
+                                        ctypes.c_int, ctypes.c_float, _P, _P, _P, _SZ, _P]),
     "loki_decode_max_seq_len": (_I32, [_I32, ctypes.c_int]),
     "loki_dense_workspace_bytes": (_SZ, [_C, _B, _I32]),
     "loki_dense_attention": (ctypes.c_int, [_C, _B, _P, _I32, _P, ctypes.c_float, _P, _P, _SZ, _P]),
@@ -179,6 +181,16 @@ def loki_decode_attention(cache, batch, q, P, r, k, out, k_per_seq=None, recent_
     _check("loki_decode_attention", _lib.loki_decode_attention(
         ctypes.byref(cache.struct), ctypes.byref(batch.struct), _ptr(q), q.shape[1], _ptr(P), r, k,
         _ptr(k_per_seq), recent_window, group_reduce, scale, _ptr(out), _ptr(selected_idx),
+        _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def loki_decode_step(cache, batch, k_new, v_new, q, P, r, k, out, k_per_seq=None, recent_window=0,
+                     group_reduce=LOKI_GROUP_SUM, scale=0.0, selected_idx=None, workspace=None, stream=None):
+    """Append the step's token, then decode (one call, the attention overlapping the append)."""
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("loki_decode_step", _lib.loki_decode_step(
+        ctypes.byref(cache.struct), ctypes.byref(batch.struct), _ptr(k_new), _ptr(v_new), _ptr(q), q.shape[1],
+        _ptr(P), r, k, _ptr(k_per_seq), recent_window, group_reduce, scale, _ptr(out), _ptr(selected_idx),
         _ptr(workspace), ws_bytes, _stream(stream)))
 
 

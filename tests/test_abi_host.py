@@ -122,11 +122,32 @@ def test_decode_rejects_bad_shapes(loki):
                                             FAKE, None, None, 0, None) == 1
 
 
+def step(loki, c, b, k_new=FAKE, v_new=FAKE, Hq=32, r=32, k=8, W=0, q=FAKE, P=FAKE, out=FAKE):
+    return loki.raw().loki_decode_step(ctypes.byref(c), ctypes.byref(b), k_new, v_new, q, Hq, P, r, k, None, W,
+                                       0, 0.0, out, None, None, 0, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(k_new=None), 1),          # append arguments are checked ...
+    (dict(v_new=None), 1),
+    (dict(P=FAKE + 4), 1),
+    (dict(k=0, W=0), 1),            # ... and so are the decode arguments, before any launch
+    (dict(r=24), 2),
+    (dict(Hq=24), 2),
+    (dict(q=None), 1),
+    (dict(out=None), 1),
+])
+def test_decode_step_rejects(loki, kw, status):
+    c, b = structs(loki)
+    assert step(loki, c, b, **kw) == status
+
+
 def test_empty_batch_is_a_no_op(loki):
     c, b = structs(loki, B=0)
     assert decode(loki, c, b, q=None, P=None, out=None) == 0
     assert loki.raw().loki_append_keys(ctypes.byref(c), ctypes.byref(b), None, None, None, None) == 0
     assert loki.raw().loki_prefill_cache(ctypes.byref(c), ctypes.byref(b), None, None, 0, None) == 0
+    assert step(loki, c, b, k_new=None, v_new=None, q=None, P=None, out=None) == 0
 
 
 def test_append_and_prefill_reject(loki):

@@ -257,6 +257,68 @@ def test_append_then_decode(cuda_lib):
             harness.check_pair(wl, b, h, out, sel, s.r, s.k, s.recent_window)
 
 
+@pytest.mark.parametrize("dtype,W,group_max", [("bf16", 4, False), ("bf16", 0, False), ("bf16", 16, True),
+                                               ("f32", 4, False), ("f32", 0, True)])
+def test_decode_step_equals_append_then_decode(cuda_lib, dtype, W, group_max):
+    """loki_decode_step (attention launched as a programmatic dependent of the
+    append) gives bit for bit what the two separate calls give, cache included."""
+    s = spec(num_q_heads=16, num_kv_heads=4, seq_lens=[1999, 37000, 3000], k=300, recent_window=W, dtype=dtype)
+    wl = synth.make_workload(s)
+    k_new, v_new = synth.draw_new_tokens(s, step=5)
+    lens = torch.tensor([n + 1 for n in s.seq_lens], dtype=torch.int32)
+    results = []
+    for fused in (False, True):
+        dev = harness.Device(wl, cuda_lib)
+        dev.batch = cuda_lib.Batch(wl.block_table.cuda(), lens.cuda(), int(lens.max()))
+        out = torch.full((s.batch, s.num_q_heads, s.head_dim), float("nan"), device="cuda")
+        sel = torch.full((s.batch, s.num_kv_heads, s.k + W), -7, dtype=torch.int32, device="cuda")
+        mode = cuda_lib.LOKI_GROUP_MAX if group_max else cuda_lib.LOKI_GROUP_SUM
+        if fused:
+            cuda_lib.loki_decode_step(dev.cache, dev.batch, k_new.cuda(), v_new.cuda(), dev.q, dev.P, s.r, s.k, out,
+                                      recent_window=W, group_reduce=mode, selected_idx=sel)
+        else:
+            cuda_lib.loki_append_keys(dev.cache, dev.batch, k_new.cuda(), v_new.cuda(), dev.P)
+            cuda_lib.loki_decode_attention(dev.cache, dev.batch, dev.q, dev.P, s.r, s.k, out, recent_window=W,
+                                           group_reduce=mode, selected_idx=sel)
+        torch.cuda.synchronize()
+        rows = [t for b in range(s.batch) for h in range(s.num_kv_heads) for t in read_pair(dev, b, h, int(lens[b]))]
+        results.append([out.cpu(), sel.cpu()] + rows)   # the written rows only: the rest of the cache is unset
+    assert cuda_lib.loki_device_error(clear=True) == 0
+    for a, b in zip(*results):
+        assert torch.equal(a, b)
+    assert not torch.isnan(results[1][0]).any()
+
+
+def test_decode_step_repeated_in_one_stream(cuda_lib):
+    """Steps issued back to back: each step's append must not overtake the
+    previous step's attention, nor its attention the append (same token slot
+    rewritten every step with a different key)."""
+    s = spec(num_q_heads=8, num_kv_heads=2, seq_lens=[30000, 12000], k=500, recent_window=8)
+    wl = synth.make_workload(s)
+    lens = torch.tensor([n + 1 for n in s.seq_lens], dtype=torch.int32)
+    steps = [synth.draw_new_tokens(s, step=i) for i in range(6)]
+    outs = {}
+    for fused in (False, True):
+        dev = harness.Device(wl, cuda_lib)
+        dev.batch = cuda_lib.Batch(wl.block_table.cuda(), lens.cuda(), int(lens.max()))
+        kv = [(k.cuda(), v.cuda()) for k, v in steps]
+        res = [torch.empty(s.batch, s.num_q_heads, s.head_dim, device="cuda") for _ in steps]
+        for (k_new, v_new), out in zip(kv, res):
+            if fused:
+                cuda_lib.loki_decode_step(dev.cache, dev.batch, k_new, v_new, dev.q, dev.P, s.r, s.k, out,
+                                          recent_window=s.recent_window)
+            else:
+                cuda_lib.loki_append_keys(dev.cache, dev.batch, k_new, v_new, dev.P)
+                cuda_lib.loki_decode_attention(dev.cache, dev.batch, dev.q, dev.P, s.r, s.k, out,
+                                               recent_window=s.recent_window)
+        torch.cuda.synchronize()
+        outs[fused] = [o.cpu() for o in res]
+    for a, b in zip(outs[False], outs[True]):
+        assert torch.equal(a, b)
+    for i in range(1, len(steps)):     # every step saw its own token
+        assert not torch.equal(outs[True][i], outs[True][i - 1])
+
+
 def test_device_checks_flag_bad_lengths_and_blocks(cuda_lib):
     s = spec(num_q_heads=4, num_kv_heads=1, seq_lens=[500, 600], k=20)
     wl = synth.make_workload(s)
