@@ -122,7 +122,9 @@ void sparse_layout(SparseParams& p, int max_seq_len, int ring_per_warp) {
     const int nblk = (max_seq_len + kBlockTokens - 1) / kBlockTokens;
     p.cta_tokens = std::max(1, (nblk + p.C - 1) / p.C) * kBlockTokens;
     p.slot_bytes = p.r * kBlockTokens * (int)sizeof(T);
-    p.slots = std::min(kMaxSlots, std::max(1, ring_per_warp / p.slot_bytes));
+    // a power of two (the kernel's ring arithmetic relies on it)
+    p.slots = 1;
+    while (2 * p.slots <= kMaxSlots && 2 * p.slots * p.slot_bytes <= ring_per_warp) p.slots *= 2;
     p.ring_bytes_per_warp = p.slots * p.slot_bytes;
     const int list_bytes = align(p.cta_tokens * 2);
     int ring_bytes = align(kWarps * p.ring_bytes_per_warp);

@@ -101,27 +101,6 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
-// cp.async.wait_group with a run-time count n in [0, 15]
-__device__ __forceinline__ void cp_async_wait_n(int n) {
-    switch (n) {
-        case 0: cp_async_wait<0>(); break;
-        case 1: cp_async_wait<1>(); break;
-        case 2: cp_async_wait<2>(); break;
-        case 3: cp_async_wait<3>(); break;
-        case 4: cp_async_wait<4>(); break;
-        case 5: cp_async_wait<5>(); break;
-        case 6: cp_async_wait<6>(); break;
-        case 7: cp_async_wait<7>(); break;
-        case 8: cp_async_wait<8>(); break;
-        case 9: cp_async_wait<9>(); break;
-        case 10: cp_async_wait<10>(); break;
-        case 11: cp_async_wait<11>(); break;
-        case 12: cp_async_wait<12>(); break;
-        case 13: cp_async_wait<13>(); break;
-        case 14: cp_async_wait<14>(); break;
-        default: cp_async_wait<15>(); break;
-    }
-}
 
 // Exclusive prefix sum over the lanes of a warp.
 __device__ __forceinline__ int warp_exclusive_scan(int v, int lane) {
@@ -305,18 +284,24 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
         const int v1 = __shfl_sync(kFull, tb1, it & 31);
         return it < 32 ? v0 : v1;
     };
-    // Ring of S slots per warp: every lane copies 16-byte pieces of a block
-    // with cp.async (pieces lane, lane + 32, ...), one commit group per
-    // iteration (empty past the warp's last block), so that waiting for block
-    // it is cp.async.wait_group S - 1.
-    auto refill = [&](int it) {  // all lanes; slot it % S is free
+    // Ring of S slots per warp (S a power of two dividing kMaxSlots): every
+    // lane copies 16-byte pieces of a block with cp.async (pieces lane,
+    // lane + 32, ...). Each refill commits kMaxSlots / S groups, the block's
+    // and empty ones (all empty past the warp's last block), so that exactly
+    // kMaxSlots - 1 groups are younger than the oldest block in flight and
+    // waiting for it is always cp.async.wait_group kMaxSlots - 1: no run-time
+    // count, no division in the loop.
+    const int smask = S - 1;
+    const int pad = kMaxSlots / S - 1;
+    auto refill = [&](int it) {  // all lanes; slot it & smask is free
         if (it < my_blocks) {
             const int pb = entry(it);
             const unsigned char* src = xbytes + page_offset(pb, h, p.Hkv, p.index_dims) * (int64_t)sizeof(T);
-            unsigned char* dst = wring + (it % S) * p.slot_bytes;
+            unsigned char* dst = wring + (it & smask) * p.slot_bytes;
             for (int o = lane * 16; o < p.slot_bytes; o += 32 * 16) cp_async16(dst + o, src + o, true);
         }
         cp_async_commit();
+        for (int i = 0; i < pad; ++i) cp_async_commit();
     };
     // Launched as the programmatic dependent of the step's append, the kernel
     // must not read the appended token (position L - 1) before that grid is
@@ -380,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     // accumulation. fp32 index: CUDA-core dot products.
     {
         auto wait_slot = [&]() {  // all lanes: the oldest slot in flight has landed
-            cp_async_wait_n(S - 1);
+            cp_async_wait<kMaxSlots - 1>();
             __syncwarp();
         };
         auto mma_body = [&](auto rmax_tag) {
@@ -415,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
             const int arow = (lane & 7) + 8 * ((lane >> 3) & 1), ahalf = lane >> 4;
             for (int it = 0; it < my_blocks; ++it) {
                 wait_slot();
-                const unsigned char* sl = wring + (it % S) * p.slot_bytes;
+                const unsigned char* sl = wring + (it & smask) * p.slot_bytes;
                 uint32_t a[RMAX][4];
 #pragma unroll
                 for (int sb = 0; sb < RMAX; ++sb)
@@ -464,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
             const int tok = lane >> 1, half = lane & 1;
             for (int it = 0; it < my_blocks; ++it) {
                 wait_slot();
-                const T* sl = reinterpret_cast<const T*>(wring + (it % S) * p.slot_bytes);
+                const T* sl = reinterpret_cast<const T*>(wring + (it & smask) * p.slot_bytes);
                 typename V8::raw_t raw[RMAX];
 #pragma unroll
                 for (int sb = 0; sb < RMAX; ++sb)
