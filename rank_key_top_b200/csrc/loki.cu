@@ -480,9 +480,17 @@ int dense_splits(int max_seq_len) { return std::max(1, (max_seq_len + kDenseSpli
 template <typename T, int D, int G>
 struct DenseLaunch {
     static loki_status run(DenseParams p, int batch, cudaStream_t s) {
+        using Geom = DenseGeom<T, D, G>;
+        auto split_kern = dense_split_kernel<T, D, G>;
+        static std::once_flag once;
+        static cudaError_t attr_err = cudaSuccess;
+        std::call_once(once, [&] {
+            attr_err = cudaFuncSetAttribute(split_kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geom::SMEM_BYTES);
+        });
+        if (attr_err != cudaSuccess) return LOKI_ERR_CUDA;
         const int pairs = batch * p.Hkv;
         rotate_query_kernel<T, D, G><<<pairs, 256, 0, s>>>(p);
-        dense_split_kernel<T, D, G><<<dim3(p.splits, pairs), 256, 0, s>>>(p);
+        split_kern<<<dim3(p.splits, pairs), kDenseThreads, Geom::SMEM_BYTES, s>>>(p);
         merge_kernel<D, G><<<batch * p.Hkv * G, D, 0, s>>>(p);
         return launch_status();
     }

@@ -91,16 +91,6 @@ struct SparseGeom {
     static constexpr int QSCRATCH_BYTES = (2048 / D) * G * D * 4;  // row groups x G x D floats
 };
 
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, bool valid) {
-    const int n = valid ? 16 : 0;  // 0: nothing is read, the 16 bytes are zero-filled
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc), "r"(n)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 // Exclusive prefix sum over the lanes of a warp.
 __device__ __forceinline__ int warp_exclusive_scan(int v, int lane) {

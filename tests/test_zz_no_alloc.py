@@ -47,7 +47,7 @@ def test_static_scratch_rejects_sizes_beyond_the_array(cuda_lib):
     lens = torch.zeros(1, dtype=torch.int32, device="cuda")
     cache = cuda_lib.Cache(1, 1, 128, torch.bfloat16)
     # one sequence long enough that the split partials exceed the array
-    max_len = 8_000_000
+    max_len = 16_000_000
     batch = cuda_lib.loki_batch(table.data_ptr(), lens.data_ptr(), 1, max_len // 16, max_len)
     need = cuda_lib.raw().loki_dense_workspace_bytes(ctypes.byref(cache.struct), ctypes.byref(batch), 4)
     assert need > cuda_lib.LOKI_DENSE_STATIC_SCRATCH_BYTES
