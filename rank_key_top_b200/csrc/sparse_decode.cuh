@@ -104,7 +104,8 @@ __device__ __forceinline__ int warp_exclusive_scan(int v, int lane) {
 }
 
 // Exclusive suffix sum over the block: returns sum of v over threads > tid.
-// wsum: 2 * kWarps words of shared scratch.
+// wsum: kWarps words of shared scratch, free again once every thread of the
+// block has passed the next block-wide barrier.
 __device__ __forceinline__ uint32_t block_suffix_exclusive(uint32_t v, uint32_t* wsum, int lane, int warp) {
     uint32_t x = v;
 #pragma unroll
@@ -114,18 +115,15 @@ __device__ __forceinline__ uint32_t block_suffix_exclusive(uint32_t v, uint32_t*
     }
     if (lane == 0) wsum[warp] = x;  // warp total
     __syncthreads();
-    if (warp == 0) {  // suffix over the warp totals, excluding the warp itself
-        uint32_t t = lane < kWarps ? wsum[lane] : 0u;
-        uint32_t s = t;
+    // every warp forms the suffix over the warp totals itself (one barrier)
+    const uint32_t t = lane < kWarps ? wsum[lane] : 0u;
+    uint32_t s = t;
 #pragma unroll
-        for (int o = 1; o < kWarps; o <<= 1) {
-            const uint32_t y = __shfl_down_sync(kFull, s, o);
-            if (lane + o < kWarps) s += y;
-        }
-        if (lane < kWarps) wsum[kWarps + lane] = s - t;
+    for (int o = 1; o < kWarps; o <<= 1) {
+        const uint32_t y = __shfl_down_sync(kFull, s, o);
+        if (lane + o < kWarps) s += y;
     }
-    __syncthreads();
-    return x - v + wsum[kWarps + warp];
+    return x - v + __shfl_sync(kFull, s - t, warp);  // totals of the warps after this one
 }
 
 // One digit of the cluster-wide radix select. Sums the cluster's histograms
@@ -137,8 +135,7 @@ __device__ __forceinline__ uint32_t block_suffix_exclusive(uint32_t v, uint32_t*
 __device__ __noinline__ int2 radix_boundary(const uint32_t* hcur, int nbins, int krem, int32_t* misc, int C) {
     cg::cluster_group cluster = cg::this_cluster();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    __syncthreads();
-    cluster.sync();
+    cluster.sync();  // every thread of every CTA: the histograms are complete and visible
     uint32_t hv[4] = {0u, 0u, 0u, 0u};  // bins 4 tid .. 4 tid + 3
     if (4 * tid < nbins) {
         for (int c = 0; c < C; ++c) {
