@@ -47,6 +47,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["loki", "reference"], default="loki")
     ap.add_argument("--profile", action="store_true",
                     help="only the timed device loop (for ncu): no e2e, dense, CPU baseline or clocks")
+    ap.add_argument("--profile-dense", action="store_true",
+                    help="with --profile: then run the dense-attention path steps + warmup times as well")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle time budget of the CPU baseline")
     return ap.parse_args()
 
@@ -344,6 +346,15 @@ def main():
     assert loki.loki_device_error() == 0
 
     if args.profile:
+        if args.profile_dense:
+            ws = torch.empty(loki.loki_dense_workspace_bytes(cache, batch, spec.num_q_heads), dtype=torch.uint8,
+                             device=dev)
+            dout = torch.empty_like(out)
+            for i in range(args.warmup + K):
+                flush_l2()
+                loki.loki_dense_attention(cache, batch, qs[i % pool], P, dout, ws, stream=stream)
+            torch.cuda.synchronize()
+            assert loki.loki_device_error() == 0
         if rank == 0:
             print(json.dumps({"profile_run": True, "ms_per_step": step_ms / K}), flush=True)
         finish(world)
