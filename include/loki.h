@@ -136,6 +136,29 @@ LOKI_API loki_status loki_prefill_cache(const loki_cache* cache, const loki_batc
                                const void* k_rot, const void* v, int32_t max_len,
                                loki_stream_t stream);
 
+/* Prefill with the rotation on the GPU (AQUA page, appendix on complexity,
+ * step 1, and the information-retention paragraph: keys are projected with P
+ * as row vectors): for every sequence b, kv head h and token t < seq_lens[b],
+ *   K~[b, h, t, :] = round(k[b, h, t, :] P[h]),  V[b, h, t, :] = v[b, h, t, :]
+ * written as loki_prefill_cache lays rows out (key rows, value rows, key
+ * index).
+ *
+ * k, v: device [batch][num_kv_heads][max_len][head_dim] in the cache type,
+ * unrotated keys and values, 16-byte aligned; max_len >= max_seq_len.
+ * P: device fp32 [num_kv_heads][head_dim][head_dim], row-major, 16-byte
+ * aligned.
+ * Precision: fp32 caches sum fp32 products in fp32, as loki_append_keys does.
+ * bf16 caches run the product on the tensor cores with P split into two bf16
+ * terms (P = P_hi + P_lo) and fp32 accumulation, i.e. about 16 significant
+ * bits of P, then round to nearest even: the stored key equals the exactly
+ * rounded product except where that product lies within about 2^-15 of its
+ * magnitude from a rounding midpoint, where it may be the other neighbour.
+ * Tokens past seq_lens[b] are not read. The key index gets the leading
+ * index_dims of every rotated key. */
+LOKI_API loki_status loki_prefill_rotate(const loki_cache* cache, const loki_batch* batch,
+                                const void* k, const void* v, const float* P, int32_t max_len,
+                                loki_stream_t stream);
+
 /* Cache update of one decode step (AQUA page, decode-step equations (1)-(2),
  * for keys kept in the PCA basis): for every sequence b and kv head h,
  *   K~[b, h, seq_lens[b]-1, :] = round(k_new[b, h, :] P[h])   (fp32 accumulation,

@@ -10,6 +10,7 @@
 
 #include "cache_kernels.cuh"
 #include "dense.cuh"
+#include "rotate_prefill.cuh"
 #include "sparse_decode.cuh"
 
 using namespace loki;
@@ -413,6 +414,65 @@ loki_status loki_prefill_cache(const loki_cache* cache, const loki_batch* batch,
         if (D == 64) prefill_kernel<float, 64><<<grid, 256, 0, s>>>(p);
         else prefill_kernel<float, 128><<<grid, 256, 0, s>>>(p);
     }
+    return launch_status();
+}
+
+loki_status loki_prefill_rotate(const loki_cache* cache, const loki_batch* batch, const void* k, const void* v,
+                                const float* P, int32_t max_len, loki_stream_t stream) {
+    loki_status st = check_cache(cache);
+    if (st != LOKI_OK) return st;
+    if ((st = check_batch(batch)) != LOKI_OK) return st;
+    if (batch->batch == 0 || batch->max_seq_len == 0) return LOKI_OK;
+    if (!k || !v || !P) return LOKI_ERR_INVALID_ARG;
+    if (max_len < batch->max_seq_len) return LOKI_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(P)) return LOKI_ERR_INVALID_ARG;
+    if ((int64_t)batch->batch * cache->num_kv_heads > 65535) return LOKI_ERR_UNSUPPORTED;
+    RotateParams p;
+    p.k_cache = cache->k_cache;
+    p.v_cache = cache->v_cache;
+    p.k_index = cache->k_index;
+    p.block_table = batch->block_table;
+    p.seq_lens = batch->seq_lens;
+    p.k = k;
+    p.v = v;
+    p.P = P;
+    p.num_blocks = cache->num_blocks;
+    p.Hkv = cache->num_kv_heads;
+    p.max_blocks = batch->max_blocks_per_seq;
+    p.max_seq_len = batch->max_seq_len;
+    p.max_len = max_len;
+    p.index_dims = cache->index_dims;
+    const int pairs = batch->batch * cache->num_kv_heads;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int D = cache->head_dim;
+    if (cache->dtype == LOKI_BF16) {
+        // enough tiles per CTA that a CTA's split of P is reused, with about
+        // two CTAs per SM in flight
+        const int tiles = (batch->max_seq_len + kRotTile - 1) / kRotTile;
+        const int64_t want = 2LL * std::max(1, device_info().sms);
+        p.tiles_per_cta = (int)std::max<int64_t>(1, ((int64_t)tiles * pairs + want - 1) / want);
+        const dim3 grid((tiles + p.tiles_per_cta - 1) / p.tiles_per_cta, pairs);
+        auto launch = [&](auto kern, int smem) {
+            static std::mutex mu;
+            static std::map<const void*, cudaError_t> done;
+            {
+                std::lock_guard<std::mutex> lk(mu);
+                auto it = done.find((const void*)kern);
+                if (it == done.end())
+                    it = done.emplace((const void*)kern,
+                                      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
+                             .first;
+                if (it->second != cudaSuccess) return LOKI_ERR_CUDA;
+            }
+            kern<<<grid, kRotThreads, smem, s>>>(p);
+            return launch_status();
+        };
+        if (D == 64) return launch(rotate_prefill_tc_kernel<64>, rotate_smem_bytes<64>());
+        return launch(rotate_prefill_tc_kernel<128>, rotate_smem_bytes<128>());
+    }
+    const dim3 grid((batch->max_seq_len + kBlockTokens - 1) / kBlockTokens, pairs);
+    if (D == 64) rotate_prefill_f32_kernel<64><<<grid, 256, 0, s>>>(p);
+    else rotate_prefill_f32_kernel<128><<<grid, 256, 0, s>>>(p);
     return launch_status();
 }
 

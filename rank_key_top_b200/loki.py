@@ -60,6 +60,7 @@ _SIGS = {
     "loki_cache_bytes": (_SZ, [_I32, _I32, _I32, ctypes.c_int]),
     "loki_index_bytes": (_SZ, [_I32, _I32, _I32, ctypes.c_int]),
     "loki_prefill_cache": (ctypes.c_int, [_C, _B, _P, _P, _I32, _P]),
+    "loki_prefill_rotate": (ctypes.c_int, [_C, _B, _P, _P, _P, _I32, _P]),
     "loki_append_keys": (ctypes.c_int, [_C, _B, _P, _P, _P, _P]),
     "loki_decode_workspace_bytes": (_SZ, [_C, _B, _I32, _I32, _I32]),
     "loki_decode_attention": (ctypes.c_int, [_C, _B, _P, _I32, _P, _I32, _I32, _P, _I32,
@@ -94,7 +95,11 @@ def _check(fn, status):
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    if t is None:
+        return None
+    if not t.is_contiguous():  # the C ABI takes dense row-major buffers
+        raise ValueError("tensor arguments must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _stream(stream):
@@ -160,6 +165,14 @@ def loki_prefill_cache(cache, batch, k_rot, v, max_len=None, stream=None):
     max_len = k_rot.shape[2] if max_len is None else max_len
     _check("loki_prefill_cache", _lib.loki_prefill_cache(
         ctypes.byref(cache.struct), ctypes.byref(batch.struct), _ptr(k_rot), _ptr(v), max_len,
+        _stream(stream)))
+
+
+def loki_prefill_rotate(cache, batch, k, v, P, max_len=None, stream=None):
+    """Prefill from unrotated keys: the library computes K~ = K P."""
+    max_len = k.shape[2] if max_len is None else max_len
+    _check("loki_prefill_rotate", _lib.loki_prefill_rotate(
+        ctypes.byref(cache.struct), ctypes.byref(batch.struct), _ptr(k), _ptr(v), _ptr(P), max_len,
         _stream(stream)))
 
 

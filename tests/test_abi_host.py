@@ -159,6 +159,17 @@ def test_append_and_prefill_reject(loki):
     assert lib.loki_prefill_cache(ctypes.byref(c), ctypes.byref(b), FAKE + 2, FAKE, 64, None) == 1
 
 
+def test_prefill_rotate_rejects(loki):
+    c, b = structs(loki)
+    lib = loki.raw()
+    assert lib.loki_prefill_rotate(ctypes.byref(c), ctypes.byref(b), None, FAKE, FAKE, 64, None) == 1
+    assert lib.loki_prefill_rotate(ctypes.byref(c), ctypes.byref(b), FAKE, FAKE, None, 64, None) == 1
+    assert lib.loki_prefill_rotate(ctypes.byref(c), ctypes.byref(b), FAKE, FAKE, FAKE + 4, 64, None) == 1
+    assert lib.loki_prefill_rotate(ctypes.byref(c), ctypes.byref(b), FAKE, FAKE, FAKE, 32, None) == 1  # max_len short
+    c0, b0 = structs(loki, B=0)
+    assert lib.loki_prefill_rotate(ctypes.byref(c0), ctypes.byref(b0), None, None, None, 0, None) == 0
+
+
 def test_dense_rejects(loki):
     c, b = structs(loki)
     lib = loki.raw()

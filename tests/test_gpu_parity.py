@@ -230,6 +230,72 @@ def test_append_matches_oracle(cuda_lib, dtype, D):
     assert not torch.equal(before_k, dev.cache.k)
 
 
+def unrotated_keys(wl):
+    """Keys in the original basis whose rotation is the workload's cache rows:
+    K = K~ P^T (P orthonormal), rounded to the cache type."""
+    K = torch.einsum("bhtd,hed->bhte", wl.Kt.double(), wl.P.double())
+    return K.to(synth.torch_dtype(wl.spec.dtype)).contiguous()
+
+
+@pytest.mark.parametrize("dtype,D,lens", [("bf16", 128, [300, 1000, 0, 1, 129]), ("bf16", 64, [257, 40]),
+                                          ("f32", 128, [300, 17, 0]), ("f32", 64, [65])])
+def test_prefill_rotate_matches_oracle(cuda_lib, dtype, D, lens):
+    """K~ = round(K P) for every prompt token, the value rows copied and the
+    key index filled, read back through the documented layout. bf16 uses the
+    tensor cores with P split into two bf16 terms: a key may differ from the
+    exactly rounded product only where that lies, within the split's error
+    (2^-17 of the products' magnitudes) plus fp32 accumulation, at the
+    rounding midpoint of the two values."""
+    s = spec(num_q_heads=4, num_kv_heads=2, head_dim=D, seq_lens=lens, dtype=dtype, r=16)
+    wl = synth.make_workload(s)
+    dev = harness.Device(wl, cuda_lib, index_dims=32)
+    dev.cache.k.fill_(0xFF)   # every row the call must write starts as a NaN pattern
+    dev.cache.v.fill_(0xFF)
+    dev.cache.x.fill_(0xFF)
+    k_in = unrotated_keys(wl)
+    cuda_lib.loki_prefill_rotate(dev.cache, dev.batch, k_in.cuda(), wl.V.cuda(), dev.P)
+    torch.cuda.synchronize()
+    assert cuda_lib.loki_device_error() == 0
+    split = 2.0 ** -17 if dtype == "bf16" else 0.0
+    for b, L in enumerate(lens):
+        for h in range(s.num_kv_heads):
+            if L == 0:
+                continue
+            K, V, X = read_pair(dev, b, h, L)
+            assert torch.equal(V, wl.V[b, h, :L])
+            assert torch.equal(X, K[:, :dev.cache.index_dims])
+            kk = k_in[b, h, :L].double().numpy()
+            Ph = wl.P[h].double().numpy()
+            want = oracle.append(kk, Ph, dtype)
+            got = K.double().numpy()
+            assert np.all(np.isfinite(got)), (b, h)
+            exact = oracle.rotate(kk, Ph)
+            mag = np.abs(kk) @ np.abs(Ph)
+            bound = (split + D * 2.0 ** -24) * mag
+            mism = got != want
+            assert np.all(np.abs(exact[mism] - (got[mism] + want[mism]) / 2) <= bound[mism]), (b, h, int(mism.sum()))
+
+
+def test_prefill_rotate_long_sequence_many_ctas(cuda_lib):
+    """One long sequence: several 128-token tiles per CTA and several CTAs per
+    (sequence, kv head); a decode on the rotated cache matches the oracle."""
+    s = spec(num_q_heads=4, num_kv_heads=1, seq_lens=[40000], k=500, recent_window=16, r=32)
+    wl = synth.make_workload(s)
+    dev = harness.Device(wl, cuda_lib)
+    k_in = unrotated_keys(wl)
+    cuda_lib.loki_prefill_rotate(dev.cache, dev.batch, k_in.cuda(), wl.V.cuda(), dev.P)
+    torch.cuda.synchronize()
+    assert cuda_lib.loki_device_error() == 0
+    K, V, X = read_pair(dev, 0, 0, 40000)
+    kk = k_in[0, 0].double().numpy()
+    want = oracle.append(kk, wl.P[0].double().numpy(), "bf16")
+    assert np.mean(K.double().numpy() == want) > 0.99
+    # the oracle's view of the cache is what the kernel wrote
+    wl.Kt = K[None, None].clone()
+    out, sel = dev.decode()
+    harness.check_pair(wl, 0, 0, out, sel, s.r, s.k, s.recent_window)
+
+
 def test_append_then_decode(cuda_lib):
     """One whole decode step: append the current token, then attend."""
     s = spec(num_q_heads=8, num_kv_heads=2, seq_lens=[1999, 3000], k=200, recent_window=4)
