@@ -1,0 +1,183 @@
+// Launch geometry of sparse_decode_kernel: the device's SM count and shared
+// memory, the cluster size, the shared-memory layout of a CTA (key ring depth,
+// regions) and the launch itself. Host code; kept beside the kernel because
+// together they fix what the kernel does on the device.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "sparse_decode.cuh"
+
+namespace loki {
+
+struct DeviceInfo {
+    int sms = 0;
+    int max_smem_optin = 0;
+};
+
+inline DeviceInfo device_info() {
+    static std::mutex mu;
+    static DeviceInfo cache[64];
+    static bool have[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev >= 0 && dev < 64 && have[dev]) return cache[dev];
+    DeviceInfo di;
+    cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&di.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (dev >= 0 && dev < 64) {
+        cache[dev] = di;
+        have[dev] = true;
+    }
+    return di;
+}
+
+// Whether at least one cluster of this shape can be resident on the device,
+// cached per kernel instantiation, cluster size and shared-memory size.
+template <typename K>
+bool cluster_fits(K kern, const cudaLaunchConfig_t& cfg, std::map<std::pair<int, int>, bool>& known,
+                  std::mutex& mu) {
+    const std::pair<int, int> key(cfg.gridDim.x, (int)cfg.dynamicSmemBytes);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = known.find(key);
+    if (it != known.end()) return it->second;
+    int n = 0;
+    cudaLaunchConfig_t probe = cfg;
+    probe.gridDim = dim3(cfg.gridDim.x, 1, 1);
+    const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kern, &probe);
+    if (e != cudaSuccess) cudaGetLastError();
+    const bool fits = e == cudaSuccess && n > 0;
+    known[key] = fits;
+    return fits;
+}
+
+// Shared-memory layout of one CTA for C CTAs per (sequence, kv head), with a
+// key-index ring of ring_per_warp bytes per warp.
+template <typename T, int D, int G>
+void sparse_layout(SparseParams& p, int max_seq_len, int ring_per_warp) {
+    using Geom = SparseGeom<T, D, G>;
+    auto align = [](int x) { return (x + 127) & ~127; };
+    const int nblk = (max_seq_len + kBlockTokens - 1) / kBlockTokens;
+    p.cta_tokens = std::max(1, (nblk + p.C - 1) / p.C) * kBlockTokens;
+    p.slot_bytes = p.r * kBlockTokens * (int)sizeof(T);
+    // a power of two (the kernel's ring arithmetic relies on it)
+    p.slots = 1;
+    while (2 * p.slots <= kMaxSlots && 2 * p.slots * p.slot_bytes <= ring_per_warp) p.slots *= 2;
+    p.ring_bytes_per_warp = p.slots * p.slot_bytes;
+    const int list_bytes = align(p.cta_tokens * 2);
+    int ring_bytes = align(kWarps * p.ring_bytes_per_warp);
+    // after the scoring the ring region holds the select's candidate
+    // segments (head, up to one key per token) and the kept list (tail)
+    const int cand_bytes = align(p.cta_tokens * 4);
+    if (ring_bytes < list_bytes + cand_bytes) ring_bytes = list_bytes + cand_bytes;
+    int keys_bytes = align(std::max(p.cta_tokens * 4, Geom::QSCRATCH_BYTES));
+    // the gather stages rows in keys + ring minus the list; the warp partials
+    // of the merge go to keys + ring
+    const int staged = std::max(Geom::STAGE_BYTES + list_bytes, Geom::WPART_BYTES);
+    if (keys_bytes + ring_bytes < staged) keys_bytes = align(staged - ring_bytes);
+    int off = 0;
+    p.off_keys = off;
+    p.keys_bytes = keys_bytes;
+    off += keys_bytes;
+    p.off_ring = off;
+    p.ring_bytes = ring_bytes;
+    off += ring_bytes;
+    p.off_list = p.off_ring + ring_bytes - list_bytes;
+    p.off_qf = off;  // merge weights
+    off = align(off + G * kWarps * 4);
+    p.off_qhat = off;
+    off = align(off + G * D * 4);
+    p.off_qs = off;
+    off = align(off + D * 4);
+    p.off_tbl = off;
+    off = align(off + (p.cta_tokens / kBlockTokens) * 4);
+    p.off_hist = off;
+    off = align(off + 2 * kHistBins * 4);
+    p.off_part = off;  // one partial slot per CTA of the cluster (used in rank 0)
+    off = align(off + p.C * G * (D + 2) * 4);
+    p.off_misc = off;
+    off = align(off + 128 * 4);
+    p.smem_bytes = off;
+}
+
+// The layout with the deepest key-index ring that fits in shared memory.
+template <typename T, int D, int G>
+bool sparse_layout_fit(SparseParams& p, int max_seq_len, int smem_optin) {
+    for (int ring_per_warp : {8192, 6144, 4096, 2048}) {
+        sparse_layout<T, D, G>(p, max_seq_len, ring_per_warp);
+        if (p.smem_bytes <= smem_optin) return true;
+    }
+    return false;
+}
+
+// Cluster size: enough CTAs that each holds at most kCtaTokenCap tokens and
+// the layout fits in shared memory, then as many as still fit every cluster
+// on the GPU at once (one CTA per SM), keeping at least 512 tokens per CTA.
+template <typename T, int D, int G>
+int choose_cluster(SparseParams& p, int max_seq_len, int pairs, int sms, int smem_optin) {
+    const int nblk = (max_seq_len + kBlockTokens - 1) / kBlockTokens;
+    const int cap_blocks = kCtaTokenCap / kBlockTokens;
+    int C = std::max(1, (nblk + cap_blocks - 1) / cap_blocks);
+    for (;; ++C) {
+        if (C > 16) return -1;
+        p.C = C;
+        if (sparse_layout_fit<T, D, G>(p, max_seq_len, smem_optin)) break;
+    }
+    for (int cand = C + 1; cand <= 16; ++cand) {
+        if ((int64_t)pairs * cand > sms) break;
+        if (nblk / cand < 32) break;
+        C = cand;
+    }
+    p.C = C;
+    sparse_layout_fit<T, D, G>(p, max_seq_len, smem_optin);
+    return C;
+}
+
+template <typename T, int D, int G>
+struct SparseLaunch {
+    static loki_status run(SparseParams p, int pairs, int max_seq_len, const DeviceInfo& di,
+                           cudaStream_t stream, bool programmatic) {
+        if (choose_cluster<T, D, G>(p, max_seq_len, pairs, di.sms, di.max_smem_optin) < 1)
+            return LOKI_ERR_UNSUPPORTED;
+        auto kern = sparse_decode_kernel<T, D, G>;
+        static std::once_flag once;
+        static cudaError_t attr_err = cudaSuccess;
+        std::call_once(once, [&] {
+            attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, di.max_smem_optin);
+            if (attr_err == cudaSuccess)
+                attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        });
+        if (attr_err != cudaSuccess) return LOKI_ERR_CUDA;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(p.C, pairs, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = p.smem_bytes;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = p.C;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        // programmatic dependent of the previous kernel in the stream (the
+        // step's append): the kernel calls griddep_wait() before it reads
+        // anything that kernel writes
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = programmatic ? 2 : 1;
+        // a cluster that can never be resident is reported, not launched
+        static std::map<std::pair<int, int>, bool> known;
+        static std::mutex known_mu;
+        if (!cluster_fits(kern, cfg, known, known_mu)) return LOKI_ERR_UNSUPPORTED;
+        if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return LOKI_ERR_CUDA;
+        return cudaPeekAtLastError() == cudaSuccess ? LOKI_OK : LOKI_ERR_CUDA;
+    }
+};
+
+}  // namespace loki
