@@ -78,7 +78,7 @@ typedef enum loki_group_reduce {
 #define LOKI_DEVERR_SEQ_LEN 0x1u  /* a seq_lens entry outside [0, max_seq_len] */
 #define LOKI_DEVERR_BLOCK_ID 0x2u /* a block-table entry outside [0, num_blocks) */
 #define LOKI_DEVERR_K 0x4u        /* a k_per_seq entry outside [0, k] */
-#define LOKI_DEVERR_TIMEOUT 0x8u  /* reserved: no current kernel spins on a wait */
+#define LOKI_DEVERR_TIMEOUT 0x8u  /* a bounded wait (tensor-core completion) gave up */
 
 /* Paged KV cache in the library's own layout (LOKI_BLOCK_TOKENS tokens per
  * block), plus a low-rank key index. Physical block p of kv head h holds:
