@@ -12,9 +12,10 @@
 // 128-byte swizzle) into a D x 128 fp32 accumulator in tensor memory: the
 // products of bf16 keys with each term are exact and the sum is accumulated
 // in fp32, so the result carries about 16 significant bits of P before it is
-// rounded to bf16. The epilogue reads the accumulator with tcgen05.ld (warp w
-// owns lanes 32w .. 32w + 31, i.e. tokens), rounds to nearest even and
-// writes key rows and index dims; the value rows are copied.
+// rounded to bf16. The epilogue reads the accumulator with tcgen05.ld (warps w
+// and w + 4 own lanes 32 (w % 4) .. + 31, i.e. tokens, and split the columns),
+// rounds to nearest even and writes key rows and index dims; the value rows
+// are copied, one 16-token block per warp.
 // fp32 caches: CUDA cores, fp32 products and sums, as the step's append.
 #pragma once
 
@@ -36,7 +37,7 @@ struct RotateParams {
 };
 
 constexpr int kRotTile = 128;     // tokens per MMA tile (the M of the instruction)
-constexpr int kRotThreads = 128;  // 4 warps: one per 32 accumulator lanes
+constexpr int kRotThreads = 256;  // 8 warps: warps w and w + 4 read accumulator lanes 32 (w % 4) .. + 31
 
 // ---------------------------------------------------------------------------
 // tcgen05 / tensor-memory wrappers (cta_group::1)
@@ -240,16 +241,20 @@ __global__ void __launch_bounds__(kRotThreads) rotate_prefill_tc_kernel(const Ro
             }
             umma_commit(bar);
         }
-        // the tile's value rows: warp w copies blocks 2w and 2w + 1 of the tile,
-        // each 16 rows contiguous in the source and in its cache page; the loads
-        // are issued before the wait for the MMAs, the stores after it
+        // the tile's value rows: warp w copies block w of the tile (16 rows,
+        // contiguous in the source and in its cache page); the loads are issued
+        // before the wait for the MMAs, the stores after it
         constexpr int PPL = D / 16;  // 16-byte pieces per lane of one block (16 rows x D bf16)
-        uint4 val[2][PPL];
-        unsigned char* vdst[2] = {nullptr, nullptr};
-        int vbytes[2] = {0, 0};
+        constexpr int BPW = kRotTile / kBlockTokens / (kRotThreads / 32);  // blocks per warp
+        static_assert(BPW >= 1 && BPW * kBlockTokens * (kRotThreads / 32) == kRotTile, "blocks per warp");
+        uint4 val[BPW][PPL];
+        unsigned char* vdst[BPW];
+        int vbytes[BPW];
 #pragma unroll
-        for (int bi = 0; bi < 2; ++bi) {
-            const int tb = t_base + (2 * warp + bi) * kBlockTokens;
+        for (int bi = 0; bi < BPW; ++bi) {
+            vdst[bi] = nullptr;
+            vbytes[bi] = 0;
+            const int tb = t_base + (BPW * warp + bi) * kBlockTokens;
             if (tb >= L) continue;
             const int pb = trow[tb >> 4];
             if (pb < 0 || pb >= p.num_blocks) {
@@ -266,7 +271,7 @@ __global__ void __launch_bounds__(kRotThreads) rotate_prefill_tc_kernel(const Ro
             }
         }
         // this thread's token for the epilogue, and its block
-        const int r = 32 * warp + lane;
+        const int r = 32 * (warp & 3) + lane;
         const int t = t_base + r;
         int pb = -1;
         if (t < L) {
@@ -281,18 +286,20 @@ __global__ void __launch_bounds__(kRotThreads) rotate_prefill_tc_kernel(const Ro
         tc_fence_after();
         if (ti + 1 < ntiles && ok) load_a(ti + 1);  // the MMAs are done with A
 #pragma unroll
-        for (int bi = 0; bi < 2; ++bi) {
+        for (int bi = 0; bi < BPW; ++bi) {
 #pragma unroll
             for (int j = 0; j < PPL; ++j) {
                 const int o = (lane + 32 * j) * 16;
                 if (o < vbytes[bi]) *reinterpret_cast<uint4*>(vdst[bi] + o) = val[bi][j];
             }
         }
-        // epilogue: thread (warp w, lane l) holds token t_base + 32 w + l
+        // epilogue: thread (warp w, lane l) holds token t_base + 32 (w % 4) + l,
+        // columns [w / 4 * D / 2, + D / 2)
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
+        for (int cc = 0; cc < D / 2; cc += 32) {
+            const int c0 = (warp >> 2) * (D / 2) + cc;
             uint32_t acc[32];
-            tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)c0, acc);
+            tmem_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)c0, acc);
             tmem_ld_wait();
             if (ok && pb >= 0) {
                 uint32_t w[16];
