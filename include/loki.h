@@ -159,6 +159,25 @@ LOKI_API loki_status loki_prefill_rotate(const loki_cache* cache, const loki_bat
                                 const void* k, const void* v, const float* P, int32_t max_len,
                                 loki_stream_t stream);
 
+/* Offline calibration of P (AQUA page, appendix on SVD: the leading columns
+ * of the basis carry the most variance; Fig. 2: P calibrated once on
+ * calibration keys): for every head h, the eigenvectors of the centred
+ * covariance C = (1/n) sum_t (x_t - mu)^T (x_t - mu) of its n calibration
+ * keys, as the columns of P[h] in descending eigenvalue order (ties to the
+ * lower index), each column's sign chosen so that its entry of largest
+ * magnitude is positive.
+ *
+ * keys: device [num_heads][n][head_dim] in `dtype`, original basis.
+ * P: device fp32 [num_heads][head_dim][head_dim], row-major (written).
+ * eigvals: nullable device fp32 [num_heads][head_dim] (written, descending).
+ * Arithmetic: fp32 (covariance sums, cyclic Jacobi rotations until every
+ * off-diagonal entry is below 2^-22 of the largest diagonal one); directions
+ * of clustered eigenvalues are defined only up to rotations within the
+ * cluster. n >= 2. No counterpart call in the pages: it is their offline
+ * calibration step done on the device. */
+LOKI_API loki_status loki_pca_basis(const void* keys, int32_t num_heads, int64_t n, int32_t head_dim,
+                           loki_dtype dtype, float* P, float* eigvals, loki_stream_t stream);
+
 /* Cache update of one decode step (AQUA page, decode-step equations (1)-(2),
  * for keys kept in the PCA basis): for every sequence b and kv head h,
  *   K~[b, h, seq_lens[b]-1, :] = round(k_new[b, h, :] P[h])   (fp32 accumulation,

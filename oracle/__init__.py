@@ -38,6 +38,8 @@ def _load():
         lib.oracle_round_bf16_array.argtypes = [_D, ctypes.c_int64, _D, _U16]
         lib.oracle_rotate.restype = None
         lib.oracle_rotate.argtypes = [_D, _D, ctypes.c_int64, ctypes.c_int, _D]
+        lib.oracle_covariance.restype = None
+        lib.oracle_covariance.argtypes = [_D, ctypes.c_int64, ctypes.c_int, _D]
         lib.oracle_append.restype = None
         lib.oracle_append.argtypes = [_D, _D, ctypes.c_int64, ctypes.c_int, ctypes.c_int, _D]
         lib.oracle_attend_set.restype = None
@@ -89,6 +91,29 @@ def rotate(x, P):
     out = np.empty((n, d))
     _load().oracle_rotate(_p(x), _p(P), n, d, _p(out))
     return out
+
+
+def covariance(x):
+    """Centred covariance (1/n) of the rows of x [n, d] (oracle.c)."""
+    x = _f64(x)
+    n, d = x.shape
+    C = np.empty((d, d))
+    _load().oracle_covariance(_p(x), n, d, _p(C))
+    return C
+
+
+def pca_basis(keys):
+    """P from calibration keys [n, d]: the eigenvectors of their centred
+    covariance as columns, in descending eigenvalue order, each column's sign
+    fixed so that its entry of largest magnitude is positive. Returns
+    (P [d, d], eigenvalues [d]). numpy's symmetric eigensolver is the step
+    that diagonalises the covariance."""
+    lam, vec = np.linalg.eigh(covariance(keys))
+    order = np.argsort(-lam, kind="stable")
+    lam, vec = lam[order], vec[:, order]
+    idx = np.argmax(np.abs(vec), axis=0)
+    vec = vec * np.sign(vec[idx, np.arange(vec.shape[1])])[None, :]
+    return vec, lam
 
 
 def append(k_new, P, dtype):

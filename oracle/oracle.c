@@ -350,6 +350,34 @@ int oracle_decode_batch(int n_pairs, const double* Kt, const double* V, const do
     return bad ? -1 : 0;
 }
 
+/* ------------------------------------------------------------------------- */
+/* Offline calibration of P: the principal directions of calibration keys.   */
+/* AQUA page, appendix on SVD (the basis whose leading columns hold the most */
+/* variance) and Fig. 2 (P calibrated once, on other data). The covariance   */
+/* is centred and normalised by 1/n (this oracle's reading; the directions   */
+/* do not depend on the normalisation). The eigendecomposition itself is a   */
+/* library step of the Python wrapper.                                       */
+/*   C[i][j] = (1/n) sum_t (x[t][i] - mu[i]) (x[t][j] - mu[j]),              */
+/*   mu[i]   = (1/n) sum_t x[t][i].                                          */
+/* ------------------------------------------------------------------------- */
+void oracle_covariance(const double* x, int64_t n, int d, double* C)
+{
+    double* mu = (double*)calloc((size_t)d, sizeof(double));
+    for (int64_t t = 0; t < n; ++t)
+        for (int i = 0; i < d; ++i)
+            mu[i] += x[t * d + i];
+    for (int i = 0; i < d; ++i)
+        mu[i] /= (double)n;
+    for (int i = 0; i < d; ++i)
+        for (int j = 0; j < d; ++j) {
+            double s = 0.0;
+            for (int64_t t = 0; t < n; ++t)
+                s += (x[t * d + i] - mu[i]) * (x[t * d + j] - mu[j]);
+            C[i * d + j] = s / (double)n;
+        }
+    free(mu);
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

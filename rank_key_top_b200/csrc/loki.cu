@@ -10,6 +10,7 @@
 
 #include "cache_kernels.cuh"
 #include "dense.cuh"
+#include "pca.cuh"
 #include "rotate_prefill.cuh"
 #include "sparse_decode.cuh"
 #include "sparse_launch.cuh"
@@ -307,6 +308,44 @@ loki_status loki_prefill_rotate(const loki_cache* cache, const loki_batch* batch
     if (D == 64) rotate_prefill_f32_kernel<64><<<grid, 256, 0, s>>>(p);
     else rotate_prefill_f32_kernel<128><<<grid, 256, 0, s>>>(p);
     return launch_status();
+}
+
+loki_status loki_pca_basis(const void* keys, int32_t num_heads, int64_t n, int32_t head_dim, loki_dtype dtype,
+                           float* P, float* eigvals, loki_stream_t stream) {
+    if (num_heads < 0 || n < 0) return LOKI_ERR_INVALID_ARG;
+    if (dtype != LOKI_F32 && dtype != LOKI_BF16) return LOKI_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return LOKI_ERR_UNSUPPORTED;
+    if (num_heads == 0) return LOKI_OK;
+    if (n < 2) return LOKI_ERR_INVALID_ARG;
+    if (!keys || !P) return LOKI_ERR_INVALID_ARG;
+    if (num_heads > 65535) return LOKI_ERR_UNSUPPORTED;
+    PcaParams p;
+    p.keys = keys;
+    p.P = P;
+    p.eigvals = eigvals;
+    p.n = n;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    auto launch = [&](auto kern, int smem) {
+        static std::mutex mu;
+        static std::map<const void*, cudaError_t> done;
+        {
+            std::lock_guard<std::mutex> lk(mu);
+            auto it = done.find((const void*)kern);
+            if (it == done.end())
+                it = done.emplace((const void*)kern,
+                                  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
+                         .first;
+            if (it->second != cudaSuccess) return LOKI_ERR_CUDA;
+        }
+        kern<<<num_heads, kPcaThreads, smem, s>>>(p);
+        return launch_status();
+    };
+    if (dtype == LOKI_BF16) {
+        if (head_dim == 64) return launch(pca_kernel<__nv_bfloat16, 64>, pca_smem_bytes<64>());
+        return launch(pca_kernel<__nv_bfloat16, 128>, pca_smem_bytes<128>());
+    }
+    if (head_dim == 64) return launch(pca_kernel<float, 64>, pca_smem_bytes<64>());
+    return launch(pca_kernel<float, 128>, pca_smem_bytes<128>());
 }
 
 loki_status loki_append_keys(const loki_cache* cache, const loki_batch* batch, const void* k_new,

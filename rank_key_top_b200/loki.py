@@ -61,6 +61,7 @@ _SIGS = {
     "loki_index_bytes": (_SZ, [_I32, _I32, _I32, ctypes.c_int]),
     "loki_prefill_cache": (ctypes.c_int, [_C, _B, _P, _P, _I32, _P]),
     "loki_prefill_rotate": (ctypes.c_int, [_C, _B, _P, _P, _P, _I32, _P]),
+    "loki_pca_basis": (ctypes.c_int, [_P, _I32, ctypes.c_int64, _I32, ctypes.c_int, _P, _P, _P]),
     "loki_append_keys": (ctypes.c_int, [_C, _B, _P, _P, _P, _P]),
     "loki_decode_workspace_bytes": (_SZ, [_C, _B, _I32, _I32, _I32]),
     "loki_decode_attention": (ctypes.c_int, [_C, _B, _P, _I32, _P, _I32, _I32, _P, _I32,
@@ -174,6 +175,13 @@ def loki_prefill_rotate(cache, batch, k, v, P, max_len=None, stream=None):
     _check("loki_prefill_rotate", _lib.loki_prefill_rotate(
         ctypes.byref(cache.struct), ctypes.byref(batch.struct), _ptr(k), _ptr(v), _ptr(P), max_len,
         _stream(stream)))
+
+
+def loki_pca_basis(keys, P, eigvals=None, stream=None):
+    """P[h] from calibration keys [heads][n][d] (device, bf16 or fp32)."""
+    H, n, d = keys.shape
+    _check("loki_pca_basis", _lib.loki_pca_basis(_ptr(keys), H, n, d, dtype_code(keys.dtype), _ptr(P),
+                                                 _ptr(eigvals), _stream(stream)))
 
 
 def loki_append_keys(cache, batch, k_new, v_new, P, stream=None):

@@ -170,6 +170,16 @@ def test_prefill_rotate_rejects(loki):
     assert lib.loki_prefill_rotate(ctypes.byref(c0), ctypes.byref(b0), None, None, None, 0, None) == 0
 
 
+def test_pca_basis_rejects(loki):
+    lib = loki.raw()
+    assert lib.loki_pca_basis(None, 2, 100, 128, 1, FAKE, None, None) == 1
+    assert lib.loki_pca_basis(FAKE, 2, 100, 128, 1, None, None, None) == 1
+    assert lib.loki_pca_basis(FAKE, 2, 1, 128, 1, FAKE, None, None) == 1       # n < 2
+    assert lib.loki_pca_basis(FAKE, 2, 100, 96, 1, FAKE, None, None) == 2      # head dim
+    assert lib.loki_pca_basis(FAKE, 2, 100, 128, 7, FAKE, None, None) == 1     # dtype
+    assert lib.loki_pca_basis(None, 0, 100, 128, 1, None, None, None) == 0     # no heads: no-op
+
+
 def test_dense_rejects(loki):
     c, b = structs(loki)
     lib = loki.raw()

@@ -296,6 +296,40 @@ def test_prefill_rotate_long_sequence_many_ctas(cuda_lib):
     harness.check_pair(wl, 0, 0, out, sel, s.r, s.k, s.recent_window)
 
 
+@pytest.mark.parametrize("dtype,D,n", [("bf16", 128, 4096), ("f32", 128, 1000), ("bf16", 64, 3000)])
+def test_pca_basis_matches_oracle(cuda_lib, dtype, D, n):
+    """P calibrated on the GPU from sample keys in the original basis against
+    the oracle's eigendecomposition of the same keys' centred covariance:
+    spectrum, leading subspaces, the well-separated leading directions (with
+    the sign convention), orthonormality and reconstruction, within what fp32
+    sums over n keys allow."""
+    s = spec(num_q_heads=4, num_kv_heads=2, head_dim=D, seq_lens=[n], dtype=dtype, r=16,
+             outlier_channels=4)
+    wl = synth.make_workload(s)
+    keys = unrotated_keys(wl)[0].contiguous()          # [heads][n][D]
+    P = torch.full((2, D, D), float("nan"), device="cuda")
+    lam = torch.full((2, D), float("nan"), device="cuda")
+    cuda_lib.loki_pca_basis(keys.cuda(), P, lam)
+    torch.cuda.synchronize()
+    assert cuda_lib.loki_device_error() == 0
+    for h in range(2):
+        x = keys[h].double().numpy()
+        Pr, lr = oracle.pca_basis(x)
+        C = oracle.covariance(x)
+        Pg, lg = P[h].cpu().double().numpy(), lam[h].cpu().double().numpy()
+        top = lr[0]
+        assert np.all(np.abs(lg - lr) <= 1e-3 * top), (h, np.abs(lg - lr).max())
+        assert np.all(np.diff(lg) <= 0)
+        assert np.abs(Pg.T @ Pg - np.eye(D)).max() <= 1e-4
+        assert np.abs(Pg @ np.diag(lg) @ Pg.T - C).max() <= 1e-3 * top
+        for r in (8, 16, 32):
+            gap = (lr[r - 1] - lr[r]) / top
+            err = np.linalg.norm(Pg[:, :r] @ Pg[:, :r].T - Pr[:, :r] @ Pr[:, :r].T, 2)
+            assert err <= 1e-3 / max(gap, 1e-3), (h, r, err, gap)
+        for j in range(4):   # the leading directions are well separated here
+            assert np.abs(Pg[:, j] - Pr[:, j]).max() <= 1e-3, (h, j)
+
+
 def test_append_then_decode(cuda_lib):
     """One whole decode step: append the current token, then attend."""
     s = spec(num_q_heads=8, num_kv_heads=2, seq_lens=[1999, 3000], k=200, recent_window=4)

@@ -456,3 +456,41 @@ def test_golden_fixture(name):
     if "expect_out" in fx:
         np.testing.assert_allclose(res.out, np.array(fx["expect_out"], float),
                                    rtol=0, atol=fx.get("atol", 1e-14))
+
+
+# ---------------------------------------------------------------------------
+# Offline calibration of P (AQUA page, appendix on SVD; Fig. 2)
+# ---------------------------------------------------------------------------
+
+def test_covariance_closed_form_and_centring():
+    # four keys on the axes: mean 0, C = diag((1 + 1) / 4, (4 + 4) / 4)
+    x = np.array([[1.0, 0.0], [-1.0, 0.0], [0.0, 2.0], [0.0, -2.0]])
+    assert np.allclose(oracle.covariance(x), np.diag([0.5, 2.0]), atol=0, rtol=0)
+    # a common offset changes nothing (the covariance is centred)
+    assert np.allclose(oracle.covariance(x + np.array([3.0, -1.0])), np.diag([0.5, 2.0]), atol=1e-15)
+    # 1/n normalisation, not 1/(n - 1)
+    y = np.array([[0.0], [2.0]])
+    assert oracle.covariance(y)[0, 0] == 1.0
+
+
+def test_pca_basis_known_answer_and_conventions():
+    x = np.array([[1.0, 0.0], [-1.0, 0.0], [0.0, 2.0], [0.0, -2.0]])
+    P, lam = oracle.pca_basis(x)
+    assert np.allclose(lam, [2.0, 0.5])
+    assert np.allclose(P, [[0.0, 1.0], [1.0, 0.0]])   # descending order, largest entry of each column positive
+
+
+def test_pca_basis_eigen_equation_and_rotation_equivariance():
+    rng = np.random.default_rng(5)
+    d, n = 16, 400
+    x = rng.standard_normal((n, d)) @ np.diag(np.arange(d, 0, -1.0))
+    P, lam = oracle.pca_basis(x)
+    C = oracle.covariance(x)
+    assert np.allclose(P.T @ P, np.eye(d), atol=1e-12)
+    assert np.allclose(C @ P, P * lam[None, :], atol=1e-9)
+    assert np.all(np.diff(lam) <= 0)
+    # keys rotated by an orthonormal Q: same spectrum, directions rotated by Q^T
+    Q, _ = np.linalg.qr(rng.standard_normal((d, d)))
+    P2, lam2 = oracle.pca_basis(x @ Q)
+    assert np.allclose(lam2, lam, rtol=1e-10)
+    assert np.allclose(np.abs(np.sum(P2 * (Q.T @ P), axis=0)), 1.0, atol=1e-9)
