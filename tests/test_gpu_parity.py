@@ -330,6 +330,32 @@ def test_pca_basis_matches_oracle(cuda_lib, dtype, D, n):
             assert np.abs(Pg[:, j] - Pr[:, j]).max() <= 1e-3, (h, j)
 
 
+@pytest.mark.parametrize("where", ["start", "end", "blocks"])
+def test_position_biased_scores(cuda_lib, where):
+    """Scores concentrated in one part of the sequence (an attention sink at
+    the start, the most recent tokens, or a few scattered blocks): nearly all
+    kept tokens fall in one CTA of the cluster and the boundary bins are
+    skewed. Set and output parity as everywhere."""
+    s = spec(num_q_heads=8, num_kv_heads=2, seq_lens=[40000, 21000], k=700, recent_window=8, r=32)
+    wl = synth.make_workload(s)
+    Kt = wl.Kt.float()
+    for b, L in enumerate(s.seq_lens):
+        if where == "start":
+            Kt[b, :, :1500] *= 3.0
+        elif where == "end":
+            Kt[b, :, L - 2000:L] *= 3.0
+        else:
+            for blk in range(7, L // 16, 97):
+                Kt[b, :, 16 * blk:16 * blk + 16] *= 3.0
+    wl.Kt = Kt.to(wl.Kt.dtype)
+    dev = harness.Device(wl, cuda_lib)
+    out, sel = dev.decode()
+    assert cuda_lib.loki_device_error() == 0
+    for b in range(s.batch):
+        for h in range(s.num_kv_heads):
+            harness.check_pair(wl, b, h, out, sel, s.r, s.k, s.recent_window)
+
+
 def test_append_then_decode(cuda_lib):
     """One whole decode step: append the current token, then attend."""
     s = spec(num_q_heads=8, num_kv_heads=2, seq_lens=[1999, 3000], k=200, recent_window=4)
@@ -417,6 +443,41 @@ def test_decode_step_repeated_in_one_stream(cuda_lib):
         assert torch.equal(a, b)
     for i in range(1, len(steps)):     # every step saw its own token
         assert not torch.equal(outs[True][i], outs[True][i - 1])
+
+
+def test_decode_step_in_a_cuda_graph(cuda_lib):
+    """The bench's form of a step: loki_decode_step captured in a CUDA graph
+    (the programmatic dependency between its two kernels becomes a graph
+    edge) and replayed gives what the eager calls give, bit for bit."""
+    s = spec(num_q_heads=16, num_kv_heads=4, seq_lens=[9000, 33000], k=400, recent_window=32)
+    wl = synth.make_workload(s)
+    lens = torch.tensor([n + 1 for n in s.seq_lens], dtype=torch.int32)
+    k_new, v_new = synth.draw_new_tokens(s, step=2)
+    results = []
+    for graphed in (False, True):
+        dev = harness.Device(wl, cuda_lib)
+        dev.batch = cuda_lib.Batch(wl.block_table.cuda(), lens.cuda(), int(lens.max()))
+        kd, vd = k_new.cuda(), v_new.cuda()
+        out = torch.full((s.batch, s.num_q_heads, s.head_dim), float("nan"), device="cuda")
+        stream = torch.cuda.Stream()
+        with torch.cuda.stream(stream):
+            def step():
+                cuda_lib.loki_decode_step(dev.cache, dev.batch, kd, vd, dev.q, dev.P, s.r, s.k, out,
+                                          recent_window=s.recent_window, stream=stream)
+            if graphed:
+                step()                      # warm-up outside the capture
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    step()
+                out.fill_(float("nan"))
+                for _ in range(3):
+                    g.replay()
+            else:
+                step()
+        torch.cuda.synchronize()
+        results.append(out.cpu())
+    assert cuda_lib.loki_device_error() == 0
+    assert torch.equal(results[0], results[1])
 
 
 def test_device_checks_flag_bad_lengths_and_blocks(cuda_lib):
