@@ -1,30 +1,34 @@
 // Fused Loki sparse decode step: one thread-block cluster of C CTAs per
-// (sequence, kv head). The sequence's tokens are split into C contiguous
-// ranges of whole 16-token blocks, one per CTA, and every phase stays on chip:
+// (sequence, kv head). CTA c owns the fixed token range [c * cta_tokens,
+// (c + 1) * cta_tokens) of its sequence (whole 16-token blocks), and every
+// phase stays on chip:
 //
 //  1. prologue: the key-index stream of phase 2 starts at once; meanwhile
 //     q_hat_j = q_j P[h] for the group's G query heads (AQUA page, appendix on
 //     complexity, step 1), register-blocked over (row group, column quad) of P.
 //  2. rank-r scoring (AQUA page, related work on LoKi: slice the leading
 //     dimensions after projection; Loki page, abstract: scores in the
-//     low-dimensional space). Each warp owns a private ring of bulk-copy
-//     slots (TMA engine, non-tensor form); a slot receives the leading r
-//     index dims of one 16-token block, one contiguous run of r*16 elements.
-//     Scores become order-preserving uint32 keys in shared memory; the
-//     histogram of their top 11 bits is built on the fly (one atomic per
-//     distinct bin per warp).
+//     low-dimensional space). Each warp owns a private ring of S slots; a
+//     slot receives the leading r index dims of one 16-token block, one
+//     contiguous run of r*16 elements, as 16-byte cp.async pieces from all
+//     lanes. Scores become order-preserving uint32 keys in shared memory;
+//     the histogram of their top 11 bits is built on the fly with shared
+//     atomics.
 //  3. top-k (Loki page, abstract: rank and select tokens): an exact radix
 //     select with digits of 11, 11 and 10 bits. After each digit the CTAs of
 //     the cluster sum their histograms through distributed shared memory, so
-//     every CTA finds the same boundary digit. The result is the k-th largest
-//     key tau and the number of keys equal to tau to keep; those go to the
-//     lowest token indices (ties to the lower index), CTA by CTA in rank
-//     order. The recent window (aitopics page, LRQK abstract) is appended.
-//     Kept tokens become an ascending list of local indices.
+//     every CTA finds the same boundary digit. One pass after the first digit
+//     sorts the keys into kept-for-sure and candidates; the later digits see
+//     only the candidates. The result is the k-th largest key tau and the
+//     number of keys equal to tau to keep; those go to the lowest token
+//     indices (ties to the lower index), CTA by CTA in rank order. The recent
+//     window (aitopics page, LRQK abstract) is appended. Kept tokens become
+//     an ascending list of local indices.
 //  4. exact attention over the kept tokens (AQUA page, decode-step equations
 //     (3)-(5)): each warp stages chunks of key rows and value rows into
 //     shared memory with cp.async (the next chunk in flight while the current
-//     one is consumed) and runs AttnCore on them.
+//     one is consumed) and runs MmaAttnCore (bf16, warp-level MMA) or
+//     AttnCore (fp32, CUDA cores) on them.
 //  5. the warps' partials merge per CTA into a slot of rank 0's shared
 //     memory (distributed shared memory stores); after one cluster barrier
 //     rank 0 combines the slots and writes the output.
@@ -344,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
 
     // ---- 2. rank-r scoring ----
     // A warp takes one block per iteration: its slot is read into registers and
-    // handed back to the bulk-copy engine before the arithmetic. bf16 index:
+    // refilled with the block S iterations ahead before the arithmetic. bf16 index:
     // the 16 x 16 tile of each slab (16 tokens x 16 dims) times a fragment whose
     // columns hold the score vector split into bf16 high part and remainder
     // (SUM: the summed query in columns 0, 1; MAX: q_hat_j in columns 2j, 2j+1,
