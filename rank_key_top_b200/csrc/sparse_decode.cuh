@@ -200,9 +200,10 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
 
     // ---- sequence geometry ----
     // CTA crank owns the fixed token range [crank * cta_tokens, + cta_tokens)
-    // of its sequence, so its block-table loads need not wait for the length;
-    // one wave of clusters runs at once, so the launch takes as long as the
-    // longest sequence whatever the split of the shorter ones.
+    // of its sequence, so its block-table loads need not wait for the length.
+    // In one wave of clusters the launch takes as long as the longest
+    // sequence whatever the split of the shorter ones; over several waves a
+    // CTA with a short or empty range ends early and frees its SM.
     const int cta_blocks = p.cta_tokens / kBlockTokens;
     const int blk0 = crank * cta_blocks;
     const int t0 = blk0 * kBlockTokens;
