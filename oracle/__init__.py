@@ -58,6 +58,9 @@ def _load():
                                             ctypes.c_int, ctypes.c_int, ctypes.c_int, _I32,
                                             ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                             ctypes.c_double, _D, _I32]
+        lib.oracle_magnitude_slabs.restype = ctypes.c_int
+        lib.oracle_magnitude_slabs.argtypes = [_D, _D, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_int, _I32, _D]
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
         _lib = lib
@@ -141,7 +144,7 @@ def attend_set(Kt, V, qhat, T, scale=0.0, return_weights=False):
 
 
 class PairResult:
-    __slots__ = ("out", "sel", "n_sel", "scores", "kth")
+    __slots__ = ("out", "sel", "n_sel", "scores", "kth", "slabs", "energy")
 
 
 def decode_pair(Kt, V, q, P, r, k, W=0, group_max=False, scale=0.0):
@@ -163,6 +166,39 @@ def decode_pair(Kt, V, q, P, r, k, W=0, group_max=False, scale=0.0):
         raise ValueError("oracle_decode_pair rejected its arguments")
     res.n_sel = n_sel.value
     res.kth = kth.value
+    return res
+
+
+def magnitude_slabs(q, P, r, index_dims, group_max=False):
+    """The r/16 slabs of 16 index dims with the most query energy, ascending,
+    and every slab's energy; see oracle_magnitude_slabs in oracle.c."""
+    q, P = _f64(q), _f64(P)
+    g, d = q.shape
+    slabs = np.empty(r // 16, dtype=np.int32)
+    energy = np.empty(index_dims // 16)
+    rc = _load().oracle_magnitude_slabs(_p(q), _p(P), d, g, index_dims, r, 1 if group_max else 0,
+                                        _p(slabs, _I32), _p(energy))
+    if rc != 0:
+        raise ValueError("oracle_magnitude_slabs rejected its arguments")
+    return slabs, energy
+
+
+def decode_pair_magnitude(Kt, V, q, P, r, k, index_dims, W=0, group_max=False, scale=0.0):
+    """decode_pair with the scoring dims chosen by query magnitude.
+
+    The chosen slabs' dims are moved to the front of the basis (the columns
+    of P and of the stored keys, the same permutation for both) and
+    decode_pair scores with the leading r of them: its approximate scores
+    then sum over the chosen dims in ascending order, and its exact logits,
+    over all dims, are unchanged by the permutation. The result also carries
+    `slabs` and `energy`."""
+    Kt, P = _f64(Kt), _f64(P)
+    d = P.shape[0]
+    slabs, energy = magnitude_slabs(q, P, r, index_dims, group_max)
+    front = np.concatenate([np.arange(16 * s, 16 * s + 16) for s in slabs])
+    perm = np.concatenate([front, np.setdiff1d(np.arange(d), front)])
+    res = decode_pair(Kt[:, perm], V, q, P[:, perm], r, k, W=W, group_max=group_max, scale=scale)
+    res.slabs, res.energy = slabs, energy
     return res
 
 

@@ -378,6 +378,62 @@ void oracle_covariance(const double* x, int64_t n, int d, double* C)
     free(mu);
 }
 
+/* ------------------------------------------------------------------------- */
+/* Magnitude-based choice of scoring dimensions for one (sequence, kv head)  */
+/* pair (AQUA page, Algorithm 1 in prose: per decode step, the dimensions    */
+/* whose projected-query magnitude is largest are the ones used to score;    */
+/* information-retention paragraph: what a choice keeps is the energy of     */
+/* the projected vector on it). This library's reading chooses whole slabs   */
+/* of 16 consecutive dimensions among the first index_dims:                  */
+/*   u = sum_j q_hat_j  (group SUM):   e_s = sum_{c in slab s} u[c]^2        */
+/*   group MAX:                        e_s = sum_j sum_{c in slab s} q_hat_j[c]^2 */
+/* and keeps the r/16 slabs of largest e_s, ties to the lower slab, listed   */
+/* in ascending order.                                                       */
+/*                                                                           */
+/* q [g][d] unrotated queries; P [d][d]; slabs [r/16] (written, ascending);  */
+/* energy [index_dims/16] (nullable). Returns 0, or -1 on bad sizes.         */
+/* ------------------------------------------------------------------------- */
+int oracle_magnitude_slabs(const double* q, const double* P, int d, int g, int index_dims, int r,
+                           int group_max, int32_t* slabs, double* energy)
+{
+    if (d < 16 || index_dims < 16 || index_dims > d || index_dims % 16 != 0 || r < 16 || r > index_dims ||
+        r % 16 != 0 || g < 1)
+        return -1;
+    int nsl = index_dims / 16, keep = r / 16;
+    double* qhat = (double*)malloc(sizeof(double) * (size_t)g * d);
+    double* e = (double*)calloc((size_t)nsl, sizeof(double));
+    oracle_rotate(q, P, g, d, qhat);
+    for (int s = 0; s < nsl; ++s)
+        for (int c = 16 * s; c < 16 * s + 16; ++c) {
+            if (group_max) {
+                for (int j = 0; j < g; ++j)
+                    e[s] += qhat[j * d + c] * qhat[j * d + c];
+            } else {
+                double u = 0.0;
+                for (int j = 0; j < g; ++j)
+                    u += qhat[j * d + c];
+                e[s] += u * u;
+            }
+        }
+    /* slab s is kept when fewer than r/16 slabs beat it (larger energy, or */
+    /* equal energy at a lower index)                                       */
+    int n = 0;
+    for (int s = 0; s < nsl; ++s) {
+        int beaten_by = 0;
+        for (int o = 0; o < nsl; ++o)
+            if (e[o] > e[s] || (e[o] == e[s] && o < s))
+                ++beaten_by;
+        if (beaten_by < keep)
+            slabs[n++] = s;
+    }
+    if (energy)
+        for (int s = 0; s < nsl; ++s)
+            energy[s] = e[s];
+    free(e);
+    free(qhat);
+    return 0;
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

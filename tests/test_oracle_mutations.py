@@ -29,6 +29,15 @@ MUTATIONS = {
                            "acc += z[t] * V[(int64_t)t * d + c];"),
     "window not excluded": ("int ncand = L - w_eff;", "int ncand = L - w_eff + (w_eff > 0);"),
     "k off by one": ("int keff = k < ncand ? k : ncand;", "int keff = k < ncand ? k - (k > 1) : ncand;"),
+    "slab energy not squared": ("e[s] += u * u;", "e[s] += fabs(u);"),
+    "slab energy of the first head only": ("for (int j = 0; j < g; ++j)\n                    e[s] +=",
+                                           "for (int j = 0; j < 1; ++j)\n                    e[s] +="),
+    "slabs: lightest kept": ("if (e[o] > e[s] || (e[o] == e[s] && o < s))",
+                             "if (e[o] < e[s] || (e[o] == e[s] && o < s))"),
+    "slab ties to the higher index": ("if (e[o] > e[s] || (e[o] == e[s] && o < s))",
+                                      "if (e[o] > e[s] || (e[o] == e[s] && o > s))"),
+    "slab off by one dim": ("for (int c = 16 * s; c < 16 * s + 16; ++c) {",
+                            "for (int c = 16 * s + 1; c < 16 * s + 16; ++c) {"),
 }
 
 PIN_FUNCS = [
@@ -47,6 +56,11 @@ PIN_FUNCS = [
     pins.test_one_hot_values_expose_the_softmax_weights,
     pins.test_recent_window_only,
     pins.test_head_permutation_within_group,
+    pins.test_magnitude_slabs_known_answer,
+    pins.test_magnitude_slabs_follow_the_basis,
+    pins.test_magnitude_slabs_energy_is_conserved,
+    pins.test_magnitude_slabs_maximise_the_kept_energy,
+    pins.test_magnitude_slabs_reduce_and_ties,
 ] + [lambda t=t: pins.test_topk_brute_force(t) for t in range(20)] + [
     lambda n=n: pins.test_golden_fixture(n)
     for n in sorted(x for x in os.listdir(pins.GOLDEN) if x.endswith(".json"))

@@ -494,3 +494,130 @@ def test_pca_basis_eigen_equation_and_rotation_equivariance():
     P2, lam2 = oracle.pca_basis(x @ Q)
     assert np.allclose(lam2, lam, rtol=1e-10)
     assert np.allclose(np.abs(np.sum(P2 * (Q.T @ P), axis=0)), 1.0, atol=1e-9)
+
+
+# ---------------------------------------------------------------------------
+# Magnitude-based choice of scoring slabs (AQUA page, Algorithm 1 in prose;
+# information-retention paragraph: the energy of the projected vector that a
+# choice of dims keeps)
+# ---------------------------------------------------------------------------
+
+def test_magnitude_slabs_known_answer():
+    """P = I and a query constant on each slab: slab s has energy 16 a_s^2
+    (one head), so the answer follows from the a_s by hand."""
+    d = 128
+    a = np.array([0.1, 3.0, -0.2, 0.5, -2.0, 0.3, 1.0, 0.0])
+    q = np.repeat(a, 16)[None, :]
+    slabs, energy = oracle.magnitude_slabs(q, np.eye(d), 48, 128)
+    assert slabs.tolist() == [1, 4, 6]
+    np.testing.assert_allclose(energy, 16 * a ** 2, rtol=1e-15)
+    # only the first index_dims are candidates: among slabs 0..3, slabs 1 and 3
+    slabs, energy = oracle.magnitude_slabs(q, np.eye(d), 32, 64)
+    assert slabs.tolist() == [1, 3] and energy.shape == (4,)
+
+
+def test_magnitude_slabs_follow_the_basis():
+    """With a permutation matrix as P, q_hat is q with its columns moved:
+    the slab that holds the large entries after the move is chosen."""
+    d = 64
+    q = np.zeros((1, d))
+    q[0, 5] = 4.0       # moved to column 40 (slab 2)
+    q[0, 20] = -3.0     # moved to column 3 (slab 0)
+    P = np.zeros((d, d))
+    rest = iter([c for c in range(d) if c not in (40, 3)])
+    for i in range(d):
+        P[i, 40 if i == 5 else 3 if i == 20 else next(rest)] = 1.0
+    slabs, _ = oracle.magnitude_slabs(q, P, 16, 64)
+    assert slabs.tolist() == [2]
+    slabs, _ = oracle.magnitude_slabs(q, P, 32, 64)
+    assert slabs.tolist() == [0, 2]
+
+
+def test_magnitude_slabs_energy_is_conserved():
+    """With index_dims = d and an orthonormal P, the slab energies sum to the
+    squared norm of the summed query (SUM) or to the summed squared norms of
+    the heads (MAX), whatever P is (Parseval)."""
+    d, g = 128, 4
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((g, d))
+    for seed in (1, 2):
+        P = orthonormal(d, seed)
+        _, e_sum = oracle.magnitude_slabs(q, P, 16, d, group_max=False)
+        _, e_max = oracle.magnitude_slabs(q, P, 16, d, group_max=True)
+        assert math.isclose(e_sum.sum(), float(np.sum(q.sum(axis=0) ** 2)), rel_tol=1e-12)
+        assert math.isclose(e_max.sum(), float(np.sum(q ** 2)), rel_tol=1e-12)
+
+
+def test_magnitude_slabs_maximise_the_kept_energy():
+    """Brute force on small cases: the chosen set has the largest total
+    energy of all sets of r/16 slabs (with distinct energies it is the only
+    such set)."""
+    d = 128
+    rng = np.random.default_rng(9)
+    for trial in range(20):
+        g = [1, 2, 4][trial % 3]
+        q = rng.standard_normal((g, d)) * rng.uniform(0.2, 3.0, size=d)
+        P = orthonormal(d, 100 + trial)
+        for r, idx in ((16, 128), (32, 128), (48, 96), (64, 128)):
+            for gm in (False, True):
+                slabs, e = oracle.magnitude_slabs(q, P, r, idx, group_max=gm)
+                best = max(itertools.combinations(range(idx // 16), r // 16), key=lambda c: sum(e[list(c)]))
+                assert tuple(slabs.tolist()) == best
+
+
+def test_magnitude_slabs_reduce_and_ties():
+    """SUM against MAX: two heads that cancel have no summed energy, so every
+    slab ties and SUM keeps the lowest slabs, while MAX keeps the slab the
+    heads live on. Equal energies go to the lower slab."""
+    d = 64
+    q = np.zeros((2, d))
+    q[0, 48:64] = 1.0
+    q[1] = -q[0]
+    assert oracle.magnitude_slabs(q, np.eye(d), 16, 64, group_max=False)[0].tolist() == [0]
+    assert oracle.magnitude_slabs(q, np.eye(d), 16, 64, group_max=True)[0].tolist() == [3]
+    q = np.ones((1, d))
+    assert oracle.magnitude_slabs(q, np.eye(d), 32, 64)[0].tolist() == [0, 1]
+
+
+def test_magnitude_decode_scores_are_exact_on_the_query_support():
+    """A rotated query that lives on two slabs: scoring with those slabs
+    gives the full dot products, so the kept set is the top-k of q_hat K~^T
+    computed by brute force, and the approximate scores equal it."""
+    d, L, k = 128, 300, 25
+    rng = np.random.default_rng(5)
+    P = orthonormal(d, 6)
+    qhat = np.zeros((1, d))
+    qhat[0, 32:48] = rng.standard_normal(16)
+    qhat[0, 96:112] = rng.standard_normal(16)
+    q = qhat @ P.T
+    Kt = rng.standard_normal((L, d))
+    V = rng.standard_normal((L, d))
+    res = oracle.decode_pair_magnitude(Kt, V, q, P, 32, k, 128)
+    assert res.slabs.tolist() == [2, 6]
+    full = Kt @ qhat[0]
+    np.testing.assert_allclose(res.scores, full, rtol=1e-9, atol=1e-12)
+    top = sorted(np.argsort(-full, kind="stable")[:k].tolist())
+    assert res.sel[:res.n_sel].tolist() == top
+    # the leading-dims scorer sees neither slab and keeps another set
+    lead = oracle.decode_pair(Kt, V, q, P, 32, k)
+    assert lead.sel[:lead.n_sel].tolist() != top
+
+
+def test_magnitude_decode_reduces_to_leading_when_slabs_are_leading():
+    """All slabs kept (r = index_dims) or all energies equal: the chosen
+    slabs are the leading ones and the result is the leading-dims scorer's."""
+    d, L = 64, 200
+    rng = np.random.default_rng(8)
+    P = orthonormal(d, 2)
+    Kt = rng.standard_normal((L, d))
+    V = rng.standard_normal((L, d))
+    q = rng.standard_normal((2, d))
+    a = oracle.decode_pair_magnitude(Kt, V, q, P, 48, 30, 48, W=3)
+    b = oracle.decode_pair(Kt, V, q, P, 48, 30, W=3)
+    assert a.slabs.tolist() == [0, 1, 2]
+    assert a.sel.tolist() == b.sel.tolist()
+    np.testing.assert_allclose(a.out, b.out, rtol=1e-12)
+    q = np.ones((1, d)) @ np.eye(d)
+    a = oracle.decode_pair_magnitude(Kt, V, q, np.eye(d), 16, 30, 64)
+    b = oracle.decode_pair(Kt, V, q, np.eye(d), 16, 30)
+    assert a.slabs.tolist() == [0] and a.sel.tolist() == b.sel.tolist()
