@@ -445,7 +445,33 @@ def main():
     rot_ms = statistics.median(a.elapsed_time(b) for a, b in zip(r0, r1))
     ntok = sum(spec.seq_lens) * spec.num_kv_heads
     rot_bytes = ntok * spec.head_dim * 2 * 4 + ntok * spec.r * 2   # K, V read; K~, V, index written
-    del K_orig, rcache
+    del rcache
+
+    # the magnitude scorer against the leading one, on a cache whose key index
+    # holds every dim (the scorer chooses r / 16 of its d / 16 slabs per pair)
+    mcache = loki.Cache(cache.struct.num_blocks, spec.num_kv_heads, spec.head_dim, torch.bfloat16, dev,
+                        index_dims=spec.head_dim)
+    loki.loki_prefill_rotate(mcache, batch, K_orig, V_dev, P, stream=stream)
+    del K_orig
+    mout = torch.empty_like(out)
+    scorer_ms = {}
+    for name, scorer in (("magnitude", loki.LOKI_SCORER_MAGNITUDE), ("leading", loki.LOKI_SCORER_LEADING)):
+        def mag_launch(i):
+            loki.loki_decode_attention_scored(mcache, batch, qs[i % pool], P, spec.r, spec.k, mout, scorer=scorer,
+                                              recent_window=spec.recent_window, stream=stream)
+        for i in range(3):
+            mag_launch(i)
+        m0 = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
+        m1 = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
+        for i in range(10):
+            flush_l2()
+            m0[i].record(stream)
+            mag_launch(i)
+            m1[i].record(stream)
+        torch.cuda.synchronize()
+        scorer_ms[name] = statistics.median(a.elapsed_time(b) for a, b in zip(m0, m1))
+    assert loki.loki_device_error() == 0
+    del mcache
 
     if rank != 0:
         finish(world)
@@ -483,6 +509,11 @@ def main():
                            "achieved_gbs": rot_bytes / (rot_ms / 1e3) / 1e9,
                            "tflops": 2.0 * ntok * spec.head_dim ** 2 / (rot_ms / 1e3) / 1e12,
                            "kernel": "rotate_prefill_tc_kernel<128> (tcgen05)"},
+        "magnitude_scorer": {"launch_ms": scorer_ms["magnitude"], "leading_launch_ms": scorer_ms["leading"],
+                             "index_dims": spec.head_dim,
+                             "note": "loki_decode_attention_scored on a cache whose key index holds all "
+                                     f"{spec.head_dim} dims; r = {spec.r}: the r/16 slabs with the most query "
+                                     "energy against the leading r dims, median of 10 L2-flushed launches"},
         "dense": {"ms_per_step": dense_ms, "steps_per_s": 1e3 / dense_ms,
                   "achieved_gbs": dense_bytes(spec) / (dense_ms / 1e3) / 1e9},
         "wall_s_timed_loop": wall,

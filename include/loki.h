@@ -46,7 +46,7 @@ extern "C" {
 #define LOKI_API
 #endif
 
-#define LOKI_ABI_VERSION 2
+#define LOKI_ABI_VERSION 3
 #define LOKI_BLOCK_TOKENS 16 /* tokens per paged-cache block */
 
 typedef void* loki_stream_t; /* a cudaStream_t */
@@ -73,6 +73,20 @@ typedef enum loki_group_reduce {
     LOKI_GROUP_SUM = 0,
     LOKI_GROUP_MAX = 1
 } loki_group_reduce;
+
+/* Which r index dims the approximate score uses (loki_decode_attention_scored).
+ * LEADING: the leading r dims, a static slice after the projection (Loki page,
+ * abstract; AQUA page, related work on LoKi). MAGNITUDE: per (sequence, kv
+ * head) and step, the r/16 slabs of 16 index dims with the most energy of the
+ * query that ranks the tokens (AQUA page, Algorithm 1 in prose: dims picked by
+ * the magnitude of the projected query; the energy kept is what the AQUA
+ * page's information-retention loss measures). The pages pick single dims;
+ * this library picks whole 16-dim slabs so that each block's selected dims
+ * remain contiguous runs of the key index. */
+typedef enum loki_scorer {
+    LOKI_SCORER_LEADING = 0,
+    LOKI_SCORER_MAGNITUDE = 1
+} loki_scorer;
 
 /* Device error word bits (loki_device_error). */
 #define LOKI_DEVERR_SEQ_LEN 0x1u  /* a seq_lens entry outside [0, max_seq_len] */
@@ -236,6 +250,24 @@ LOKI_API loki_status loki_decode_attention(const loki_cache* cache, const loki_b
                                   float scale, float* out, int32_t* selected_idx,
                                   void* workspace, size_t workspace_bytes,
                                   loki_stream_t stream);
+
+/* loki_decode_attention with a choice of scorer; LOKI_SCORER_LEADING gives
+ * the same results as loki_decode_attention. With LOKI_SCORER_MAGNITUDE,
+ * step 2 scores with the selected slabs instead of the leading r dims:
+ *   energy e_s = sum_{c in slab s} u[c]^2 for each slab s < index_dims/16,
+ *     u = sum_{j in group(h)} q_hat_j (SUM), or
+ *     e_s = sum_{j in group(h)} sum_{c in slab s} q_hat_j[c]^2 (MAX)   (fp32);
+ *   the r/16 slabs of largest e_s (ties to the lower slab) form the set S and
+ *   s_t = reduce_j sum_{s in S, ascending} q_hat_j[slab s] . K~[t, slab s].
+ * Steps 1, 3 and 4 are unchanged. Arguments as for loki_decode_attention;
+ * an unknown scorer is LOKI_ERR_INVALID_ARG. */
+LOKI_API loki_status loki_decode_attention_scored(const loki_cache* cache, const loki_batch* batch,
+                                         const void* q, int32_t num_q_heads, const float* P,
+                                         int32_t r, int32_t k, const int32_t* k_per_seq,
+                                         int32_t recent_window, loki_group_reduce group_reduce,
+                                         float scale, loki_scorer scorer, float* out,
+                                         int32_t* selected_idx, void* workspace,
+                                         size_t workspace_bytes, loki_stream_t stream);
 
 /* One whole decode step: loki_append_keys(k_new, v_new, P) followed by
  * loki_decode_attention(...) on the same stream, with the same arguments and

@@ -141,7 +141,7 @@ loki_status check_decode(const loki_cache* cache, const loki_batch* batch, const
 loki_status launch_decode(const loki_cache* cache, const loki_batch* batch, const void* q, int32_t num_q_heads,
                           const float* P, int32_t r, int32_t k, const int32_t* k_per_seq, int32_t recent_window,
                           loki_group_reduce group_reduce, float scale, float* out, int32_t* selected_idx,
-                          cudaStream_t s, bool programmatic) {
+                          cudaStream_t s, bool programmatic, bool magnitude = false) {
     const int Hkv = cache->num_kv_heads, D = cache->head_dim;
     const int G = num_q_heads / Hkv;
     const int pairs = batch->batch * Hkv;
@@ -168,7 +168,8 @@ loki_status launch_decode(const loki_cache* cache, const loki_batch* batch, cons
     p.group_max = group_reduce == LOKI_GROUP_MAX ? 1 : 0;
     const double sc = scale == 0.f ? 1.0 / std::sqrt((double)D) : (double)scale;
     p.scale_log2 = (float)(sc * kLog2e);
-    return dispatch_tdg<SparseLaunch>(cache->dtype, D, G, p, pairs, (int)batch->max_seq_len, di, s, programmatic);
+    return dispatch_tdg<SparseLaunch>(cache->dtype, D, G, p, pairs, (int)batch->max_seq_len, di, s, programmatic,
+                                      magnitude);
 }
 
 }  // namespace
@@ -384,6 +385,23 @@ loki_status loki_decode_attention(const loki_cache* cache, const loki_batch* bat
     if (st != LOKI_OK || batch->batch == 0) return st;
     return launch_decode(cache, batch, q, num_q_heads, P, r, k, k_per_seq, recent_window, group_reduce, scale, out,
                          selected_idx, reinterpret_cast<cudaStream_t>(stream), false);
+}
+
+loki_status loki_decode_attention_scored(const loki_cache* cache, const loki_batch* batch, const void* q,
+                                         int32_t num_q_heads, const float* P, int32_t r, int32_t k,
+                                         const int32_t* k_per_seq, int32_t recent_window,
+                                         loki_group_reduce group_reduce, float scale, loki_scorer scorer,
+                                         float* out, int32_t* selected_idx, void* workspace,
+                                         size_t workspace_bytes, loki_stream_t stream) {
+    (void)workspace;
+    (void)workspace_bytes;
+    if (scorer != LOKI_SCORER_LEADING && scorer != LOKI_SCORER_MAGNITUDE) return LOKI_ERR_INVALID_ARG;
+    const loki_status st = check_decode(cache, batch, q, num_q_heads, P, r, k, recent_window, group_reduce, scale,
+                                        out);
+    if (st != LOKI_OK || batch->batch == 0) return st;
+    return launch_decode(cache, batch, q, num_q_heads, P, r, k, k_per_seq, recent_window, group_reduce, scale, out,
+                         selected_idx, reinterpret_cast<cudaStream_t>(stream), false,
+                         scorer == LOKI_SCORER_MAGNITUDE);
 }
 
 loki_status loki_decode_step(const loki_cache* cache, const loki_batch* batch, const void* k_new, const void* v_new,

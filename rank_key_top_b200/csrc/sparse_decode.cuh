@@ -164,7 +164,13 @@ __device__ __noinline__ int2 radix_boundary(const uint32_t* hcur, int nbins, int
     return make_int2(misc[0], misc[1]);
 }
 
-template <typename T, int D, int G>
+// MAG selects the scorer. false: the leading r index dims (Loki). true: the
+// r / 16 index slabs (16 dims each) that hold the most energy of the group's
+// rotated query (AQUA page, Algorithm 1 in prose: the dims are picked by the
+// magnitude of q_hat per decode step; the retained energy is what its
+// information-retention loss measures). Here a slab is the unit of choice, so
+// that a block's selected dims stay whole 512-byte (bf16) runs of the index.
+template <typename T, int D, int G, bool MAG>
 __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const SparseParams p) {
     using Geom = SparseGeom<T, D, G>;
     using Core = typename Geom::Core;
@@ -196,7 +202,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     float* part = reinterpret_cast<float*>(smem + p.off_part);
     int32_t* misc = reinterpret_cast<int32_t*>(smem + p.off_misc);
     // misc: [0] boundary digit, [1] count above it, [8..39] suffix-sum scratch,
-    //       [40..55] warp kept counts, [56..71] warp equal counts, [72] list length
+    //       [40..55] warp kept counts, [56..71] warp equal counts, [72] list length,
+    //       [96..103] selected index slabs, [104..111] slab energies (MAG)
 
     // ---- sequence geometry ----
     // CTA crank owns the fixed token range [crank * cta_tokens, + cta_tokens)
@@ -290,7 +297,15 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
             const int pb = entry(it);
             const unsigned char* src = xbytes + page_offset(pb, h, p.Hkv, p.index_dims) * (int64_t)sizeof(T);
             unsigned char* dst = wring + (it & smask) * p.slot_bytes;
-            for (int o = lane * 16; o < p.slot_bytes; o += 32 * 16) cp_async16(dst + o, src + o, true);
+            if constexpr (MAG) {  // slot slab i <- index slab misc[96 + i] of the page
+                constexpr int SLAB = kBlockTokens * kSlabDims * (int)sizeof(T);
+                for (int o = lane * 16; o < p.slot_bytes; o += 32 * 16) {
+                    const int i = o / SLAB;
+                    cp_async16(dst + o, src + misc[96 + i] * SLAB + (o - i * SLAB), true);
+                }
+            } else {
+                for (int o = lane * 16; o < p.slot_bytes; o += 32 * 16) cp_async16(dst + o, src + o, true);
+            }
         }
         cp_async_commit();
         for (int i = 0; i < pad; ++i) cp_async_commit();
@@ -301,8 +316,11 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     // first read by the gather; without one the key index may hold it.
     // (The scoring copies whole 16-token blocks: bytes of a token that is not
     // a candidate may be read while being written; they are never used.)
-    if (p.W == 0) griddep_wait();
-    for (int it = 0; it < S; ++it) refill(it);
+    // (the magnitude scorer knows which slabs to fetch only after q_hat)
+    if constexpr (!MAG) {
+        if (p.W == 0) griddep_wait();
+        for (int it = 0; it < S; ++it) refill(it);
+    }
     for (int i = tid; i < 2 * kHistBins; i += kThreads) hist[i] = 0;
     if (j0 < nblk_loc) tbl[j0] = tb0;
     if (j1 < nblk_loc) tbl[j1] = tb1;
@@ -338,13 +356,43 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
         }
         __syncthreads();
         if (!p.group_max) {
-            for (int c = tid; c < p.r; c += kThreads) {
+            for (int c = tid; c < (MAG ? p.index_dims : p.r); c += kThreads) {
                 float s = 0.f;
                 for (int j = 0; j < G; ++j) s += qhat[j * D + c];
                 qs[c] = s;
             }
         }
         __syncthreads();
+        if constexpr (MAG) {
+            // slab energy: squared norm of the summed query over the slab (SUM),
+            // or summed over the group's heads (MAX); the r / 16 largest, ties
+            // to the lower slab, listed in ascending slab order
+            const int nsl = p.index_dims / kSlabDims, R16 = p.r / kSlabDims;
+            float* en = reinterpret_cast<float*>(misc + 104);
+            if (tid < nsl) {
+                float w = 0.f;
+                for (int c = tid * kSlabDims; c < (tid + 1) * kSlabDims; ++c) {
+                    if (!p.group_max) {
+                        w = fmaf(qs[c], qs[c], w);
+                    } else {
+                        for (int j = 0; j < G; ++j) w = fmaf(qhat[j * D + c], qhat[j * D + c], w);
+                    }
+                }
+                en[tid] = w;
+            }
+            __syncthreads();
+            if (tid == 0) {
+                int n = 0;
+                for (int sl = 0; sl < nsl; ++sl) {
+                    int rank = 0;
+                    for (int o = 0; o < nsl; ++o) rank += en[o] > en[sl] || (en[o] == en[sl] && o < sl);
+                    if (rank < R16) misc[96 + n++] = sl;
+                }
+            }
+            __syncthreads();
+            if (p.W == 0) griddep_wait();
+            for (int it = 0; it < S; ++it) refill(it);
+        }
     }
 
     // ---- 2. rank-r scoring ----
@@ -374,9 +422,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
                     float v[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int d = sb * 16 + 2 * t + (e & 1) + (e >> 1) * 8;
                         float x = 0.f;
                         if (sb < R16) {
+                            const int d = (MAG ? misc[96 + sb] : sb) * 16 + 2 * t + (e & 1) + (e >> 1) * 8;
                             if (!p.group_max) {
                                 x = (ng == 0 && g < 2) ? split_part(qs[d], g & 1) : 0.f;
                             } else {
@@ -456,8 +504,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
                         if (sb >= R16) break;
                         float kf[8];
                         V8::to_float(raw[sb], kf);
-                        const float4 q0 = *reinterpret_cast<const float4*>(qs + sb * 16 + half * 8);
-                        const float4 q1 = *reinterpret_cast<const float4*>(qs + sb * 16 + half * 8 + 4);
+                        const int d0 = (MAG ? misc[96 + sb] : sb) * 16 + half * 8;
+                        const float4 q0 = *reinterpret_cast<const float4*>(qs + d0);
+                        const float4 q1 = *reinterpret_cast<const float4*>(qs + d0 + 4);
                         a = fmaf(q0.x, kf[0], a);
                         a = fmaf(q0.y, kf[1], a);
                         a = fmaf(q0.z, kf[2], a);
@@ -479,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
                         V8::to_float(raw[sb], kf);
 #pragma unroll
                         for (int j = 0; j < G; ++j) {
-                            const float* qq = qhat + j * D + sb * 16 + half * 8;
+                            const float* qq = qhat + j * D + (MAG ? misc[96 + sb] : sb) * 16 + half * 8;
 #pragma unroll
                             for (int i = 0; i < 8; ++i) ag[j] = fmaf(qq[i], kf[i], ag[j]);
                         }

@@ -23,6 +23,8 @@ LOKI_F32 = 0
 LOKI_BF16 = 1
 LOKI_GROUP_SUM = 0
 LOKI_GROUP_MAX = 1
+LOKI_SCORER_LEADING = 0
+LOKI_SCORER_MAGNITUDE = 1
 
 LOKI_DEVERR_SEQ_LEN = 0x1
 LOKI_DEVERR_BLOCK_ID = 0x2
@@ -66,6 +68,9 @@ _SIGS = {
     "loki_decode_workspace_bytes": (_SZ, [_C, _B, _I32, _I32, _I32]),
     "loki_decode_attention": (ctypes.c_int, [_C, _B, _P, _I32, _P, _I32, _I32, _P, _I32,
                                              ctypes.c_int, ctypes.c_float, _P, _P, _P, _SZ, _P]),
+    "loki_decode_attention_scored": (ctypes.c_int, [_C, _B, _P, _I32, _P, _I32, _I32, _P, _I32,
+                                                    ctypes.c_int, ctypes.c_float, ctypes.c_int, _P, _P,
+                                                    _P, _SZ, _P]),
     "loki_decode_step": (ctypes.c_int, [_C, _B, _P, _P, _P, _I32, _P, _I32, _I32, _P, _I32,
                                         ctypes.c_int, ctypes.c_float, _P, _P, _P, _SZ, _P]),
     "loki_decode_max_seq_len": (_I32, [_I32, ctypes.c_int]),
@@ -202,6 +207,16 @@ def loki_decode_attention(cache, batch, q, P, r, k, out, k_per_seq=None, recent_
     _check("loki_decode_attention", _lib.loki_decode_attention(
         ctypes.byref(cache.struct), ctypes.byref(batch.struct), _ptr(q), q.shape[1], _ptr(P), r, k,
         _ptr(k_per_seq), recent_window, group_reduce, scale, _ptr(out), _ptr(selected_idx),
+        _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def loki_decode_attention_scored(cache, batch, q, P, r, k, out, scorer=LOKI_SCORER_LEADING, k_per_seq=None,
+                                 recent_window=0, group_reduce=LOKI_GROUP_SUM, scale=0.0, selected_idx=None,
+                                 workspace=None, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("loki_decode_attention_scored", _lib.loki_decode_attention_scored(
+        ctypes.byref(cache.struct), ctypes.byref(batch.struct), _ptr(q), q.shape[1], _ptr(P), r, k,
+        _ptr(k_per_seq), recent_window, group_reduce, scale, scorer, _ptr(out), _ptr(selected_idx),
         _ptr(workspace), ws_bytes, _stream(stream)))
 
 

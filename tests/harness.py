@@ -10,6 +10,7 @@ from rank_key_top_b200 import synth
 BF16_RTOL = 2e-3   # max normwise relative error of outputs, bf16 caches
 F32_RTOL = 1e-5    # the same for fp32 caches
 TIE_BAND = 1e-3    # selected sets may differ only where |s_t - s_(k)| <= TIE_BAND |s_(k)|
+SLAB_MARGIN = 1e-3  # magnitude scorer: the last kept slab must beat the first dropped one by this much
 
 
 def tol_for(spec):
@@ -24,6 +25,7 @@ class Device:
         self.wl, self.loki = wl, loki
         if index_dims is None:
             index_dims = max(s.r, min(64, s.head_dim))
+        self.index_dims = index_dims
         self.cache = loki.Cache(wl.num_blocks, s.num_kv_heads, s.head_dim, synth.torch_dtype(s.dtype), device,
                                 index_dims=index_dims)
         self.batch = loki.Batch(wl.block_table.to(device), wl.seq_lens.to(device),
@@ -34,7 +36,7 @@ class Device:
         if s.max_seq_len > 0:
             loki.loki_prefill_cache(self.cache, self.batch, wl.Kt.to(device), wl.V.to(device))
 
-    def decode(self, r=None, k=None, W=None, group_max=False, q=None, scale=0.0):
+    def decode(self, r=None, k=None, W=None, group_max=False, q=None, scale=0.0, scorer=None):
         s, loki = self.wl.spec, self.loki
         r = s.r if r is None else r
         k = s.k if k is None else k
@@ -42,10 +44,15 @@ class Device:
         q = self.q if q is None else q
         out = torch.full((s.batch, s.num_q_heads, s.head_dim), float("nan"), device=q.device)
         sel = torch.full((s.batch, s.num_kv_heads, k + W), -7, dtype=torch.int32, device=q.device)
-        loki.loki_decode_attention(self.cache, self.batch, q, self.P, r, k, out,
-                                   k_per_seq=self.k_per_seq, recent_window=W,
-                                   group_reduce=loki.LOKI_GROUP_MAX if group_max else loki.LOKI_GROUP_SUM,
-                                   scale=scale, selected_idx=sel)
+        reduce = loki.LOKI_GROUP_MAX if group_max else loki.LOKI_GROUP_SUM
+        if scorer is None:
+            loki.loki_decode_attention(self.cache, self.batch, q, self.P, r, k, out,
+                                       k_per_seq=self.k_per_seq, recent_window=W, group_reduce=reduce,
+                                       scale=scale, selected_idx=sel)
+        else:
+            loki.loki_decode_attention_scored(self.cache, self.batch, q, self.P, r, k, out, scorer=scorer,
+                                              k_per_seq=self.k_per_seq, recent_window=W,
+                                              group_reduce=reduce, scale=scale, selected_idx=sel)
         torch.cuda.synchronize()
         return out.cpu(), sel.cpu()
 
@@ -71,16 +78,28 @@ def pair_inputs(wl, b, h, q=None):
 
 
 def check_pair(wl, b, h, out_gpu, sel_gpu, r, k, W, group_max=False, scale=0.0, q=None, rtol=None,
-               inputs=None):
+               inputs=None, magnitude_dims=None):
     """Set parity (with the tie band) and output parity for one pair.
 
+    magnitude_dims: the key index's width when the magnitude scorer ran (the
+    oracle then chooses the scoring slabs the same way, and the input must
+    separate the last kept slab from the first dropped one by SLAB_MARGIN, so
+    that both sides' choice is the same whatever their precision).
     Returns (output error on the GPU's set, output error on the oracle's set)."""
     s = wl.spec
     g = s.group
     L = s.seq_lens[b]
     kb = int(wl.k_per_seq[b]) if wl.k_per_seq is not None else k
     Kt, V, qq, P = inputs if inputs is not None else pair_inputs(wl, b, h, q)
-    res = oracle.decode_pair(Kt, V, qq, P, r=r, k=kb, W=W, group_max=group_max, scale=scale)
+    if magnitude_dims is None:
+        res = oracle.decode_pair(Kt, V, qq, P, r=r, k=kb, W=W, group_max=group_max, scale=scale)
+    else:
+        res = oracle.decode_pair_magnitude(Kt, V, qq, P, r, kb, magnitude_dims, W=W, group_max=group_max,
+                                           scale=scale)
+        e = np.sort(res.energy)[::-1]
+        if r // 16 < e.size:
+            assert e[r // 16 - 1] - e[r // 16] > SLAB_MARGIN * e[r // 16 - 1], (
+                f"pair {(b, h)}: input without a slab-selection margin")
     width = k + W
     row = sel_gpu[b, h].numpy()
     n = res.n_sel

@@ -36,7 +36,7 @@ def test_library_exports_every_declared_symbol(loki):
     for name in declared_symbols():
         assert hasattr(lib, name), name
     assert sorted(loki.EXPORTED) == declared_symbols()
-    assert loki.loki_abi_version() == 2
+    assert loki.loki_abi_version() == 3
 
 
 def test_status_strings(loki):
@@ -142,12 +142,32 @@ def test_decode_step_rejects(loki, kw, status):
     assert step(loki, c, b, **kw) == status
 
 
+def scored(loki, c, b, scorer, Hq=32, r=32, k=8, W=0, q=FAKE, P=FAKE, out=FAKE):
+    return loki.raw().loki_decode_attention_scored(ctypes.byref(c), ctypes.byref(b), q, Hq, P, r, k, None, W,
+                                                   0, 0.0, scorer, out, None, None, 0, None)
+
+
+@pytest.mark.parametrize("scorer,kw,status", [
+    (2, {}, 1),                     # unknown scorer
+    (-1, {}, 1),
+    (1, dict(r=48), 1),             # r above index_dims (32), for either scorer
+    (0, dict(r=48), 1),
+    (1, dict(k=0, W=0), 1),
+    (1, dict(Hq=24), 2),
+    (1, dict(out=None), 1),
+])
+def test_decode_scored_rejects(loki, scorer, kw, status):
+    c, b = structs(loki)
+    assert scored(loki, c, b, scorer, **kw) == status
+
+
 def test_empty_batch_is_a_no_op(loki):
     c, b = structs(loki, B=0)
     assert decode(loki, c, b, q=None, P=None, out=None) == 0
     assert loki.raw().loki_append_keys(ctypes.byref(c), ctypes.byref(b), None, None, None, None) == 0
     assert loki.raw().loki_prefill_cache(ctypes.byref(c), ctypes.byref(b), None, None, 0, None) == 0
     assert step(loki, c, b, k_new=None, v_new=None, q=None, P=None, out=None) == 0
+    assert scored(loki, c, b, 1, q=None, P=None, out=None) == 0
 
 
 def test_append_and_prefill_reject(loki):

@@ -553,3 +553,78 @@ def test_long_context_outliers_sweep(cuda_lib):
             inputs = harness.pair_inputs(wl, b, h)
             for (r, k), (out, sel) in results.items():
                 harness.check_pair(wl, b, h, out, sel, r, k, 0, inputs=inputs)
+
+
+# ---------------------------------------------------------------------------
+# Magnitude scorer: the scoring slabs chosen by query energy
+# ---------------------------------------------------------------------------
+
+def magnitude_queries(wl, group_max, seed):
+    """Queries whose rotated slabs carry the energies 1.3^(2i), i = 0 .. d/16 - 1,
+    in a shuffled order per (sequence, kv head): the energy the chosen reduce
+    measures (of the summed query for SUM, summed over heads for MAX) is set
+    exactly, so the choice of slabs has a wide margin. q = q_hat P^T."""
+    s = wl.spec
+    g, d = s.group, s.head_dim
+    gen = torch.Generator().manual_seed(seed)
+    q = torch.empty(s.batch, s.num_q_heads, d, dtype=torch.float64)
+    for b in range(s.batch):
+        for h in range(s.num_kv_heads):
+            qhat = torch.randn(g, d, generator=gen, dtype=torch.float64)
+            mags = 1.3 ** torch.randperm(d // 16, generator=gen).double()
+            for sl in range(d // 16):
+                blk = qhat[:, 16 * sl:16 * sl + 16]
+                norm = blk.pow(2).sum().sqrt() if group_max else blk.sum(0).pow(2).sum().sqrt()
+                qhat[:, 16 * sl:16 * sl + 16] = blk * (mags[sl] / norm)
+            q[b, h * g:(h + 1) * g] = qhat @ wl.P[h].double().T
+    return q.to(wl.q.dtype)
+
+
+@pytest.mark.parametrize("dtype,D,Hq,Hkv,index_dims,r,group_max,lens", [
+    ("bf16", 128, 8, 2, 128, 32, False, [20000, 3000, 777, 33]),
+    ("bf16", 128, 16, 2, 64, 16, True, [3000, 777]),
+    ("bf16", 64, 2, 1, 64, 48, False, [3000, 1]),
+    ("f32", 128, 4, 1, 128, 64, True, [3000, 0, 500]),
+    ("f32", 64, 4, 4, 64, 16, False, [2500, 777]),
+])
+def test_magnitude_scorer_matches_oracle(cuda_lib, dtype, D, Hq, Hkv, index_dims, r, group_max, lens):
+    """Set and output parity with the oracle, which chooses the slabs from
+    the same queries; at least one pair must choose slabs other than the
+    leading ones, or the case would not test the choice."""
+    s = spec(dtype=dtype, head_dim=D, num_q_heads=Hq, num_kv_heads=Hkv, seq_lens=lens, r=r, k=150,
+             recent_window=5)
+    wl = synth.make_workload(s)
+    wl.q = magnitude_queries(wl, group_max, seed=21)
+    dev = harness.Device(wl, cuda_lib, index_dims=index_dims)
+    out, sel = dev.decode(group_max=group_max, scorer=cuda_lib.LOKI_SCORER_MAGNITUDE)
+    assert cuda_lib.loki_device_error() == 0
+    moved = 0
+    for b in range(s.batch):
+        for h in range(s.num_kv_heads):
+            harness.check_pair(wl, b, h, out, sel, r, s.k, s.recent_window, group_max=group_max,
+                               magnitude_dims=index_dims)
+            qq, P = harness.pair_inputs(wl, b, h)[2:]
+            slabs, _ = oracle.magnitude_slabs(qq, P, r, index_dims, group_max)
+            moved += slabs.tolist() != list(range(r // 16))
+    assert moved > 0
+
+
+def test_scored_entry_with_leading_scorer_is_decode_attention(cuda_lib):
+    s = spec(num_q_heads=8, num_kv_heads=2, seq_lens=[5000, 123], k=200, recent_window=4)
+    wl = synth.make_workload(s)
+    dev = harness.Device(wl, cuda_lib)
+    a = dev.decode()
+    b = dev.decode(scorer=cuda_lib.LOKI_SCORER_LEADING)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("group_max", [False, True])
+def test_magnitude_scorer_with_every_slab_is_leading(cuda_lib, group_max):
+    """r = index_dims: every slab is chosen, in ascending order, so the
+    magnitude scorer computes what the leading scorer does, bit for bit."""
+    s = spec(num_q_heads=4, num_kv_heads=1, seq_lens=[4000, 900], r=64, k=100, recent_window=2)
+    wl = synth.make_workload(s)
+    dev = harness.Device(wl, cuda_lib, index_dims=64)
+    a = dev.decode(group_max=group_max)
+    b = dev.decode(group_max=group_max, scorer=cuda_lib.LOKI_SCORER_MAGNITUDE)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
