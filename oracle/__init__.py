@@ -58,6 +58,13 @@ def _load():
                                             ctypes.c_int, ctypes.c_int, ctypes.c_int, _I32,
                                             ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                             ctypes.c_double, _D, _I32]
+        lib.oracle_index_keys.restype = None
+        lib.oracle_index_keys.argtypes = [_D, _D, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, _D]
+        lib.oracle_decode_pair_asym.restype = ctypes.c_int
+        lib.oracle_decode_pair_asym.argtypes = [_D, _D, _D, _D, _D, _D, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_int, ctypes.c_int, ctypes.c_double, _D, _I32,
+                                                ctypes.POINTER(ctypes.c_int), _D, _D]
         lib.oracle_magnitude_slabs.restype = ctypes.c_int
         lib.oracle_magnitude_slabs.argtypes = [_D, _D, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                ctypes.c_int, ctypes.c_int, _I32, _D]
@@ -200,6 +207,77 @@ def decode_pair_magnitude(Kt, V, q, P, r, k, index_dims, W=0, group_max=False, s
     res = decode_pair(Kt[:, perm], V, q, P[:, perm], r, k, W=W, group_max=group_max, scale=scale)
     res.slabs, res.energy = slabs, energy
     return res
+
+
+def index_keys(k, Ak, dtype):
+    """Key-index rows round(k A_k) of keys k [n, d] in the original basis,
+    A_k [d, ri]; see oracle_index_keys in oracle.c. dtype: 'bf16' or 'f32'."""
+    k, Ak = _f64(k), _f64(Ak)
+    n, d = k.shape
+    ri = Ak.shape[1]
+    out = np.empty((n, ri))
+    _load().oracle_index_keys(_p(k), _p(Ak), n, d, ri, 1 if dtype == "bf16" else 0, _p(out))
+    return out
+
+
+def decode_pair_asym(Kt, V, Kidx, q, P, Aq, r, k, W=0, group_max=False, scale=0.0):
+    """One pair's decode with scores from the key index Kidx [L, ri] and the
+    query factor q A_q; see oracle_decode_pair_asym in oracle.c."""
+    Kt, V, Kidx, q, P, Aq = _f64(Kt), _f64(V), _f64(Kidx), _f64(q), _f64(P), _f64(Aq)
+    L, d = Kt.shape
+    ri = Aq.shape[1]
+    g = q.shape[0]
+    res = PairResult()
+    res.out = np.empty((g, d))
+    res.sel = np.empty(k + W, dtype=np.int32)
+    n_sel = ctypes.c_int(0)
+    res.scores = np.empty(L)
+    kth = ctypes.c_double(0.0)
+    rc = _load().oracle_decode_pair_asym(_p(Kt), _p(V), _p(Kidx), _p(q), _p(P), _p(Aq), L, d, ri, g, r, k, W,
+                                         1 if group_max else 0, scale, _p(res.out), _p(res.sel, _I32),
+                                         ctypes.byref(n_sel), _p(res.scores), ctypes.byref(kth))
+    if rc != 0:
+        raise ValueError("oracle_decode_pair_asym rejected its arguments")
+    res.n_sel = n_sel.value
+    res.kth = kth.value
+    return res
+
+
+def _sym_power(S, power):
+    lam, vec = np.linalg.eigh(S)
+    if lam.min() <= 0:
+        raise ValueError("second-moment matrix is not positive definite")
+    return (vec * lam ** power) @ vec.T
+
+
+def saki_factors(Q, K, r):
+    """Rank-r asymmetric score factors from calibration queries Q [n_q, d] and
+    keys K [n_k, d] (SAKI page, abstract: the expected score distortion of a
+    rank-r approximation q W k^T of q k^T is a covariance-weighted low-rank
+    objective, solved in closed form by the SVD of the covariance-weighted
+    query-key operator).
+
+    Reading: with the second moments S_q = Q^T Q / n_q and S_k = K^T K / n_k
+    (uncentred: the score is a raw inner product), the distortion of W is
+    E[(q (I - W) k^T)^2] = ||S_q^1/2 (I - W) S_k^1/2||_F^2, minimised over
+    rank r by S_q^1/2 W S_k^1/2 = the rank-r SVD truncation U_r s_r V_r^T of
+    C = S_q^1/2 S_k^1/2 (Eckart-Young). Factored as W = A_q A_k^T with
+    A_q = S_q^-1/2 U_r diag(s_r)^1/2 and A_k = S_k^-1/2 V_r diag(s_r)^1/2;
+    the first r' < r columns of the factors are the rank-r' solution.
+    The abstract's random-matrix noise correction is not part of this
+    reading (the abstract stops before saying how it is done).
+
+    numpy's symmetric eigensolver (matrix square roots) and SVD are the
+    library steps. Returns (A_q [d, r], A_k [d, r], all singular values of C)."""
+    Q, K = _f64(Q), _f64(K)
+    Sq = Q.T @ Q / Q.shape[0]
+    Sk = K.T @ K / K.shape[0]
+    C = _sym_power(Sq, 0.5) @ _sym_power(Sk, 0.5)
+    U, s, Vt = np.linalg.svd(C)
+    root = np.sqrt(s[:r])
+    Aq = _sym_power(Sq, -0.5) @ (U[:, :r] * root)
+    Ak = _sym_power(Sk, -0.5) @ (Vt[:r].T * root)
+    return Aq, Ak, s
 
 
 def dense_pair(K, V, q, P=None, scale=0.0):

@@ -189,6 +189,25 @@ static int by_index(const void* pa, const void* pb)
     return (a > b) - (a < b);
 }
 
+/* Step 4 of a decode: keep the k best of the ncand candidates, ties to the  */
+/* lower index, in ascending order, then add the recent window (LRQK: top-k  */
+/* tokens plus a fixed set of recent ones). cand is sorted in place; T has   */
+/* room for ncand + w_eff entries. Returns the number kept; *kth (nullable)  */
+/* gets the score of the last token kept by score, NaN if none.              */
+static int keep_top_k_and_window(scored_token* cand, int ncand, int k, int w_eff, int32_t* T, double* kth)
+{
+    int keff = k < ncand ? k : ncand;
+    qsort(cand, (size_t)ncand, sizeof(scored_token), by_score_then_index);
+    if (kth)
+        *kth = keff > 0 ? cand[keff - 1].s : NAN;
+    for (int i = 0; i < keff; ++i)
+        T[i] = cand[i].t;
+    qsort(T, (size_t)keff, sizeof(int32_t), by_index);
+    for (int i = 0; i < w_eff; ++i)
+        T[keff + i] = ncand + i;
+    return keff + w_eff;
+}
+
 /* ------------------------------------------------------------------------- */
 /* One decode step of Loki-style sparse attention for one (sequence, kv      */
 /* head) pair and its g query heads.                                         */
@@ -251,19 +270,9 @@ int oracle_decode_pair(const double* Kt, const double* V, const double* q, const
             scores[t] = cand[t].s;
     }
 
-    /* Step 4: keep the k best candidates, ties to the lower index, and add   */
-    /* the recent window (LRQK: top-k tokens plus a fixed set of recent ones). */
-    int keff = k < ncand ? k : ncand;
-    qsort(cand, (size_t)ncand, sizeof(scored_token), by_score_then_index);
-    if (kth)
-        *kth = keff > 0 ? cand[keff - 1].s : NAN;
-    int nT = keff + w_eff;
-    int32_t* T = (int32_t*)malloc(sizeof(int32_t) * (size_t)(nT > 0 ? nT : 1));
-    for (int i = 0; i < keff; ++i)
-        T[i] = cand[i].t;
-    qsort(T, (size_t)keff, sizeof(int32_t), by_index);
-    for (int i = 0; i < w_eff; ++i)
-        T[keff + i] = ncand + i;
+    /* Step 4: keep the k best candidates and the recent window.             */
+    int32_t* T = (int32_t*)malloc(sizeof(int32_t) * (size_t)(ncand + w_eff + 1));
+    int nT = keep_top_k_and_window(cand, ncand, k, w_eff, T, kth);
 
     /* Step 5: exact softmax attention over the kept set (equations (3)-(5)). */
     oracle_attend_set(Kt, V, qhat, T, nT, d, g, scale, out, NULL);
@@ -276,6 +285,106 @@ int oracle_decode_pair(const double* Kt, const double* V, const double* q, const
         *n_sel = nT;
     free(T);
     free(cand);
+    free(qhat);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Key index of an asymmetric score factorisation (SAKI page, abstract: a    */
+/* rank-r factorisation of the query-key score operator with its own key     */
+/* factor): idx = round(k A_k) to the cache type, row vectors.               */
+/* k [n][d]; Ak [d][ri] row-major; out [n][ri]. dtype 1 = bf16, 0 = binary32. */
+/* ------------------------------------------------------------------------- */
+void oracle_index_keys(const double* k, const double* Ak, int64_t n, int d, int ri, int dtype, double* out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        for (int c = 0; c < ri; ++c) {
+            double acc = 0.0;
+            for (int a = 0; a < d; ++a)
+                acc += k[i * d + a] * Ak[(int64_t)a * ri + c];
+            out[i * ri + c] = dtype == 1 ? oracle_round_bf16(acc) : (double)(float)acc;
+        }
+}
+
+/* ------------------------------------------------------------------------- */
+/* One decode step whose approximate scores come from an asymmetric pair of */
+/* factors (SAKI page, abstract: the score q k^T is approximated as          */
+/* (q A_q)(k A_k)^T, A_q and A_k of rank r from the SVD of the covariance-   */
+/* weighted query-key operator). The key index holds the stored rows         */
+/* Kidx[t] = round(k_t A_k); for the candidates                               */
+/*   s_t = reduce_j sum_{c < r} (q_j A_q)[c] * Kidx[t][c].                    */
+/* Steps 2, 4 and 5 are those of oracle_decode_pair: the exact attention     */
+/* uses q_hat = q P against the full keys Kt in the PCA basis.                */
+/* Kidx [L][ri]; Aq [d][ri] row-major, its first r columns are used.         */
+/* Other arguments and the return value as for oracle_decode_pair.           */
+/* ------------------------------------------------------------------------- */
+int oracle_decode_pair_asym(const double* Kt, const double* V, const double* Kidx, const double* q,
+                            const double* P, const double* Aq, int L, int d, int ri, int g, int r, int k,
+                            int W, int group_max, double scale, double* out, int32_t* sel, int* n_sel,
+                            double* scores, double* kth)
+{
+    if (k < 0 || W < 0 || (k == 0 && W == 0) || r < 1 || r > ri || ri > d || L < 0)
+        return -1;
+    if (scale == 0.0)
+        scale = 1.0 / sqrt((double)d);
+
+    /* Step 1: the query in the PCA basis (exact attention) and its score    */
+    /* factor q A_q (first r columns).                                       */
+    double* qhat = (double*)malloc(sizeof(double) * (size_t)g * d);
+    double* qt = (double*)malloc(sizeof(double) * (size_t)g * r);
+    oracle_rotate(q, P, g, d, qhat);
+    for (int j = 0; j < g; ++j)
+        for (int c = 0; c < r; ++c) {
+            double acc = 0.0;
+            for (int a = 0; a < d; ++a)
+                acc += q[j * d + a] * Aq[(int64_t)a * ri + c];
+            qt[j * r + c] = acc;
+        }
+
+    /* Step 2: candidates are the tokens outside the forced recent window.    */
+    int w_eff = W < L ? W : L;
+    int ncand = L - w_eff;
+
+    /* Step 3: approximate scores from the key index and the query factor.   */
+    scored_token* cand = (scored_token*)malloc(sizeof(scored_token) * (size_t)(ncand > 0 ? ncand : 1));
+    for (int t = 0; t < ncand; ++t) {
+        const double* x = Kidx + (int64_t)t * ri;
+        double s = group_max ? -INFINITY : 0.0;
+        for (int j = 0; j < g; ++j) {
+            double sj = 0.0;
+            for (int c = 0; c < r; ++c)
+                sj += qt[j * r + c] * x[c];
+            if (group_max)
+                s = sj > s ? sj : s;
+            else
+                s += sj;
+        }
+        cand[t].s = s;
+        cand[t].t = t;
+    }
+    if (scores) {
+        for (int t = 0; t < L; ++t)
+            scores[t] = NAN;
+        for (int t = 0; t < ncand; ++t)
+            scores[t] = cand[t].s;
+    }
+
+    /* Step 4: keep the k best candidates and the recent window.             */
+    int32_t* T = (int32_t*)malloc(sizeof(int32_t) * (size_t)(ncand + w_eff + 1));
+    int nT = keep_top_k_and_window(cand, ncand, k, w_eff, T, kth);
+
+    /* Step 5: exact softmax attention over the kept set (equations (3)-(5)). */
+    oracle_attend_set(Kt, V, qhat, T, nT, d, g, scale, out, NULL);
+
+    if (sel) {
+        for (int i = 0; i < k + W; ++i)
+            sel[i] = i < nT ? T[i] : -1;
+    }
+    if (n_sel)
+        *n_sel = nT;
+    free(T);
+    free(cand);
+    free(qt);
     free(qhat);
     return 0;
 }

@@ -16,18 +16,22 @@ from tests import test_oracle_pins as pins
 MUTATIONS = {
     "rotation transposed": ("acc += x[i * d + a] * P[(int64_t)a * d + c];",
                             "acc += x[i * d + a] * P[(int64_t)c * d + a];"),
-    "trailing dims scored": ("for (int c = 0; c < r; ++c)\n                sj +=",
-                             "for (int c = d - r; c < d; ++c)\n                sj +="),
+    "trailing dims scored": ("for (int c = 0; c < r; ++c)\n                sj += qhat[j * d + c] * kt[c];",
+                             "for (int c = d - r; c < d; ++c)\n                sj += qhat[j * d + c] * kt[c];"),
     "ties to the higher index": ("return (a->t > b->t) - (a->t < b->t);",
                                  "return (a->t < b->t) - (a->t > b->t);"),
     "scale dropped": ("z[i] = s * scale;", "z[i] = s;"),
     "softmax sign": ("z[i] = exp(z[i] - zmax);", "z[i] = exp(zmax - z[i]);"),
     "recent window shifted": ("T[keff + i] = ncand + i;", "T[keff + i] = ncand + i - 1;"),
-    "group: last head only": ("                s += sj;", "                s = sj;"),
+    "group: last head only": ("* kt[c];\n            if (group_max)\n                s = sj > s ? sj : s;\n"
+                              "            else\n                s += sj;",
+                              "* kt[c];\n            if (group_max)\n                s = sj > s ? sj : s;\n"
+                              "            else\n                s = sj;"),
     "bf16 truncates": ("nearbyint(ldexp(v, -spacing_exp))", "trunc(ldexp(v, -spacing_exp))"),
     "dense unnormalised": ("acc += z[t] / denom * V[(int64_t)t * d + c];",
                            "acc += z[t] * V[(int64_t)t * d + c];"),
-    "window not excluded": ("int ncand = L - w_eff;", "int ncand = L - w_eff + (w_eff > 0);"),
+    "window not excluded": ("int ncand = L - w_eff;\n\n    /* Step 3: approximate scores from the leading",
+                            "int ncand = L - w_eff + (w_eff > 0);\n\n    /* Step 3: approximate scores from the leading"),
     "k off by one": ("int keff = k < ncand ? k : ncand;", "int keff = k < ncand ? k - (k > 1) : ncand;"),
     "slab energy not squared": ("e[s] += u * u;", "e[s] += fabs(u);"),
     "slab energy of the first head only": ("for (int j = 0; j < g; ++j)\n                    e[s] +=",
@@ -38,6 +42,14 @@ MUTATIONS = {
                                       "if (e[o] > e[s] || (e[o] == e[s] && o > s))"),
     "slab off by one dim": ("for (int c = 16 * s; c < 16 * s + 16; ++c) {",
                             "for (int c = 16 * s + 1; c < 16 * s + 16; ++c) {"),
+    "asym query factor is P": ("acc += q[j * d + a] * Aq[(int64_t)a * ri + c];",
+                               "acc += q[j * d + a] * P[(int64_t)a * d + c];"),
+    "asym index not rounded": ("out[i * ri + c] = dtype == 1 ? oracle_round_bf16(acc) : (double)(float)acc;",
+                               "out[i * ri + c] = acc;"),
+    "asym group: last head only": ("* x[c];\n            if (group_max)\n                s = sj > s ? sj : s;\n"
+                                   "            else\n                s += sj;",
+                                   "* x[c];\n            if (group_max)\n                s = sj > s ? sj : s;\n"
+                                   "            else\n                s = sj;"),
 }
 
 PIN_FUNCS = [
@@ -61,6 +73,9 @@ PIN_FUNCS = [
     pins.test_magnitude_slabs_energy_is_conserved,
     pins.test_magnitude_slabs_maximise_the_kept_energy,
     pins.test_magnitude_slabs_reduce_and_ties,
+    pins.test_index_keys_with_pca_factor_is_the_appended_slice,
+    pins.test_asym_decode_with_symmetric_factors_is_the_leading_decode,
+    pins.test_asym_decode_brute_force,
 ] + [lambda t=t: pins.test_topk_brute_force(t) for t in range(20)] + [
     lambda n=n: pins.test_golden_fixture(n)
     for n in sorted(x for x in os.listdir(pins.GOLDEN) if x.endswith(".json"))
