@@ -473,6 +473,26 @@ def main():
     assert loki.loki_device_error() == 0
     del mcache
 
+    # the asymmetric scorer (query factor A_q, here P's leading columns) on
+    # the bench cache, same conditions
+    Aq = P[:, :, :spec.r].contiguous()
+
+    def asym_launch(i):
+        loki.loki_decode_attention_asym(cache, batch, qs[i % pool], P, Aq, spec.r, spec.k, mout,
+                                        recent_window=spec.recent_window, stream=stream)
+    for i in range(3):
+        asym_launch(i)
+    a0 = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
+    a1 = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
+    for i in range(10):
+        flush_l2()
+        a0[i].record(stream)
+        asym_launch(i)
+        a1[i].record(stream)
+    torch.cuda.synchronize()
+    asym_ms = statistics.median(x.elapsed_time(y) for x, y in zip(a0, a1))
+    assert loki.loki_device_error() == 0
+
     if rank != 0:
         finish(world)
         return
@@ -514,6 +534,9 @@ def main():
                              "note": "loki_decode_attention_scored on a cache whose key index holds all "
                                      f"{spec.head_dim} dims; r = {spec.r}: the r/16 slabs with the most query "
                                      "energy against the leading r dims, median of 10 L2-flushed launches"},
+        "asym_scorer": {"launch_ms": asym_ms,
+                        "note": "loki_decode_attention_asym on the bench cache (index of the leading 32 dims, "
+                                "A_q = the leading 32 columns of P), median of 10 L2-flushed launches"},
         "dense": {"ms_per_step": dense_ms, "steps_per_s": 1e3 / dense_ms,
                   "achieved_gbs": dense_bytes(spec) / (dense_ms / 1e3) / 1e9},
         "wall_s_timed_loop": wall,

@@ -189,6 +189,22 @@ LOKI_API loki_status loki_prefill_rotate(const loki_cache* cache, const loki_bat
  * of clustered eigenvalues are defined only up to rotations within the
  * cluster. n >= 2. No counterpart call in the pages: it is their offline
  * calibration step done on the device. */
+/* Key index of an asymmetric score factorisation (SAKI page, abstract: the
+ * score q k^T approximated as (q A_q)(k A_k)^T with rank-r factors from the
+ * SVD of the covariance-weighted query-key operator), for every cached
+ * token: index[b, h, t, c] = round(sum_i k[b, h, t, i] A_k[h][i][c]) for
+ * c < index_dims (fp32 sums in row order i = 0, 1, ..., round to nearest
+ * even to the cache type). The key and value rows are not touched.
+ *
+ * k: device [batch][num_kv_heads][max_len][head_dim] in the cache type, keys
+ *    in the original basis (row t of sequence b, head h at
+ *    ((b * num_kv_heads + h) * max_len + t) * head_dim).
+ * A_k: device fp32 [num_kv_heads][head_dim][index_dims], row-major, 16-byte
+ *    aligned. Computing A_k (and A_q) from calibration samples is the
+ *    caller's offline step. max_len >= max_seq_len. */
+LOKI_API loki_status loki_index_keys(const loki_cache* cache, const loki_batch* batch, const void* k,
+                            const float* A_k, int32_t max_len, loki_stream_t stream);
+
 LOKI_API loki_status loki_pca_basis(const void* keys, int32_t num_heads, int64_t n, int32_t head_dim,
                            loki_dtype dtype, float* P, float* eigvals, loki_stream_t stream);
 
@@ -207,6 +223,16 @@ LOKI_API loki_status loki_pca_basis(const void* keys, int32_t num_heads, int64_t
 LOKI_API loki_status loki_append_keys(const loki_cache* cache, const loki_batch* batch,
                              const void* k_new, const void* v_new, const float* P,
                              loki_stream_t stream);
+
+/* loki_append_keys for a cache whose key index holds k A_k (see
+ * loki_index_keys): the key and value rows as loki_append_keys writes them,
+ * the index row round(k_new A_k[h]) with the sums of loki_index_keys, so the
+ * two give identical rows for the same key. A_k: device fp32
+ * [num_kv_heads][head_dim][index_dims], 16-byte aligned (NULL is
+ * LOKI_ERR_INVALID_ARG). */
+LOKI_API loki_status loki_append_keys_asym(const loki_cache* cache, const loki_batch* batch,
+                                  const void* k_new, const void* v_new, const float* P,
+                                  const float* A_k, loki_stream_t stream);
 
 /* Workspace bytes loki_decode_attention needs for these sizes (may be 0). */
 LOKI_API size_t loki_decode_workspace_bytes(const loki_cache* cache, const loki_batch* batch,
@@ -268,6 +294,23 @@ LOKI_API loki_status loki_decode_attention_scored(const loki_cache* cache, const
                                          float scale, loki_scorer scorer, float* out,
                                          int32_t* selected_idx, void* workspace,
                                          size_t workspace_bytes, loki_stream_t stream);
+
+/* loki_decode_attention for a key index that holds k A_k (loki_index_keys,
+ * loki_append_keys_asym): step 2 scores with the query factor instead,
+ *   s_t = reduce_{j in group(h)} (q_j A_q[h])[:r] . index[t, :r]   (fp32),
+ * where q_j A_q[h] is summed in the same order as q_hat (SAKI page, abstract:
+ * asymmetric query and key factors of the score operator). Steps 1, 3 and 4
+ * are unchanged: the exact attention uses q_hat = q P against the full keys.
+ * A_q: device fp32 [num_kv_heads][head_dim][index_dims], 16-byte aligned;
+ * its first r columns are used. Other arguments as for
+ * loki_decode_attention. */
+LOKI_API loki_status loki_decode_attention_asym(const loki_cache* cache, const loki_batch* batch,
+                                       const void* q, int32_t num_q_heads, const float* P,
+                                       const float* A_q, int32_t r, int32_t k,
+                                       const int32_t* k_per_seq, int32_t recent_window,
+                                       loki_group_reduce group_reduce, float scale, float* out,
+                                       int32_t* selected_idx, void* workspace,
+                                       size_t workspace_bytes, loki_stream_t stream);
 
 /* One whole decode step: loki_append_keys(k_new, v_new, P) followed by
  * loki_decode_attention(...) on the same stream, with the same arguments and

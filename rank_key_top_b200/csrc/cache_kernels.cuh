@@ -69,7 +69,8 @@ struct AppendParams {
     const int32_t* seq_lens;
     const void* k_new;
     const void* v_new;
-    const float* P;  // nullable
+    const float* P;   // nullable
+    const float* Ak;  // nullable: [Hkv][D][index_dims], the index row is k A_k
     int num_blocks, Hkv, max_blocks, max_seq_len, index_dims;
 };
 
@@ -139,11 +140,101 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
         const T kt = Elem<T>::from_f(x);
         const int64_t page = page_offset(pb, h, p.Hkv, D);
         reinterpret_cast<T*>(p.k_cache)[page + row_offset_in_page(row, c, D)] = kt;
-        if (c < p.index_dims)
+        if (c < p.index_dims) {
+            T xv = kt;
+            if (p.Ak) {  // key factor of an asymmetric score: (k A_k)[c], summed in row order
+                const float* Ac = p.Ak + (int64_t)h * D * p.index_dims + c;
+                float s = 0.f;
+                for (int i = 0; i < D; ++i) s = fmaf(kin[i], Ac[(int64_t)i * p.index_dims], s);
+                xv = Elem<T>::from_f(s);
+            }
             reinterpret_cast<T*>(p.k_index)[page_offset(pb, h, p.Hkv, p.index_dims) + index_offset_in_page(row, c)] =
-                kt;
+                xv;
+        }
         reinterpret_cast<T*>(p.v_cache)[page + row_offset_in_page(row, c, D)] =
             reinterpret_cast<const T*>(p.v_new)[src + c];
+    }
+}
+
+// Key index of an asymmetric score factorisation for every cached token
+// (SAKI page, abstract: the keys' own rank-r factor): index row
+// round((k A_k)[c]) from keys k in the original basis, fp32 sums in row order
+// (the same order as the append, so both write identical rows).
+struct IndexParams {
+    void* k_index;
+    const int32_t* block_table;
+    const int32_t* seq_lens;
+    const void* k;     // [batch][Hkv][max_len][D], original basis
+    const float* Ak;   // [Hkv][D][index_dims]
+    int num_blocks, Hkv, max_blocks, max_seq_len, max_len, index_dims;
+};
+
+constexpr int kIndexTile = 64;  // tokens per CTA
+
+template <int D>
+constexpr int index_smem_bytes(int index_dims) {
+    return D * index_dims * 4 + kIndexTile * (D + 1) * 4;
+}
+
+// grid (tiles of kIndexTile tokens, batch * Hkv), 256 threads. A_k[h] and the
+// tile's keys (as fp32, rows padded to D + 1 words: conflict-free column
+// reads) are staged in shared memory; each work item is 4 tokens x 4 columns.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) index_keys_kernel(const IndexParams p) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int I = p.index_dims;
+    float* A = reinterpret_cast<float*>(smem);  // [D][I]
+    float* kt = A + D * I;                      // [kIndexTile][D + 1]
+    const int tile = blockIdx.x, pair = blockIdx.y;
+    const int b = pair / p.Hkv, h = pair - b * p.Hkv;
+    int L = p.seq_lens[b];
+    if (L < 0 || L > p.max_seq_len) {
+        if (threadIdx.x == 0 && tile == 0) flag_error(LOKI_DEVERR_SEQ_LEN);
+        L = L < 0 ? 0 : p.max_seq_len;
+    }
+    const int t0 = tile * kIndexTile;
+    if (t0 >= L) return;
+    const int nt = min(kIndexTile, L - t0);
+    const float4* Ah = reinterpret_cast<const float4*>(p.Ak + (int64_t)h * D * I);
+    for (int e = threadIdx.x; e < D * I / 4; e += blockDim.x) reinterpret_cast<float4*>(A)[e] = Ah[e];
+    const T* ks = reinterpret_cast<const T*>(p.k) + (((int64_t)b * p.Hkv + h) * p.max_len + t0) * D;
+    for (int e = threadIdx.x; e < kIndexTile * D; e += blockDim.x) {
+        const int t = e / D, a = e - t * D;
+        kt[t * (D + 1) + a] = t < nt ? Elem<T>::to_f(ks[e]) : 0.f;
+    }
+    __syncthreads();
+    const int nq = I / 4;
+    for (int item = threadIdx.x; item < (kIndexTile / 4) * nq; item += blockDim.x) {
+        const int tq = item / nq, cq = item - tq * nq;
+        if (4 * tq >= nt) continue;
+        float acc[4][4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) acc[u][0] = acc[u][1] = acc[u][2] = acc[u][3] = 0.f;
+        for (int a = 0; a < D; ++a) {
+            const float4 w = *reinterpret_cast<const float4*>(A + a * I + 4 * cq);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float x = kt[(4 * tq + u) * (D + 1) + a];
+                acc[u][0] = fmaf(x, w.x, acc[u][0]);
+                acc[u][1] = fmaf(x, w.y, acc[u][1]);
+                acc[u][2] = fmaf(x, w.z, acc[u][2]);
+                acc[u][3] = fmaf(x, w.w, acc[u][3]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int t = t0 + 4 * tq + u;
+            if (4 * tq + u >= nt) break;
+            const int pb = p.block_table[(int64_t)b * p.max_blocks + t / kBlockTokens];
+            if (pb < 0 || pb >= p.num_blocks) {
+                flag_error(LOKI_DEVERR_BLOCK_ID);
+                continue;
+            }
+            T* xd = reinterpret_cast<T*>(p.k_index) + page_offset(pb, h, p.Hkv, I);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+                xd[index_offset_in_page(t % kBlockTokens, 4 * cq + v)] = Elem<T>::from_f(acc[u][v]);
+        }
     }
 }
 

@@ -86,8 +86,9 @@ loki_status check_append(const loki_cache* cache, const loki_batch* batch, const
 }
 
 loki_status launch_append(const loki_cache* cache, const loki_batch* batch, const void* k_new, const void* v_new,
-                          const float* P, cudaStream_t s) {
+                          const float* P, cudaStream_t s, const float* Ak = nullptr) {
     AppendParams p;
+    p.Ak = Ak;
     p.k_cache = cache->k_cache;
     p.v_cache = cache->v_cache;
     p.k_index = cache->k_index;
@@ -141,7 +142,8 @@ loki_status check_decode(const loki_cache* cache, const loki_batch* batch, const
 loki_status launch_decode(const loki_cache* cache, const loki_batch* batch, const void* q, int32_t num_q_heads,
                           const float* P, int32_t r, int32_t k, const int32_t* k_per_seq, int32_t recent_window,
                           loki_group_reduce group_reduce, float scale, float* out, int32_t* selected_idx,
-                          cudaStream_t s, bool programmatic, bool magnitude = false) {
+                          cudaStream_t s, bool programmatic, int scorer = kScoreLeading,
+                          const float* Aq = nullptr) {
     const int Hkv = cache->num_kv_heads, D = cache->head_dim;
     const int G = num_q_heads / Hkv;
     const int pairs = batch->batch * Hkv;
@@ -155,6 +157,7 @@ loki_status launch_decode(const loki_cache* cache, const loki_batch* batch, cons
     p.k_per_seq = k_per_seq;
     p.q = q;
     p.P = P;
+    p.Aq = Aq;
     p.out = out;
     p.sel = selected_idx;
     p.num_blocks = cache->num_blocks;
@@ -169,7 +172,7 @@ loki_status launch_decode(const loki_cache* cache, const loki_batch* batch, cons
     const double sc = scale == 0.f ? 1.0 / std::sqrt((double)D) : (double)scale;
     p.scale_log2 = (float)(sc * kLog2e);
     return dispatch_tdg<SparseLaunch>(cache->dtype, D, G, p, pairs, (int)batch->max_seq_len, di, s, programmatic,
-                                      magnitude);
+                                      scorer);
 }
 
 }  // namespace
@@ -356,6 +359,52 @@ loki_status loki_append_keys(const loki_cache* cache, const loki_batch* batch, c
     return launch_append(cache, batch, k_new, v_new, P, reinterpret_cast<cudaStream_t>(stream));
 }
 
+loki_status loki_append_keys_asym(const loki_cache* cache, const loki_batch* batch, const void* k_new,
+                                  const void* v_new, const float* P, const float* A_k, loki_stream_t stream) {
+    const loki_status st = check_append(cache, batch, k_new, v_new, P);
+    if (st != LOKI_OK || batch->batch == 0) return st;
+    if (!A_k || !aligned16(A_k)) return LOKI_ERR_INVALID_ARG;
+    return launch_append(cache, batch, k_new, v_new, P, reinterpret_cast<cudaStream_t>(stream), A_k);
+}
+
+loki_status loki_index_keys(const loki_cache* cache, const loki_batch* batch, const void* k, const float* A_k,
+                            int32_t max_len, loki_stream_t stream) {
+    loki_status st = check_cache(cache);
+    if (st != LOKI_OK) return st;
+    if ((st = check_batch(batch)) != LOKI_OK) return st;
+    if (batch->batch == 0 || batch->max_seq_len == 0) return LOKI_OK;
+    if (!k || !A_k || max_len < batch->max_seq_len) return LOKI_ERR_INVALID_ARG;
+    if (!aligned16(A_k)) return LOKI_ERR_INVALID_ARG;
+    if ((int64_t)batch->batch * cache->num_kv_heads > 65535) return LOKI_ERR_UNSUPPORTED;
+    IndexParams p;
+    p.k_index = cache->k_index;
+    p.block_table = batch->block_table;
+    p.seq_lens = batch->seq_lens;
+    p.k = k;
+    p.Ak = A_k;
+    p.num_blocks = cache->num_blocks;
+    p.Hkv = cache->num_kv_heads;
+    p.max_blocks = batch->max_blocks_per_seq;
+    p.max_seq_len = batch->max_seq_len;
+    p.max_len = max_len;
+    p.index_dims = cache->index_dims;
+    const dim3 grid((batch->max_seq_len + kIndexTile - 1) / kIndexTile, batch->batch * cache->num_kv_heads);
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int D = cache->head_dim;
+    auto launch = [&](auto kern, int smem) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return LOKI_ERR_CUDA;
+        kern<<<grid, 256, smem, s>>>(p);
+        return launch_status();
+    };
+    if (cache->dtype == LOKI_BF16) {
+        if (D == 64) return launch(index_keys_kernel<__nv_bfloat16, 64>, index_smem_bytes<64>(p.index_dims));
+        return launch(index_keys_kernel<__nv_bfloat16, 128>, index_smem_bytes<128>(p.index_dims));
+    }
+    if (D == 64) return launch(index_keys_kernel<float, 64>, index_smem_bytes<64>(p.index_dims));
+    return launch(index_keys_kernel<float, 128>, index_smem_bytes<128>(p.index_dims));
+}
+
 int32_t loki_decode_max_seq_len(int32_t head_dim, loki_dtype dtype) {
     (void)dtype;
     if (head_dim != 64 && head_dim != 128) return 0;
@@ -401,7 +450,23 @@ loki_status loki_decode_attention_scored(const loki_cache* cache, const loki_bat
     if (st != LOKI_OK || batch->batch == 0) return st;
     return launch_decode(cache, batch, q, num_q_heads, P, r, k, k_per_seq, recent_window, group_reduce, scale, out,
                          selected_idx, reinterpret_cast<cudaStream_t>(stream), false,
-                         scorer == LOKI_SCORER_MAGNITUDE);
+                         scorer == LOKI_SCORER_MAGNITUDE ? kScoreMagnitude : kScoreLeading);
+}
+
+loki_status loki_decode_attention_asym(const loki_cache* cache, const loki_batch* batch, const void* q,
+                                       int32_t num_q_heads, const float* P, const float* A_q, int32_t r, int32_t k,
+                                       const int32_t* k_per_seq, int32_t recent_window,
+                                       loki_group_reduce group_reduce, float scale, float* out,
+                                       int32_t* selected_idx, void* workspace, size_t workspace_bytes,
+                                       loki_stream_t stream) {
+    (void)workspace;
+    (void)workspace_bytes;
+    const loki_status st = check_decode(cache, batch, q, num_q_heads, P, r, k, recent_window, group_reduce, scale,
+                                        out);
+    if (st != LOKI_OK || batch->batch == 0) return st;
+    if (!A_q || !aligned16(A_q)) return LOKI_ERR_INVALID_ARG;
+    return launch_decode(cache, batch, q, num_q_heads, P, r, k, k_per_seq, recent_window, group_reduce, scale, out,
+                         selected_idx, reinterpret_cast<cudaStream_t>(stream), false, kScoreAsym, A_q);
 }
 
 loki_status loki_decode_step(const loki_cache* cache, const loki_batch* batch, const void* k_new, const void* v_new,

@@ -59,6 +59,7 @@ struct SparseParams {
     const int32_t* k_per_seq;
     const void* q;
     const float* P;
+    const float* Aq;  // [Hkv][D][index_dims] query factor (asymmetric scorer only)
     float* out;
     int32_t* sel;
     int num_blocks, Hkv, max_blocks, max_seq_len, index_dims;
@@ -164,14 +165,23 @@ __device__ __noinline__ int2 radix_boundary(const uint32_t* hcur, int nbins, int
     return make_int2(misc[0], misc[1]);
 }
 
-// MAG selects the scorer. false: the leading r index dims (Loki). true: the
-// r / 16 index slabs (16 dims each) that hold the most energy of the group's
-// rotated query (AQUA page, Algorithm 1 in prose: the dims are picked by the
-// magnitude of q_hat per decode step; the retained energy is what its
-// information-retention loss measures). Here a slab is the unit of choice, so
-// that a block's selected dims stay whole 512-byte (bf16) runs of the index.
-template <typename T, int D, int G, bool MAG>
+// Scorers (template argument SC):
+//  kScoreLeading: q_hat_j against the leading r index dims (Loki).
+//  kScoreMagnitude: the r / 16 index slabs (16 dims each) that hold the most
+//    energy of the group's rotated query (AQUA page, Algorithm 1 in prose: the
+//    dims are picked by the magnitude of q_hat per decode step; the retained
+//    energy is what its information-retention loss measures). A slab is the
+//    unit of choice, so that a block's selected dims stay whole 512-byte
+//    (bf16) runs of the index.
+//  kScoreAsym: q_j A_q[h] against the leading r dims of an index that holds
+//    k A_k (SAKI page, abstract: asymmetric query and key factors of the
+//    score operator); the exact attention still uses q_hat = q P.
+constexpr int kScoreLeading = 0, kScoreMagnitude = 1, kScoreAsym = 2;
+
+template <typename T, int D, int G, int SC>
 __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const SparseParams p) {
+    constexpr bool MAG = SC == kScoreMagnitude;
+    constexpr bool ASYM = SC == kScoreAsym;
     using Geom = SparseGeom<T, D, G>;
     using Core = typename Geom::Core;
     constexpr int NCH = Geom::NCH;
@@ -200,6 +210,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     int32_t* tbl = reinterpret_cast<int32_t*>(smem + p.off_tbl);
     uint32_t* hist = reinterpret_cast<uint32_t*>(smem + p.off_hist);
     float* part = reinterpret_cast<float*>(smem + p.off_part);
+    // the query the scoring uses, [G][D] rows: q_hat, or (asymmetric) q A_q
+    // in `part`, whose first G x D floats only rank 0's own merge writes
+    const float* qsc = ASYM ? part : qhat;
     int32_t* misc = reinterpret_cast<int32_t*>(smem + p.off_misc);
     // misc: [0] boundary digit, [1] count above it, [8..39] suffix-sum scratch,
     //       [40..55] warp kept counts, [56..71] warp equal counts, [72] list length,
@@ -355,10 +368,49 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
             qhat[o] = s;
         }
         __syncthreads();
+        if constexpr (ASYM) {
+            // q A_q[h], first r columns, with q_hat's blocking: thread
+            // (rg, cq) sums its RPG rows for its 4 columns, the row groups'
+            // partial sums are added in the same order as for q_hat
+            const int I = p.index_dims;
+            float a[G][4];
+#pragma unroll
+            for (int j = 0; j < G; ++j) a[j][0] = a[j][1] = a[j][2] = a[j][3] = 0.f;
+            if (4 * cq < p.r) {
+                const float* Ah = p.Aq + (int64_t)h * D * I;
+                float qv[G][RPG];
+#pragma unroll
+                for (int j = 0; j < G; ++j) Vec<T, RPG>::to_float(qraw[j], qv[j]);
+#pragma unroll
+                for (int i = 0; i < RPG; ++i) {
+                    const float4 av = *reinterpret_cast<const float4*>(Ah + (int64_t)(rg * RPG + i) * I + 4 * cq);
+#pragma unroll
+                    for (int j = 0; j < G; ++j) {
+                        const float x = qv[j][i];
+                        a[j][0] = fmaf(x, av.x, a[j][0]);
+                        a[j][1] = fmaf(x, av.y, a[j][1]);
+                        a[j][2] = fmaf(x, av.z, a[j][2]);
+                        a[j][3] = fmaf(x, av.w, a[j][3]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < G; ++j)
+                *reinterpret_cast<float4*>(qscratch + (rg * G + j) * D + 4 * cq) =
+                    make_float4(a[j][0], a[j][1], a[j][2], a[j][3]);
+            __syncthreads();
+            for (int o = tid; o < G * D; o += kThreads) {
+                if (o % D >= p.r) continue;
+                float s = 0.f;
+                for (int g = 0; g < NRG; ++g) s += qscratch[g * G * D + o];
+                part[o] = s;
+            }
+            __syncthreads();
+        }
         if (!p.group_max) {
             for (int c = tid; c < (MAG ? p.index_dims : p.r); c += kThreads) {
                 float s = 0.f;
-                for (int j = 0; j < G; ++j) s += qhat[j * D + c];
+                for (int j = 0; j < G; ++j) s += qsc[j * D + c];
                 qs[c] = s;
             }
         }
@@ -429,7 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
                                 x = (ng == 0 && g < 2) ? split_part(qs[d], g & 1) : 0.f;
                             } else {
                                 const int head = ng * 4 + (g >> 1);
-                                x = head < G ? split_part(qhat[head * D + d], g & 1) : 0.f;
+                                x = head < G ? split_part(qsc[head * D + d], g & 1) : 0.f;
                             }
                         }
                         v[e] = x;
@@ -528,7 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
                         V8::to_float(raw[sb], kf);
 #pragma unroll
                         for (int j = 0; j < G; ++j) {
-                            const float* qq = qhat + j * D + (MAG ? misc[96 + sb] : sb) * 16 + half * 8;
+                            const float* qq = qsc + j * D + (MAG ? misc[96 + sb] : sb) * 16 + half * 8;
 #pragma unroll
                             for (int i = 0; i < 8; ++i) ag[j] = fmaf(qq[i], kf[i], ag[j]);
                         }

@@ -141,19 +141,20 @@ int choose_cluster(SparseParams& p, int max_seq_len, int pairs, int sms, int sme
 
 template <typename T, int D, int G>
 struct SparseLaunch {
-    // magnitude: the scorer that picks index slabs by query energy
+    // scorer: kScoreLeading, kScoreMagnitude or kScoreAsym
     static loki_status run(SparseParams p, int pairs, int max_seq_len, const DeviceInfo& di,
-                           cudaStream_t stream, bool programmatic, bool magnitude) {
-        return magnitude ? run_kernel<true>(p, pairs, max_seq_len, di, stream, programmatic)
-                         : run_kernel<false>(p, pairs, max_seq_len, di, stream, programmatic);
+                           cudaStream_t stream, bool programmatic, int scorer) {
+        if (scorer == kScoreMagnitude) return run_kernel<kScoreMagnitude>(p, pairs, max_seq_len, di, stream, programmatic);
+        if (scorer == kScoreAsym) return run_kernel<kScoreAsym>(p, pairs, max_seq_len, di, stream, programmatic);
+        return run_kernel<kScoreLeading>(p, pairs, max_seq_len, di, stream, programmatic);
     }
 
-    template <bool MAG>
+    template <int SC>
     static loki_status run_kernel(SparseParams p, int pairs, int max_seq_len, const DeviceInfo& di,
                                   cudaStream_t stream, bool programmatic) {
         if (choose_cluster<T, D, G>(p, max_seq_len, pairs, di.sms, di.max_smem_optin) < 1)
             return LOKI_ERR_UNSUPPORTED;
-        auto kern = sparse_decode_kernel<T, D, G, MAG>;
+        auto kern = sparse_decode_kernel<T, D, G, SC>;
         static std::once_flag once;
         static cudaError_t attr_err = cudaSuccess;
         std::call_once(once, [&] {

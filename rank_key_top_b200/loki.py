@@ -71,6 +71,10 @@ _SIGS = {
     "loki_decode_attention_scored": (ctypes.c_int, [_C, _B, _P, _I32, _P, _I32, _I32, _P, _I32,
                                                     ctypes.c_int, ctypes.c_float, ctypes.c_int, _P, _P,
                                                     _P, _SZ, _P]),
+    "loki_decode_attention_asym": (ctypes.c_int, [_C, _B, _P, _I32, _P, _P, _I32, _I32, _P, _I32,
+                                                  ctypes.c_int, ctypes.c_float, _P, _P, _P, _SZ, _P]),
+    "loki_append_keys_asym": (ctypes.c_int, [_C, _B, _P, _P, _P, _P, _P]),
+    "loki_index_keys": (ctypes.c_int, [_C, _B, _P, _P, _I32, _P]),
     "loki_decode_step": (ctypes.c_int, [_C, _B, _P, _P, _P, _I32, _P, _I32, _I32, _P, _I32,
                                         ctypes.c_int, ctypes.c_float, _P, _P, _P, _SZ, _P]),
     "loki_decode_max_seq_len": (_I32, [_I32, ctypes.c_int]),
@@ -218,6 +222,28 @@ def loki_decode_attention_scored(cache, batch, q, P, r, k, out, scorer=LOKI_SCOR
         ctypes.byref(cache.struct), ctypes.byref(batch.struct), _ptr(q), q.shape[1], _ptr(P), r, k,
         _ptr(k_per_seq), recent_window, group_reduce, scale, scorer, _ptr(out), _ptr(selected_idx),
         _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def loki_decode_attention_asym(cache, batch, q, P, A_q, r, k, out, k_per_seq=None, recent_window=0,
+                               group_reduce=LOKI_GROUP_SUM, scale=0.0, selected_idx=None, workspace=None,
+                               stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("loki_decode_attention_asym", _lib.loki_decode_attention_asym(
+        ctypes.byref(cache.struct), ctypes.byref(batch.struct), _ptr(q), q.shape[1], _ptr(P), _ptr(A_q), r, k,
+        _ptr(k_per_seq), recent_window, group_reduce, scale, _ptr(out), _ptr(selected_idx),
+        _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def loki_append_keys_asym(cache, batch, k_new, v_new, P, A_k, stream=None):
+    _check("loki_append_keys_asym", _lib.loki_append_keys_asym(
+        ctypes.byref(cache.struct), ctypes.byref(batch.struct), _ptr(k_new), _ptr(v_new), _ptr(P), _ptr(A_k),
+        _stream(stream)))
+
+
+def loki_index_keys(cache, batch, k, A_k, stream=None):
+    """Fill the key index with k A_k; k is [batch, Hkv, max_len, head_dim]."""
+    _check("loki_index_keys", _lib.loki_index_keys(
+        ctypes.byref(cache.struct), ctypes.byref(batch.struct), _ptr(k), _ptr(A_k), k.shape[2], _stream(stream)))
 
 
 def loki_decode_step(cache, batch, k_new, v_new, q, P, r, k, out, k_per_seq=None, recent_window=0,

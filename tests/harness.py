@@ -78,20 +78,25 @@ def pair_inputs(wl, b, h, q=None):
 
 
 def check_pair(wl, b, h, out_gpu, sel_gpu, r, k, W, group_max=False, scale=0.0, q=None, rtol=None,
-               inputs=None, magnitude_dims=None):
+               inputs=None, magnitude_dims=None, asym=None):
     """Set parity (with the tie band) and output parity for one pair.
 
     magnitude_dims: the key index's width when the magnitude scorer ran (the
     oracle then chooses the scoring slabs the same way, and the input must
     separate the last kept slab from the first dropped one by SLAB_MARGIN, so
     that both sides' choice is the same whatever their precision).
+    asym: (Kidx, A_q) of the pair when the asymmetric scorer ran: the
+    oracle's own key-index rows round(k A_k) and the query factor.
     Returns (output error on the GPU's set, output error on the oracle's set)."""
     s = wl.spec
     g = s.group
     L = s.seq_lens[b]
     kb = int(wl.k_per_seq[b]) if wl.k_per_seq is not None else k
     Kt, V, qq, P = inputs if inputs is not None else pair_inputs(wl, b, h, q)
-    if magnitude_dims is None:
+    if asym is not None:
+        res = oracle.decode_pair_asym(Kt, V, asym[0], qq, P, asym[1], r, kb, W=W, group_max=group_max,
+                                      scale=scale)
+    elif magnitude_dims is None:
         res = oracle.decode_pair(Kt, V, qq, P, r=r, k=kb, W=W, group_max=group_max, scale=scale)
     else:
         res = oracle.decode_pair_magnitude(Kt, V, qq, P, r, kb, magnitude_dims, W=W, group_max=group_max,

@@ -161,6 +161,31 @@ def test_decode_scored_rejects(loki, scorer, kw, status):
     assert scored(loki, c, b, scorer, **kw) == status
 
 
+def test_asymmetric_entries_reject(loki):
+    c, b = structs(loki)
+    lib = loki.raw()
+
+    def dec(Aq, r=32):
+        return lib.loki_decode_attention_asym(ctypes.byref(c), ctypes.byref(b), FAKE, 32, FAKE, Aq, r, 8, None, 0,
+                                              0, 0.0, FAKE, None, None, 0, None)
+    assert dec(None) == 1
+    assert dec(FAKE + 4) == 1
+    assert dec(FAKE, r=48) == 1        # r above index_dims
+    assert dec(FAKE, r=24) == 2
+    assert lib.loki_append_keys_asym(ctypes.byref(c), ctypes.byref(b), FAKE, FAKE, FAKE, None, None) == 1
+    assert lib.loki_append_keys_asym(ctypes.byref(c), ctypes.byref(b), FAKE, FAKE, FAKE, FAKE + 8, None) == 1
+    assert lib.loki_append_keys_asym(ctypes.byref(c), ctypes.byref(b), None, FAKE, FAKE, FAKE, None) == 1
+    assert lib.loki_index_keys(ctypes.byref(c), ctypes.byref(b), None, FAKE, 64, None) == 1
+    assert lib.loki_index_keys(ctypes.byref(c), ctypes.byref(b), FAKE, None, 64, None) == 1
+    assert lib.loki_index_keys(ctypes.byref(c), ctypes.byref(b), FAKE, FAKE + 4, 64, None) == 1
+    assert lib.loki_index_keys(ctypes.byref(c), ctypes.byref(b), FAKE, FAKE, 32, None) == 1  # max_len short
+    c0, b0 = structs(loki, B=0)
+    assert lib.loki_index_keys(ctypes.byref(c0), ctypes.byref(b0), None, None, 0, None) == 0
+    assert lib.loki_append_keys_asym(ctypes.byref(c0), ctypes.byref(b0), None, None, None, None, None) == 0
+    assert lib.loki_decode_attention_asym(ctypes.byref(c0), ctypes.byref(b0), None, 32, None, None, 32, 8, None, 0,
+                                          0, 0.0, None, None, None, 0, None) == 0
+
+
 def test_empty_batch_is_a_no_op(loki):
     c, b = structs(loki, B=0)
     assert decode(loki, c, b, q=None, P=None, out=None) == 0

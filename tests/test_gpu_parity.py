@@ -628,3 +628,141 @@ def test_magnitude_scorer_with_every_slab_is_leading(cuda_lib, group_max):
     a = dev.decode(group_max=group_max)
     b = dev.decode(group_max=group_max, scorer=cuda_lib.LOKI_SCORER_MAGNITUDE)
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+# ---------------------------------------------------------------------------
+# Asymmetric score factors: key index k A_k, append, decode with q A_q
+# ---------------------------------------------------------------------------
+
+def saki_inputs(wl, index_dims):
+    """Keys in the original basis, and per kv head the oracle's closed-form
+    factors A_q, A_k [Hkv, d, index_dims] calibrated on the head's cached keys
+    plus fresh key draws, and on fresh query batches: at least 4 d samples of
+    each, so that both second moments are well conditioned."""
+    s = wl.spec
+    g, d = s.group, s.head_dim
+    K_orig = unrotated_keys(wl)
+    need = 4 * d
+    qcal = torch.cat([synth.draw_query_batch(s, 100 + i) for i in range(-(-need // (s.batch * g)))])
+    kcal = torch.cat([synth.draw_new_tokens(s, 300 + i)[0] for i in range(-(-need // s.batch))])
+    Aq = torch.empty(s.num_kv_heads, d, index_dims)
+    Ak = torch.empty_like(Aq)
+    for h in range(s.num_kv_heads):
+        Kcal = torch.cat([K_orig[b, h, :L] for b, L in enumerate(s.seq_lens)] + [kcal[:, h]]).double().numpy()
+        Qcal = qcal[:, h * g:(h + 1) * g].reshape(-1, d).double().numpy()
+        a, b, _ = oracle.saki_factors(Qcal, Kcal, index_dims)
+        Aq[h], Ak[h] = torch.from_numpy(a), torch.from_numpy(b)
+    return K_orig, Aq, Ak
+
+
+def check_index_rows(got, k, A, dtype):
+    """Index rows against the oracle's round(k A): equal, except where the
+    exact value lies within the fp32 summation bound of the rounding
+    midpoint between the two."""
+    want = oracle.index_keys(k, A, dtype)
+    exact = k @ A
+    bound = k.shape[1] * 2.0 ** -24 * (np.abs(k)[:, :, None] * np.abs(A)[None]).sum(axis=1)
+    mism = got != want
+    assert np.all(np.abs(exact[mism] - (got[mism] + want[mism]) / 2) <= bound[mism])
+    return int(mism.sum())
+
+
+@pytest.mark.parametrize("dtype,D,I,lens", [("bf16", 128, 32, [300, 1000, 0, 1, 129]), ("f32", 64, 64, [257, 40]),
+                                            ("bf16", 64, 16, [70])])
+def test_index_keys_matches_oracle(cuda_lib, dtype, D, I, lens):
+    s = spec(num_q_heads=4, num_kv_heads=2, seq_lens=lens, head_dim=D, dtype=dtype, r=16)
+    wl = synth.make_workload(s)
+    dev = harness.Device(wl, cuda_lib, index_dims=I)
+    K_orig, _, Ak = saki_inputs(wl, I)
+    cuda_lib.loki_index_keys(dev.cache, dev.batch, K_orig.cuda(), Ak.cuda().contiguous())
+    torch.cuda.synchronize()
+    assert cuda_lib.loki_device_error() == 0
+    for b, L in enumerate(lens):
+        for h in range(s.num_kv_heads):
+            K, V, X = read_pair(dev, b, h, L)
+            assert torch.equal(K, wl.Kt[b, h, :L]) and torch.equal(V, wl.V[b, h, :L])
+            check_index_rows(X.double().numpy(), K_orig[b, h, :L].double().numpy(), Ak[h].double().numpy(), dtype)
+
+
+@pytest.mark.parametrize("dtype,D", [("bf16", 128), ("f32", 64)])
+def test_append_asym_matches_oracle_and_index_keys(cuda_lib, dtype, D):
+    """The appended index row is round(k_new A_k), and bit-identical to the
+    row loki_index_keys writes for the same key."""
+    s = spec(num_q_heads=8, num_kv_heads=4, seq_lens=[31, 32, 100, 0], head_dim=D, dtype=dtype)
+    wl = synth.make_workload(s)
+    I = 32
+    dev = harness.Device(wl, cuda_lib, index_dims=I)
+    K_orig, _, Ak = saki_inputs(wl, I)
+    Ak_dev = Ak.cuda().contiguous()
+    k_new, v_new = synth.draw_new_tokens(s, step=0)
+    lens = torch.tensor([n + 1 for n in s.seq_lens], dtype=torch.int32)
+    batch = cuda_lib.Batch(wl.block_table.cuda(), lens.cuda(), int(lens.max()))
+    cuda_lib.loki_append_keys_asym(dev.cache, batch, k_new.cuda(), v_new.cuda(), dev.P, Ak_dev)
+    torch.cuda.synchronize()
+    assert cuda_lib.loki_device_error() == 0
+    appended = {}
+    for b, L in enumerate(lens.tolist()):
+        for h in range(s.num_kv_heads):
+            K, V, X = read_pair(dev, b, h, L)
+            assert torch.equal(V[L - 1], v_new[b, h])
+            assert torch.equal(K[:L - 1], wl.Kt[b, h, :L - 1])
+            check_index_rows(X[L - 1:].double().numpy(), k_new[b, h][None].double().numpy(),
+                             Ak[h].double().numpy(), dtype)
+            appended[(b, h)] = X[L - 1].clone()
+    K_full = torch.zeros(s.batch, s.num_kv_heads, int(lens.max()), D, dtype=K_orig.dtype)
+    K_full[:, :, :K_orig.shape[2]] = K_orig[:, :, :int(lens.max())]
+    for b, L in enumerate(lens.tolist()):
+        K_full[b, :, L - 1] = k_new[b]
+    cuda_lib.loki_index_keys(dev.cache, batch, K_full.cuda(), Ak_dev)
+    torch.cuda.synchronize()
+    for (b, h), row in appended.items():
+        assert torch.equal(read_pair(dev, b, h, lens[b].item())[2][-1], row)
+
+
+@pytest.mark.parametrize("dtype,D,Hq,Hkv,I,r,group_max,lens", [
+    ("bf16", 128, 8, 2, 32, 32, False, [20000, 3000, 777, 33]),
+    ("bf16", 128, 16, 2, 64, 16, True, [3000, 777]),
+    ("f32", 64, 4, 1, 64, 48, False, [3000, 0, 500]),
+    ("bf16", 64, 2, 2, 32, 32, True, [2500, 1]),
+])
+def test_asym_decode_matches_oracle(cuda_lib, dtype, D, Hq, Hkv, I, r, group_max, lens):
+    s = spec(dtype=dtype, head_dim=D, num_q_heads=Hq, num_kv_heads=Hkv, seq_lens=lens, r=r, k=150,
+             recent_window=5)
+    wl = synth.make_workload(s)
+    dev = harness.Device(wl, cuda_lib, index_dims=I)
+    K_orig, Aq, Ak = saki_inputs(wl, I)
+    cuda_lib.loki_index_keys(dev.cache, dev.batch, K_orig.cuda(), Ak.cuda().contiguous())
+    out = torch.full((s.batch, Hq, D), float("nan"), device="cuda")
+    sel = torch.full((s.batch, Hkv, s.k + s.recent_window), -7, dtype=torch.int32, device="cuda")
+    cuda_lib.loki_decode_attention_asym(dev.cache, dev.batch, dev.q, dev.P, Aq.cuda().contiguous(), r, s.k, out,
+                                        recent_window=s.recent_window,
+                                        group_reduce=cuda_lib.LOKI_GROUP_MAX if group_max else cuda_lib.LOKI_GROUP_SUM,
+                                        selected_idx=sel)
+    torch.cuda.synchronize()
+    assert cuda_lib.loki_device_error() == 0
+    out, sel = out.cpu(), sel.cpu()
+    for b, L in enumerate(lens):
+        for h in range(Hkv):
+            Kidx = oracle.index_keys(K_orig[b, h, :L].double().numpy(), Ak[h].double().numpy(), dtype)
+            harness.check_pair(wl, b, h, out, sel, r, s.k, s.recent_window, group_max=group_max,
+                               asym=(Kidx, Aq[h].double().numpy()))
+
+
+@pytest.mark.parametrize("group_max", [False, True])
+def test_asym_decode_with_pca_factor_is_leading(cuda_lib, group_max):
+    """A_q = the first index_dims columns of P on an index that holds the
+    keys' leading dims: q A_q is summed like q_hat, so the asymmetric decode
+    is the leading decode bit for bit."""
+    s = spec(num_q_heads=8, num_kv_heads=2, seq_lens=[6000, 900], r=32, k=200, recent_window=3)
+    wl = synth.make_workload(s)
+    dev = harness.Device(wl, cuda_lib, index_dims=64)
+    a = dev.decode(group_max=group_max)
+    out = torch.full_like(a[0], float("nan")).cuda()
+    sel = torch.full_like(a[1], -7).cuda()
+    Aq = dev.P[:, :, :64].contiguous()
+    cuda_lib.loki_decode_attention_asym(dev.cache, dev.batch, dev.q, dev.P, Aq, s.r, s.k, out,
+                                        recent_window=s.recent_window,
+                                        group_reduce=cuda_lib.LOKI_GROUP_MAX if group_max else cuda_lib.LOKI_GROUP_SUM,
+                                        selected_idx=sel)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], out.cpu()) and torch.equal(a[1], sel.cpu())
