@@ -181,7 +181,7 @@ constexpr int index_smem_bytes(int index_dims) {
 // reads) are staged in shared memory; each work item is 4 tokens x 4 columns.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) index_keys_kernel(const IndexParams p) {
-    extern __shared__ __align__(16) unsigned char smem[];
+    extern __shared__ __align__(128) unsigned char smem[];
     const int I = p.index_dims;
     float* A = reinterpret_cast<float*>(smem);  // [D][I]
     float* kt = A + D * I;                      // [kIndexTile][D + 1]

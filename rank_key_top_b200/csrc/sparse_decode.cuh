@@ -490,15 +490,18 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
                     qb[ng][sb][1] = pack_bf16(v[2], v[3]);
                 }
             const int arow = (lane & 7) + 8 * ((lane >> 3) & 1), ahalf = lane >> 4;
-            for (int it = 0; it < my_blocks; ++it) {
+            // block it's slot into fragments, then the slot's refill
+            auto load_block = [&](int it, uint32_t (&a)[RMAX][4]) {
                 wait_slot();
                 const unsigned char* sl = wring + (it & smask) * p.slot_bytes;
-                uint32_t a[RMAX][4];
 #pragma unroll
                 for (int sb = 0; sb < RMAX; ++sb)
                     if (sb < R16) ldmatrix_x4(a[sb][0], a[sb][1], a[sb][2], a[sb][3], sl + sb * 512 + arow * 32 + ahalf * 16);
                 __syncwarp();
                 refill(it + S);
+            };
+            // block it's scores, keys and digit-0 histogram counts
+            auto score_block = [&](int it, const uint32_t (&a)[RMAX][4]) {
                 float sc0 = -INFINITY, sc1 = -INFINITY;  // tokens g and g + 8
 #pragma unroll
                 for (int ng = 0; ng < SG; ++ng) {
@@ -532,6 +535,19 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
                         atomicAdd(&hist[key >> 21], 1u);
                     }
                 }
+            };
+            // U blocks per iteration (two when the fragments are small): both
+            // are loaded before either is scored, so their MMA chains overlap.
+            // A second block past the warp's last one reads a stale slot and
+            // stores nothing (its tokens are past n_cand_loc); its refill
+            // commits empty groups only.
+            constexpr int U = RMAX <= 2 ? 2 : 1;
+            for (int it = 0; it < my_blocks; it += U) {
+                uint32_t a[U][RMAX][4];
+#pragma unroll
+                for (int u = 0; u < U; ++u) load_block(it + u, a[u]);
+#pragma unroll
+                for (int u = 0; u < U; ++u) score_block(it + u, a[u]);
             }
         };
         auto body = [&](auto rmax_tag) {
