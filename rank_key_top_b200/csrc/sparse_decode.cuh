@@ -11,9 +11,12 @@
 //     low-dimensional space). Each warp owns a private ring of S slots; a
 //     slot receives the leading r index dims of one 16-token block, one
 //     contiguous run of r*16 elements, as 16-byte cp.async pieces from all
-//     lanes. Scores become order-preserving uint32 keys in shared memory;
-//     the histogram of their top 11 bits is built on the fly with shared
-//     atomics.
+//     lanes; with r <= 32 a warp loads two blocks before scoring either.
+//     Scores become order-preserving uint32 keys in shared memory; the
+//     histogram of their top 11 bits is built on the fly with shared
+//     atomics. Two other scorers share the kernel (template argument SC, at
+//     the kernel's declaration): the index slabs with the most query energy,
+//     and asymmetric factors (q A_q against an index of k A_k).
 //  3. top-k (Loki page, abstract: rank and select tokens): an exact radix
 //     select with digits of 11, 11 and 10 bits. After each digit the CTAs of
 //     the cluster sum their histograms through distributed shared memory, so
