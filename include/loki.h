@@ -267,8 +267,11 @@ LOKI_API size_t loki_decode_workspace_bytes(const loki_cache* cache, const loki_
  * workspace: device, >= loki_decode_workspace_bytes(); may be NULL if that is 0.
  *
  * Unsupported (LOKI_ERR_UNSUPPORTED): head_dim other than 64/128, group size
- * other than 1, 2, 4, 8, r not a multiple of 16, or max_seq_len above
- * loki_decode_max_seq_len(). */
+ * other than 1, 2, 4, 8, r not a multiple of 16, max_seq_len above
+ * loki_decode_max_seq_len(), or a long sequence whose per-CTA state does not
+ * fit in shared memory for any cluster size (only above 16384 tokens, for
+ * some combinations of group size, cache type and head_dim; group size 8 is
+ * the most limited). All of these are found before anything is launched. */
 LOKI_API loki_status loki_decode_attention(const loki_cache* cache, const loki_batch* batch,
                                   const void* q, int32_t num_q_heads, const float* P,
                                   int32_t r, int32_t k, const int32_t* k_per_seq,
@@ -331,7 +334,12 @@ LOKI_API loki_status loki_decode_step(const loki_cache* cache, const loki_batch*
                              void* workspace, size_t workspace_bytes,
                              loki_stream_t stream);
 
-/* Largest max_seq_len loki_decode_attention accepts for this cache shape. */
+/* Largest max_seq_len loki_decode_attention accepts for this cache shape
+ * (262144 tokens). Some group sizes fit less in a CTA's shared memory: for
+ * those, longer sequences are rejected with LOKI_ERR_UNSUPPORTED before any
+ * launch (bf16: from 131072 tokens at head_dim 64 with group size 8; fp32:
+ * from 65536 tokens at head_dim 128 with group size 8; every combination
+ * accepts at least 16384 tokens). */
 LOKI_API int32_t loki_decode_max_seq_len(int32_t head_dim, loki_dtype dtype);
 
 /* Workspace bytes loki_dense_attention needs for these sizes. */

@@ -139,6 +139,14 @@ loki_status check_decode(const loki_cache* cache, const loki_batch* batch, const
     return LOKI_OK;
 }
 
+// Long sequences with large groups can exceed the shared memory of any
+// cluster size: checked after the arguments, before anything is launched.
+loki_status check_decode_fits(const loki_cache* cache, const loki_batch* batch, int32_t num_q_heads, int32_t r) {
+    const int Hkv = cache->num_kv_heads;
+    return dispatch_tdg<SparseFits>(cache->dtype, cache->head_dim, num_q_heads / Hkv, (int)r,
+                                    (int)(batch->batch * Hkv), (int)batch->max_seq_len, device_info());
+}
+
 loki_status launch_decode(const loki_cache* cache, const loki_batch* batch, const void* q, int32_t num_q_heads,
                           const float* P, int32_t r, int32_t k, const int32_t* k_per_seq, int32_t recent_window,
                           loki_group_reduce group_reduce, float scale, float* out, int32_t* selected_idx,
@@ -429,9 +437,9 @@ loki_status loki_decode_attention(const loki_cache* cache, const loki_batch* bat
                                   loki_stream_t stream) {
     (void)workspace;
     (void)workspace_bytes;
-    const loki_status st = check_decode(cache, batch, q, num_q_heads, P, r, k, recent_window, group_reduce, scale,
-                                        out);
+    loki_status st = check_decode(cache, batch, q, num_q_heads, P, r, k, recent_window, group_reduce, scale, out);
     if (st != LOKI_OK || batch->batch == 0) return st;
+    if ((st = check_decode_fits(cache, batch, num_q_heads, r)) != LOKI_OK) return st;
     return launch_decode(cache, batch, q, num_q_heads, P, r, k, k_per_seq, recent_window, group_reduce, scale, out,
                          selected_idx, reinterpret_cast<cudaStream_t>(stream), false);
 }
@@ -445,9 +453,9 @@ loki_status loki_decode_attention_scored(const loki_cache* cache, const loki_bat
     (void)workspace;
     (void)workspace_bytes;
     if (scorer != LOKI_SCORER_LEADING && scorer != LOKI_SCORER_MAGNITUDE) return LOKI_ERR_INVALID_ARG;
-    const loki_status st = check_decode(cache, batch, q, num_q_heads, P, r, k, recent_window, group_reduce, scale,
-                                        out);
+    loki_status st = check_decode(cache, batch, q, num_q_heads, P, r, k, recent_window, group_reduce, scale, out);
     if (st != LOKI_OK || batch->batch == 0) return st;
+    if ((st = check_decode_fits(cache, batch, num_q_heads, r)) != LOKI_OK) return st;
     return launch_decode(cache, batch, q, num_q_heads, P, r, k, k_per_seq, recent_window, group_reduce, scale, out,
                          selected_idx, reinterpret_cast<cudaStream_t>(stream), false,
                          scorer == LOKI_SCORER_MAGNITUDE ? kScoreMagnitude : kScoreLeading);
@@ -461,10 +469,10 @@ loki_status loki_decode_attention_asym(const loki_cache* cache, const loki_batch
                                        loki_stream_t stream) {
     (void)workspace;
     (void)workspace_bytes;
-    const loki_status st = check_decode(cache, batch, q, num_q_heads, P, r, k, recent_window, group_reduce, scale,
-                                        out);
+    loki_status st = check_decode(cache, batch, q, num_q_heads, P, r, k, recent_window, group_reduce, scale, out);
     if (st != LOKI_OK || batch->batch == 0) return st;
     if (!A_q || !aligned16(A_q)) return LOKI_ERR_INVALID_ARG;
+    if ((st = check_decode_fits(cache, batch, num_q_heads, r)) != LOKI_OK) return st;
     return launch_decode(cache, batch, q, num_q_heads, P, r, k, k_per_seq, recent_window, group_reduce, scale, out,
                          selected_idx, reinterpret_cast<cudaStream_t>(stream), false, kScoreAsym, A_q);
 }
@@ -480,6 +488,7 @@ loki_status loki_decode_step(const loki_cache* cache, const loki_batch* batch, c
     if (st != LOKI_OK) return st;
     st = check_decode(cache, batch, q, num_q_heads, P, r, k, recent_window, group_reduce, scale, out);
     if (st != LOKI_OK || batch->batch == 0) return st;
+    if ((st = check_decode_fits(cache, batch, num_q_heads, r)) != LOKI_OK) return st;
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((st = launch_append(cache, batch, k_new, v_new, P, s)) != LOKI_OK) return st;
     return launch_decode(cache, batch, q, num_q_heads, P, r, k, k_per_seq, recent_window, group_reduce, scale, out,

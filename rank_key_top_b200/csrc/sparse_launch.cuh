@@ -117,8 +117,10 @@ bool sparse_layout_fit(SparseParams& p, int max_seq_len, int smem_optin) {
 }
 
 // Cluster size: enough CTAs that each holds at most kCtaTokenCap tokens and
-// the layout fits in shared memory, then as many as still fit every cluster
-// on the GPU at once (one CTA per SM), keeping at least 512 tokens per CTA.
+// the layout fits in shared memory, then the largest size that still fits
+// every cluster on the GPU at once (one CTA per SM), keeps at least 512
+// tokens per CTA and whose layout fits (rank 0's merge slots grow with the
+// cluster). Returns -1 when no size up to 16 fits.
 template <typename T, int D, int G>
 int choose_cluster(SparseParams& p, int max_seq_len, int pairs, int sms, int smem_optin) {
     const int nblk = (max_seq_len + kBlockTokens - 1) / kBlockTokens;
@@ -129,15 +131,30 @@ int choose_cluster(SparseParams& p, int max_seq_len, int pairs, int sms, int sme
         p.C = C;
         if (sparse_layout_fit<T, D, G>(p, max_seq_len, smem_optin)) break;
     }
+    int best = C;
     for (int cand = C + 1; cand <= 16; ++cand) {
         if ((int64_t)pairs * cand > sms) break;
         if (nblk / cand < 32) break;
-        C = cand;
+        p.C = cand;
+        if (sparse_layout_fit<T, D, G>(p, max_seq_len, smem_optin)) best = cand;
     }
+    C = best;
     p.C = C;
     sparse_layout_fit<T, D, G>(p, max_seq_len, smem_optin);
     return C;
 }
+
+// Whether the decode kernel has a cluster size and layout for this shape
+// (checked before anything of a call is launched).
+template <typename T, int D, int G>
+struct SparseFits {
+    static loki_status run(int r, int pairs, int max_seq_len, const DeviceInfo& di) {
+        SparseParams p = {};
+        p.r = r;
+        return choose_cluster<T, D, G>(p, max_seq_len, pairs, di.sms, di.max_smem_optin) < 1 ? LOKI_ERR_UNSUPPORTED
+                                                                                           : LOKI_OK;
+    }
+};
 
 template <typename T, int D, int G>
 struct SparseLaunch {
