@@ -10,6 +10,10 @@
 #include <cstdio>
 #include <cstdlib>
 
+#include "cache_kernels.cuh"
+#include "dense.cuh"
+#include "pca.cuh"
+#include "rotate_prefill.cuh"
 #include "sparse_launch.cuh"
 
 using namespace loki;
@@ -107,8 +111,58 @@ void check_groups(const char* tname, int sms, int optin) {
     check<T, D, 8>(tname, sms, optin);
 }
 
+// The other kernels' fixed shared-memory sizes against the opt-in limit.
+template <typename T, int D, int G>
+void check_dense(const char* tname, int optin) {
+    using Geom = DenseGeom<T, D, G>;
+    ++cases;
+    if (!(Geom::SMEM_BYTES <= optin && Geom::GS >= 1)) {
+        std::printf("FAIL dense T=%s D=%d G=%d smem=%d\n", tname, D, G, Geom::SMEM_BYTES);
+        ++failures;
+    }
+}
+
+template <int D>
+void check_fixed(int optin) {
+    const int pca_static = 4 * (D / 2) * 4;  // the Jacobi round's rotation table
+    const int sizes[] = {rotate_smem_bytes<D>(), pca_smem_bytes<D>() + pca_static};
+    const char* names[] = {"rotate_prefill", "pca"};
+    for (int i = 0; i < 2; ++i) {
+        ++cases;
+        if (sizes[i] > optin) {
+            std::printf("FAIL %s D=%d smem=%d\n", names[i], D, sizes[i]);
+            ++failures;
+        }
+    }
+    for (int I = 16; I <= D; I += 16) {
+        ++cases;
+        if (index_smem_bytes<D>(I) > optin) {
+            std::printf("FAIL index_keys D=%d I=%d smem=%d\n", D, I, index_smem_bytes<D>(I));
+            ++failures;
+        }
+    }
+}
+
 int main() {
     const int sms = 148, optin = 227 * 1024;  // B200: SMs, opt-in shared memory per block
+    check_dense<__nv_bfloat16, 64, 1>("bf16", optin);
+    check_dense<__nv_bfloat16, 64, 2>("bf16", optin);
+    check_dense<__nv_bfloat16, 64, 4>("bf16", optin);
+    check_dense<__nv_bfloat16, 64, 8>("bf16", optin);
+    check_dense<__nv_bfloat16, 128, 1>("bf16", optin);
+    check_dense<__nv_bfloat16, 128, 2>("bf16", optin);
+    check_dense<__nv_bfloat16, 128, 4>("bf16", optin);
+    check_dense<__nv_bfloat16, 128, 8>("bf16", optin);
+    check_dense<float, 64, 1>("f32", optin);
+    check_dense<float, 64, 2>("f32", optin);
+    check_dense<float, 64, 4>("f32", optin);
+    check_dense<float, 64, 8>("f32", optin);
+    check_dense<float, 128, 1>("f32", optin);
+    check_dense<float, 128, 2>("f32", optin);
+    check_dense<float, 128, 4>("f32", optin);
+    check_dense<float, 128, 8>("f32", optin);
+    check_fixed<64>(optin);
+    check_fixed<128>(optin);
     check_groups<__nv_bfloat16, 64>("bf16", sms, optin);
     check_groups<__nv_bfloat16, 128>("bf16", sms, optin);
     check_groups<float, 64>("f32", sms, optin);

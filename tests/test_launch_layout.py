@@ -1,6 +1,7 @@
-"""Host-side invariants of the decode kernel's launch geometry (cluster size,
-shared-memory layout), checked by compiling tests/host/layout_check.cu
-against the library's own launch header and running it on the CPU."""
+"""Host-side invariants of the launch geometry: the decode kernel's cluster
+size and shared-memory layout for every supported shape, and the other
+kernels' shared-memory sizes against the opt-in limit. tests/host/layout_check.cu
+is compiled against the library's own headers and run on the CPU."""
 import os
 import shutil
 import subprocess
