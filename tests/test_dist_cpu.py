@@ -50,3 +50,39 @@ def test_single_process_defaults(monkeypatch):
     assert rdist.init_from_env("gloo")[1] == 1
     assert rdist.max_over_ranks(3.0, 1) == 3.0
     assert rdist.aggregate_rate(10, 1, 2.0) == 5.0
+
+
+def leaving_worker(rank, world, port, out):
+    """Rank 1 joins the group, then leaves between steps (exits without its
+    next collective); rank 0's next collective must end with an error, not
+    wait for ever."""
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    r, w, _ = rdist.init_from_env("gloo", timeout_s=10)
+    rdist.barrier(w)
+    if r == 1:
+        out[r] = "left"
+        os._exit(0)
+    try:
+        rdist.max_over_ranks(1.0, w, device="cpu")
+        out[r] = "no error"
+    except Exception as e:  # the process group reports the missing peer
+        out[r] = "error: " + type(e).__name__
+    os._exit(0)
+
+
+def test_rank_that_leaves_ends_the_others_collective():
+    port = free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        ctx = mp.spawn(leaving_worker, args=(2, port, out), nprocs=2, join=False)
+        for p in ctx.processes:
+            p.join(timeout=90)
+        alive = [p.is_alive() for p in ctx.processes]
+        for p in ctx.processes:
+            if p.is_alive():
+                p.kill()
+        res = dict(out)
+    assert not any(alive), "a rank was still waiting"
+    assert res[1] == "left"
+    assert res[0].startswith("error"), res[0]
