@@ -68,6 +68,14 @@ def _load():
         lib.oracle_magnitude_slabs.restype = ctypes.c_int
         lib.oracle_magnitude_slabs.argtypes = [_D, _D, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                ctypes.c_int, ctypes.c_int, _I32, _D]
+        lib.oracle_magnitude_dims.restype = ctypes.c_int
+        lib.oracle_magnitude_dims.argtypes = [_D, _D, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_int, ctypes.c_int, _I32, _D]
+        lib.oracle_decode_pair_dims.restype = ctypes.c_int
+        lib.oracle_decode_pair_dims.argtypes = [_D, _D, _D, _D, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_int, ctypes.c_double, _D, _I32,
+                                                ctypes.POINTER(ctypes.c_int), _D, _D, _I32]
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
         _lib = lib
@@ -151,7 +159,7 @@ def attend_set(Kt, V, qhat, T, scale=0.0, return_weights=False):
 
 
 class PairResult:
-    __slots__ = ("out", "sel", "n_sel", "scores", "kth", "slabs", "energy")
+    __slots__ = ("out", "sel", "n_sel", "scores", "kth", "slabs", "energy", "dims", "weight")
 
 
 def decode_pair(Kt, V, q, P, r, k, W=0, group_max=False, scale=0.0):
@@ -206,6 +214,47 @@ def decode_pair_magnitude(Kt, V, q, P, r, k, index_dims, W=0, group_max=False, s
     perm = np.concatenate([front, np.setdiff1d(np.arange(d), front)])
     res = decode_pair(Kt[:, perm], V, q, P[:, perm], r, k, W=W, group_max=group_max, scale=scale)
     res.slabs, res.energy = slabs, energy
+    return res
+
+
+def magnitude_dims(q, P, r, index_dims, group_max=False):
+    """The r index dims of largest projected-query magnitude, ascending, and
+    every dim's magnitude; see oracle_magnitude_dims in oracle.c (AQUA page,
+    Algorithm 1 in prose and appendix on complexity, step 2)."""
+    q, P = _f64(q), _f64(P)
+    g, d = q.shape
+    dims = np.empty(r, dtype=np.int32)
+    weight = np.empty(index_dims)
+    rc = _load().oracle_magnitude_dims(_p(q), _p(P), d, g, index_dims, r, 1 if group_max else 0,
+                                       _p(dims, _I32), _p(weight))
+    if rc != 0:
+        raise ValueError("oracle_magnitude_dims rejected its arguments")
+    return dims, weight
+
+
+def decode_pair_dims(Kt, V, q, P, r, k, index_dims, W=0, group_max=False, scale=0.0):
+    """One pair's decode step scored with the r dims of largest query
+    magnitude; see oracle_decode_pair_dims in oracle.c. The result also
+    carries `dims` and `weight`."""
+    Kt, V, q, P = _f64(Kt), _f64(V), _f64(q), _f64(P)
+    L, d = Kt.shape
+    g = q.shape[0]
+    res = PairResult()
+    res.out = np.empty((g, d))
+    res.sel = np.empty(k + W, dtype=np.int32)
+    res.dims = np.empty(r, dtype=np.int32)
+    n_sel = ctypes.c_int(0)
+    res.scores = np.empty(L)
+    kth = ctypes.c_double(0.0)
+    rc = _load().oracle_decode_pair_dims(_p(Kt), _p(V), _p(q), _p(P), L, d, g, index_dims, r, k, W,
+                                         1 if group_max else 0, scale, _p(res.out), _p(res.sel, _I32),
+                                         ctypes.byref(n_sel), _p(res.scores), ctypes.byref(kth),
+                                         _p(res.dims, _I32))
+    if rc != 0:
+        raise ValueError("oracle_decode_pair_dims rejected its arguments")
+    res.n_sel = n_sel.value
+    res.kth = kth.value
+    res.weight = magnitude_dims(q, P, r, index_dims, group_max)[1]
     return res
 
 

@@ -543,6 +543,149 @@ int oracle_magnitude_slabs(const double* q, const double* P, int d, int g, int i
     return 0;
 }
 
+/* ------------------------------------------------------------------------- */
+/* Magnitude-based choice of single scoring dimensions for one (sequence,    */
+/* kv head) pair: AQUA page, Algorithm 1 in prose (at each decode step the   */
+/* indices of the top dimensions by magnitude of the projected query are     */
+/* found, and the approximate scores use only those dimensions of the query  */
+/* and of the key cache) and its appendix on complexity, steps 2-4 (the      */
+/* element-wise absolute value of q_hat, a selection of the top indices,     */
+/* the slice of those columns of the key cache, the product with the sliced  */
+/* query).                                                                   */
+/*                                                                           */
+/* The page scores one query; for a group of g query heads that share a kv   */
+/* head (the pages are silent on grouped-query attention) this oracle reads  */
+/* the magnitude of dimension c as                                           */
+/*   SUM: w[c] = |u[c]|, u = sum_j q_hat_j  (the query that ranks the tokens) */
+/*   MAX: w[c] = sqrt(sum_j q_hat_j[c]^2)  (every head scores alone)         */
+/* so that for g = 1 both are |q_hat[c]|. The r dimensions of largest w      */
+/* among the first index_dims are kept, ties to the lower dimension, and are */
+/* listed in ascending order.                                                */
+/*                                                                           */
+/* q [g][d] unrotated queries; P [d][d]; dims [r] (written, ascending);      */
+/* weight [index_dims] (nullable): w. Returns 0, or -1 on bad sizes.         */
+/* ------------------------------------------------------------------------- */
+int oracle_magnitude_dims(const double* q, const double* P, int d, int g, int index_dims, int r,
+                          int group_max, int32_t* dims, double* weight)
+{
+    if (d < 1 || g < 1 || index_dims < 1 || index_dims > d || r < 1 || r > index_dims)
+        return -1;
+    double* qhat = (double*)malloc(sizeof(double) * (size_t)g * d);
+    double* w = (double*)malloc(sizeof(double) * (size_t)index_dims);
+    /* appendix step 1: project the query */
+    oracle_rotate(q, P, g, d, qhat);
+    /* appendix step 2: element-wise magnitude */
+    for (int c = 0; c < index_dims; ++c) {
+        double acc = 0.0;
+        if (group_max) {
+            for (int j = 0; j < g; ++j)
+                acc += qhat[j * d + c] * qhat[j * d + c];
+            w[c] = sqrt(acc);
+        } else {
+            for (int j = 0; j < g; ++j)
+                acc += qhat[j * d + c];
+            w[c] = fabs(acc);
+        }
+    }
+    /* appendix step 2: the indices of the r largest magnitudes. Dimension c */
+    /* is kept when fewer than r dimensions beat it (a larger magnitude, or  */
+    /* an equal one at a lower index).                                       */
+    int n = 0;
+    for (int c = 0; c < index_dims; ++c) {
+        int beaten_by = 0;
+        for (int o = 0; o < index_dims; ++o)
+            if (w[o] > w[c] || (w[o] == w[c] && o < c))
+                ++beaten_by;
+        if (beaten_by < r)
+            dims[n++] = c;
+    }
+    if (weight)
+        for (int c = 0; c < index_dims; ++c)
+            weight[c] = w[c];
+    free(w);
+    free(qhat);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* One decode step whose approximate scores use the dimensions that          */
+/* oracle_magnitude_dims chooses (AQUA page, appendix on complexity, steps   */
+/* 3-4: the key cache sliced to those columns, times the sliced query):      */
+/*   s_t = reduce_j sum_{c in dims, ascending} q_hat_j[c] * K~[t][c].        */
+/* Steps 2, 4 and 5 are those of oracle_decode_pair. index_dims bounds the   */
+/* dimensions to choose from; dims_out [r] (nullable) receives the choice.   */
+/* Other arguments and the return value as for oracle_decode_pair.           */
+/* ------------------------------------------------------------------------- */
+int oracle_decode_pair_dims(const double* Kt, const double* V, const double* q, const double* P,
+                            int L, int d, int g, int index_dims, int r, int k, int W, int group_max,
+                            double scale, double* out, int32_t* sel, int* n_sel, double* scores,
+                            double* kth, int32_t* dims_out)
+{
+    if (k < 0 || W < 0 || (k == 0 && W == 0) || r < 1 || r > index_dims || index_dims > d || L < 0)
+        return -1;
+    if (scale == 0.0)
+        scale = 1.0 / sqrt((double)d);
+
+    /* Steps 1-2 of the appendix: the query in the PCA basis and the r       */
+    /* dimensions of largest magnitude.                                      */
+    int32_t* dims = (int32_t*)malloc(sizeof(int32_t) * (size_t)r);
+    if (oracle_magnitude_dims(q, P, d, g, index_dims, r, group_max, dims, NULL) != 0) {
+        free(dims);
+        return -1;
+    }
+    double* qhat = (double*)malloc(sizeof(double) * (size_t)g * d);
+    oracle_rotate(q, P, g, d, qhat);
+
+    /* Candidates are the tokens outside the forced recent window.           */
+    int w_eff = W < L ? W : L;
+    int ncand = L - w_eff;
+
+    /* Steps 3-4 of the appendix: scores from the chosen columns only.       */
+    scored_token* cand = (scored_token*)malloc(sizeof(scored_token) * (size_t)(ncand > 0 ? ncand : 1));
+    for (int t = 0; t < ncand; ++t) {
+        const double* kt = Kt + (int64_t)t * d;
+        double s = group_max ? -INFINITY : 0.0;
+        for (int j = 0; j < g; ++j) {
+            double sj = 0.0;
+            for (int i = 0; i < r; ++i)
+                sj += qhat[j * d + dims[i]] * kt[dims[i]];
+            if (group_max)
+                s = sj > s ? sj : s;
+            else
+                s += sj;
+        }
+        cand[t].s = s;
+        cand[t].t = t;
+    }
+    if (scores) {
+        for (int t = 0; t < L; ++t)
+            scores[t] = NAN;
+        for (int t = 0; t < ncand; ++t)
+            scores[t] = cand[t].s;
+    }
+
+    /* Keep the k best candidates and the recent window, then attend exactly */
+    /* over the full head dimension (equations (3)-(5)).                     */
+    int32_t* T = (int32_t*)malloc(sizeof(int32_t) * (size_t)(ncand + w_eff + 1));
+    int nT = keep_top_k_and_window(cand, ncand, k, w_eff, T, kth);
+    oracle_attend_set(Kt, V, qhat, T, nT, d, g, scale, out, NULL);
+
+    if (sel) {
+        for (int i = 0; i < k + W; ++i)
+            sel[i] = i < nT ? T[i] : -1;
+    }
+    if (n_sel)
+        *n_sel = nT;
+    if (dims_out)
+        for (int i = 0; i < r; ++i)
+            dims_out[i] = dims[i];
+    free(T);
+    free(cand);
+    free(qhat);
+    free(dims);
+    return 0;
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

@@ -42,6 +42,17 @@ MUTATIONS = {
                                       "if (e[o] > e[s] || (e[o] == e[s] && o > s))"),
     "slab off by one dim": ("for (int c = 16 * s; c < 16 * s + 16; ++c) {",
                             "for (int c = 16 * s + 1; c < 16 * s + 16; ++c) {"),
+    "dims: lightest kept": ("if (w[o] > w[c] || (w[o] == w[c] && o < c))",
+                            "if (w[o] < w[c] || (w[o] == w[c] && o < c))"),
+    "dim ties to the higher index": ("if (w[o] > w[c] || (w[o] == w[c] && o < c))",
+                                     "if (w[o] > w[c] || (w[o] == w[c] && o > c))"),
+    "dim magnitude signed": ("w[c] = fabs(acc);", "w[c] = acc;"),
+    "dim magnitude of the first head only": ("for (int j = 0; j < g; ++j)\n                acc += qhat[j * d + c];",
+                                             "for (int j = 0; j < 1; ++j)\n                acc += qhat[j * d + c];"),
+    "dims decode scores the leading dims": ("sj += qhat[j * d + dims[i]] * kt[dims[i]];",
+                                            "sj += qhat[j * d + i] * kt[i];"),
+    "dims decode drops the last chosen dim": ("for (int i = 0; i < r; ++i)\n                sj += qhat",
+                                              "for (int i = 0; i < r - 1; ++i)\n                sj += qhat"),
     "asym query factor is P": ("acc += q[j * d + a] * Aq[(int64_t)a * ri + c];",
                                "acc += q[j * d + a] * P[(int64_t)a * d + c];"),
     "asym index not rounded": ("out[i * ri + c] = dtype == 1 ? oracle_round_bf16(acc) : (double)(float)acc;",
@@ -73,6 +84,13 @@ PIN_FUNCS = [
     pins.test_magnitude_slabs_energy_is_conserved,
     pins.test_magnitude_slabs_maximise_the_kept_energy,
     pins.test_magnitude_slabs_reduce_and_ties,
+    pins.test_magnitude_dims_known_answer,
+    pins.test_magnitude_dims_follow_the_basis,
+    pins.test_magnitude_dims_energy_is_conserved,
+    pins.test_magnitude_dims_maximise_the_kept_energy,
+    pins.test_magnitude_dims_reduce_and_ties,
+    pins.test_dims_decode_scores_are_exact_on_the_query_support,
+    pins.test_dims_decode_reduces_to_leading_and_to_slabs,
     pins.test_index_keys_with_pca_factor_is_the_appended_slice,
     pins.test_asym_decode_with_symmetric_factors_is_the_leading_decode,
     pins.test_asym_decode_brute_force,

@@ -448,10 +448,13 @@ def load_golden(name):
 @pytest.mark.parametrize("name", sorted(n for n in os.listdir(GOLDEN) if n.endswith(".json")))
 def test_golden_fixture(name):
     fx = load_golden(name)
-    res = oracle.decode_pair(np.array(fx["Kt"], float), np.array(fx["V"], float),
-                             np.array(fx["q"], float), np.array(fx["P"], float),
-                             r=fx["r"], k=fx["k"], W=fx["W"],
-                             group_max=fx.get("group_max", False), scale=fx.get("scale", 0.0))
+    args = (np.array(fx["Kt"], float), np.array(fx["V"], float), np.array(fx["q"], float),
+            np.array(fx["P"], float))
+    kw = dict(W=fx["W"], group_max=fx.get("group_max", False), scale=fx.get("scale", 0.0))
+    if fx.get("scorer") == "magnitude_dims":
+        res = oracle.decode_pair_dims(*args, fx["r"], fx["k"], fx["index_dims"], **kw)
+    else:
+        res = oracle.decode_pair(*args, r=fx["r"], k=fx["k"], **kw)
     np.testing.assert_array_equal(res.sel[:res.n_sel], fx["expect_selected"])
     if "expect_out" in fx:
         np.testing.assert_allclose(res.out, np.array(fx["expect_out"], float),
@@ -621,6 +624,144 @@ def test_magnitude_decode_reduces_to_leading_when_slabs_are_leading():
     a = oracle.decode_pair_magnitude(Kt, V, q, np.eye(d), 16, 30, 64)
     b = oracle.decode_pair(Kt, V, q, np.eye(d), 16, 30)
     assert a.slabs.tolist() == [0] and a.sel.tolist() == b.sel.tolist()
+
+
+# ---------------------------------------------------------------------------
+# Magnitude-based choice of single scoring dims (AQUA page, Algorithm 1 in
+# prose; appendix on complexity, steps 2-4: the element-wise magnitude of
+# q_hat, the indices of its largest entries, the key cache sliced to those
+# columns times the sliced query)
+# ---------------------------------------------------------------------------
+
+def test_magnitude_dims_known_answer():
+    """P = I: q_hat = q, so the chosen dims are those of the largest |q| by
+    hand, listed in ascending order; only the first index_dims compete."""
+    d = 16
+    q = np.array([[0.1, -5.0, 0.3, 2.0, 0.0, -0.7, 4.0, 0.2, -3.0, 0.05, 1.0, 0.6, -0.4, 0.01, 2.5, -0.9]])
+    dims, w = oracle.magnitude_dims(q, np.eye(d), 4, 16)
+    assert dims.tolist() == [1, 6, 8, 14]
+    np.testing.assert_array_equal(w, np.abs(q[0]))
+    dims, w = oracle.magnitude_dims(q, np.eye(d), 3, 8)
+    assert dims.tolist() == [1, 3, 6] and w.shape == (8,)
+
+
+def test_magnitude_dims_follow_the_basis():
+    """With a permutation matrix as P, q_hat is q with its columns moved, and
+    the dims that receive the large entries are chosen."""
+    d = 32
+    q = np.zeros((1, d))
+    q[0, 5] = 4.0       # moved to column 20
+    q[0, 20] = -3.0     # moved to column 3
+    q[0, 9] = 1.0       # moved to column 30
+    P = np.zeros((d, d))
+    target = {5: 20, 20: 3, 9: 30}
+    rest = iter([c for c in range(d) if c not in target.values()])
+    for i in range(d):
+        P[i, target[i] if i in target else next(rest)] = 1.0
+    assert oracle.magnitude_dims(q, P, 1, d)[0].tolist() == [20]
+    assert oracle.magnitude_dims(q, P, 2, d)[0].tolist() == [3, 20]
+    assert oracle.magnitude_dims(q, P, 3, d)[0].tolist() == [3, 20, 30]
+
+
+def test_magnitude_dims_energy_is_conserved():
+    """With index_dims = d and an orthonormal P, the squared magnitudes sum to
+    the squared norm of the summed query (SUM) or to the heads' summed squared
+    norms (MAX), whatever P is (Parseval)."""
+    d, g = 64, 4
+    rng = np.random.default_rng(13)
+    q = rng.standard_normal((g, d))
+    for seed in (3, 4):
+        P = orthonormal(d, seed)
+        w_sum = oracle.magnitude_dims(q, P, 8, d, group_max=False)[1]
+        w_max = oracle.magnitude_dims(q, P, 8, d, group_max=True)[1]
+        assert math.isclose(float(np.sum(w_sum ** 2)), float(np.sum(q.sum(axis=0) ** 2)), rel_tol=1e-12)
+        assert math.isclose(float(np.sum(w_max ** 2)), float(np.sum(q ** 2)), rel_tol=1e-12)
+
+
+def test_magnitude_dims_maximise_the_kept_energy():
+    """Brute force over every subset of r of the 16 dims: the chosen set
+    keeps the most energy of the projected query (the smallest information
+    retention loss of the AQUA page), and with distinct magnitudes it is the
+    only such set."""
+    d = 16
+    rng = np.random.default_rng(21)
+    for trial in range(6):
+        g = [1, 2, 4][trial % 3]
+        q = rng.standard_normal((g, d)) * rng.uniform(0.2, 3.0, size=d)
+        P = orthonormal(d, 200 + trial)
+        for gm in (False, True):
+            w = oracle.magnitude_dims(q, P, 1, d, group_max=gm)[1]
+            for r in (1, 3, 5, 8, 12):
+                dims = oracle.magnitude_dims(q, P, r, d, group_max=gm)[0]
+                best = max(itertools.combinations(range(d), r), key=lambda c: sum(w[list(c)] ** 2))
+                assert tuple(dims.tolist()) == best
+
+
+def test_magnitude_dims_reduce_and_ties():
+    """Two heads that cancel: the summed query is zero, every dim ties and
+    SUM keeps the lowest dims; MAX keeps the dims the heads live on. Equal
+    magnitudes go to the lower dim, whatever the sign."""
+    d = 16
+    q = np.zeros((2, d))
+    q[0, [11, 13]] = 1.0
+    q[1] = -q[0]
+    assert oracle.magnitude_dims(q, np.eye(d), 2, d, group_max=False)[0].tolist() == [0, 1]
+    assert oracle.magnitude_dims(q, np.eye(d), 2, d, group_max=True)[0].tolist() == [11, 13]
+    q = np.array([[1.0, -1.0, 1.0, -2.0] + [0.0] * 12])
+    assert oracle.magnitude_dims(q, np.eye(d), 2, d)[0].tolist() == [0, 3]
+
+
+def test_dims_decode_scores_are_exact_on_the_query_support():
+    """A rotated query that lives on r scattered dims: scoring with those dims
+    gives the full dot products, so the kept set is the brute-force top-k of
+    q_hat K~^T; the leading-dims scorer and the slab scorer miss them."""
+    d, L, k, r = 128, 300, 25, 32
+    rng = np.random.default_rng(17)
+    P = orthonormal(d, 7)
+    support = np.sort(rng.choice(d, size=r, replace=False))
+    qhat = np.zeros((1, d))
+    qhat[0, support] = rng.standard_normal(r) + np.sign(rng.standard_normal(r)) * 0.5
+    q = qhat @ P.T
+    Kt = rng.standard_normal((L, d))
+    V = rng.standard_normal((L, d))
+    res = oracle.decode_pair_dims(Kt, V, q, P, r, k, d)
+    assert res.dims.tolist() == support.tolist()
+    full = Kt @ qhat[0]
+    np.testing.assert_allclose(res.scores, full, rtol=1e-9, atol=1e-12)
+    top = sorted(np.argsort(-full, kind="stable")[:k].tolist())
+    assert res.sel[:res.n_sel].tolist() == top
+    assert oracle.decode_pair(Kt, V, q, P, r, k).sel[:k].tolist() != top
+
+
+def test_dims_decode_reduces_to_leading_and_to_slabs():
+    """All dims kept (r = index_dims), or equal magnitudes: the chosen dims are
+    the leading ones and the result is the leading-dims scorer's. A query
+    whose largest entries fill whole slabs: the single-dim choice is those
+    slabs' dims and the result is the slab scorer's."""
+    d, L = 64, 200
+    rng = np.random.default_rng(19)
+    P = orthonormal(d, 2)
+    Kt = rng.standard_normal((L, d))
+    V = rng.standard_normal((L, d))
+    q = rng.standard_normal((2, d))
+    a = oracle.decode_pair_dims(Kt, V, q, P, 48, 30, 48, W=3)
+    b = oracle.decode_pair(Kt, V, q, P, 48, 30, W=3)
+    assert a.dims.tolist() == list(range(48))
+    assert a.sel.tolist() == b.sel.tolist()
+    np.testing.assert_allclose(a.out, b.out, rtol=1e-12)
+    a = oracle.decode_pair_dims(Kt, V, np.ones((1, d)), np.eye(d), 16, 30, 64)
+    b = oracle.decode_pair(Kt, V, np.ones((1, d)), np.eye(d), 16, 30)
+    assert a.dims.tolist() == list(range(16)) and a.sel.tolist() == b.sel.tolist()
+    qhat = rng.uniform(0.01, 0.1, size=(1, d))
+    qhat[0, 16:32] = rng.uniform(1.0, 2.0, size=16) * np.sign(rng.standard_normal(16))
+    qhat[0, 48:64] = rng.uniform(1.0, 2.0, size=16)
+    q = qhat @ P.T
+    a = oracle.decode_pair_dims(Kt, V, q, P, 32, 40, 64, W=2)
+    c = oracle.decode_pair_magnitude(Kt, V, q, P, 32, 40, 64, W=2)
+    assert a.dims.tolist() == list(range(16, 32)) + list(range(48, 64))
+    assert c.slabs.tolist() == [1, 3]
+    assert a.sel.tolist() == c.sel.tolist()
+    np.testing.assert_allclose(a.out, c.out, rtol=1e-12)
 
 
 # ---------------------------------------------------------------------------
