@@ -273,6 +273,7 @@ def main():
     ks = [k.to(dev) for k, _ in kvs]
     vs = [v.to(dev) for _, v in kvs]
     out = torch.empty(spec.batch, spec.num_q_heads, spec.head_dim, device=dev)
+    ws = loki.decode_workspace(cache, batch, spec.num_q_heads, spec.k, spec.recent_window, dev)
     flush = torch.empty(64 * 2 ** 20, dtype=torch.float32, device=dev)  # 256 MB > L2
     flush_sum = torch.empty((), dtype=torch.float32, device=dev)
 
@@ -295,7 +296,7 @@ def main():
     def step(i, q=None, k=None, v=None):
         loki.loki_decode_step(cache, batch, ks[i % pool] if k is None else k, vs[i % pool] if v is None else v,
                               qs[i % pool] if q is None else q, P, spec.r, spec.k, out,
-                              recent_window=spec.recent_window, stream=stream)
+                              recent_window=spec.recent_window, workspace=ws, stream=stream)
 
     # warm-up
     for i in range(args.warmup):
@@ -349,7 +350,7 @@ def main():
         flush_l2()
         evm[i].record(stream)
         loki.loki_decode_attention(cache, batch, qs[i % pool], P, spec.r, spec.k, out,
-                                   recent_window=spec.recent_window, stream=stream)
+                                   recent_window=spec.recent_window, workspace=ws, stream=stream)
         ev1[i].record(stream)
     torch.cuda.synchronize()
     decode_ms = sum(a.elapsed_time(b) for a, b in zip(evm, ev1))
@@ -455,10 +456,11 @@ def main():
     del K_orig
     mout = torch.empty_like(out)
     scorer_ms = {}
-    for name, scorer in (("magnitude", loki.LOKI_SCORER_MAGNITUDE), ("leading", loki.LOKI_SCORER_LEADING)):
+    for name, scorer in (("magnitude", loki.LOKI_SCORER_MAGNITUDE), ("slabs", loki.LOKI_SCORER_MAGNITUDE_SLABS),
+                         ("leading", loki.LOKI_SCORER_LEADING)):
         def mag_launch(i):
             loki.loki_decode_attention_scored(mcache, batch, qs[i % pool], P, spec.r, spec.k, mout, scorer=scorer,
-                                              recent_window=spec.recent_window, stream=stream)
+                                              recent_window=spec.recent_window, workspace=ws, stream=stream)
         for i in range(3):
             mag_launch(i)
         m0 = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
@@ -479,7 +481,7 @@ def main():
 
     def asym_launch(i):
         loki.loki_decode_attention_asym(cache, batch, qs[i % pool], P, Aq, spec.r, spec.k, mout,
-                                        recent_window=spec.recent_window, stream=stream)
+                                        recent_window=spec.recent_window, workspace=ws, stream=stream)
     for i in range(3):
         asym_launch(i)
     a0 = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
@@ -529,11 +531,12 @@ def main():
                            "achieved_gbs": rot_bytes / (rot_ms / 1e3) / 1e9,
                            "tflops": 2.0 * ntok * spec.head_dim ** 2 / (rot_ms / 1e3) / 1e12,
                            "kernel": "rotate_prefill_tc_kernel<128> (tcgen05)"},
-        "magnitude_scorer": {"launch_ms": scorer_ms["magnitude"], "leading_launch_ms": scorer_ms["leading"],
-                             "index_dims": spec.head_dim,
+        "magnitude_scorer": {"launch_ms": scorer_ms["magnitude"], "slabs_launch_ms": scorer_ms["slabs"],
+                             "leading_launch_ms": scorer_ms["leading"], "index_dims": spec.head_dim,
                              "note": "loki_decode_attention_scored on a cache whose key index holds all "
-                                     f"{spec.head_dim} dims; r = {spec.r}: the r/16 slabs with the most query "
-                                     "energy against the leading r dims, median of 10 L2-flushed launches"},
+                                     f"{spec.head_dim} dims; r = {spec.r}: the r single dims of largest query "
+                                     "magnitude (AQUA), the r/16 slabs with the most query energy, and the "
+                                     "leading r dims, median of 10 L2-flushed launches each"},
         "asym_scorer": {"launch_ms": asym_ms,
                         "note": "loki_decode_attention_asym on the bench cache (index of the leading 32 dims, "
                                 "A_q = the leading 32 columns of P), median of 10 L2-flushed launches"},

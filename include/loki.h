@@ -46,7 +46,7 @@ extern "C" {
 #define LOKI_API
 #endif
 
-#define LOKI_ABI_VERSION 3
+#define LOKI_ABI_VERSION 4
 #define LOKI_BLOCK_TOKENS 16 /* tokens per paged-cache block */
 
 typedef void* loki_stream_t; /* a cudaStream_t */
@@ -76,16 +76,19 @@ typedef enum loki_group_reduce {
 
 /* Which r index dims the approximate score uses (loki_decode_attention_scored).
  * LEADING: the leading r dims, a static slice after the projection (Loki page,
- * abstract; AQUA page, related work on LoKi). MAGNITUDE: per (sequence, kv
- * head) and step, the r/16 slabs of 16 index dims with the most energy of the
- * query that ranks the tokens (AQUA page, Algorithm 1 in prose: dims picked by
- * the magnitude of the projected query; the energy kept is what the AQUA
- * page's information-retention loss measures). The pages pick single dims;
- * this library picks whole 16-dim slabs so that each block's selected dims
- * remain contiguous runs of the key index. */
+ * abstract; AQUA page, related work on LoKi).
+ * MAGNITUDE: per (sequence, kv head) and step, the r single index dims of
+ * largest magnitude of the query that ranks the tokens (AQUA page, Algorithm 1
+ * in prose and appendix on complexity, steps 2-4: the top dims of |q_hat|, the
+ * key cache sliced to those columns). Each chosen dim of a 16-token block is
+ * one 16-element run of the dim-major key index.
+ * MAGNITUDE_SLABS: a coarser variant that picks the r/16 slabs of 16
+ * consecutive index dims with the most energy of that query (whole 16-dim
+ * runs; not the pages' algorithm, kept for comparison). */
 typedef enum loki_scorer {
     LOKI_SCORER_LEADING = 0,
-    LOKI_SCORER_MAGNITUDE = 1
+    LOKI_SCORER_MAGNITUDE = 1,
+    LOKI_SCORER_MAGNITUDE_SLABS = 2
 } loki_scorer;
 
 /* Device error word bits (loki_device_error). */
@@ -98,11 +101,12 @@ typedef enum loki_scorer {
  * block), plus a low-rank key index. Physical block p of kv head h holds:
  *   keys (PCA basis)  [16 tokens][head_dim]  at element (p*Hkv + h)*16*head_dim
  *   values            [16 tokens][head_dim]  at element (p*Hkv + h)*16*head_dim
- *   key index         [index_dims/16 slabs][16 tokens][16 dims]
- *                                            at element (p*Hkv + h)*16*index_dims
- * The key index repeats the leading index_dims rotated dims of every key. Its
- * slab layout makes the leading r <= index_dims dims of a block one
- * contiguous run of r*16 elements, which is what rank-r scoring streams; the
+ *   key index         [index_dims][16 tokens]  at element (p*Hkv + h)*16*index_dims
+ * The key index repeats the leading index_dims rotated dims of every key,
+ * dim-major: element (c, t) of a block is at c*16 + t. The leading r <=
+ * index_dims dims of a block are one contiguous run of r*16 elements, which is
+ * what rank-r scoring streams, and any single dim of a block is one run of 16
+ * elements (32 bytes in bf16), which is what the magnitude scorer reads; the
  * key rows stay whole (one contiguous row per token) for the exact attention
  * over the kept tokens. The index costs index_dims/head_dim of the key cache
  * (12.5% of keys + values for index_dims = 32, head_dim = 128). */
@@ -281,15 +285,20 @@ LOKI_API loki_status loki_decode_attention(const loki_cache* cache, const loki_b
                                   loki_stream_t stream);
 
 /* loki_decode_attention with a choice of scorer; LOKI_SCORER_LEADING gives
- * the same results as loki_decode_attention. With LOKI_SCORER_MAGNITUDE,
- * step 2 scores with the selected slabs instead of the leading r dims:
- *   energy e_s = sum_{c in slab s} u[c]^2 for each slab s < index_dims/16,
- *     u = sum_{j in group(h)} q_hat_j (SUM), or
- *     e_s = sum_{j in group(h)} sum_{c in slab s} q_hat_j[c]^2 (MAX)   (fp32);
- *   the r/16 slabs of largest e_s (ties to the lower slab) form the set S and
- *   s_t = reduce_j sum_{s in S, ascending} q_hat_j[slab s] . K~[t, slab s].
- * Steps 1, 3 and 4 are unchanged. Arguments as for loki_decode_attention;
- * an unknown scorer is LOKI_ERR_INVALID_ARG. */
+ * the same results as loki_decode_attention. Otherwise step 2 scores with a
+ * set S of r index dims chosen per (sequence, kv head) and step among the
+ * first index_dims (fp32, with u = sum_{j in group(h)} q_hat_j):
+ *   LOKI_SCORER_MAGNITUDE (AQUA page, Algorithm 1 in prose; appendix on
+ *     complexity, steps 2-4): the r dims c of largest |u[c]| (SUM) or of
+ *     largest sum_j q_hat_j[c]^2 (MAX), ties to the lower dim;
+ *   LOKI_SCORER_MAGNITUDE_SLABS: the r/16 slabs s (16 consecutive dims) of
+ *     largest sum_{c in s} u[c]^2 (SUM) or sum_j sum_{c in s} q_hat_j[c]^2
+ *     (MAX), ties to the lower slab;
+ * and s_t = reduce_j sum_{c in S, ascending} q_hat_j[c] K~[t, c]. Steps 1, 3
+ * and 4 are unchanged. The bytes read per candidate token are the same r
+ * index elements as the leading scorer's; the index must hold the dims to
+ * choose from. Arguments as for loki_decode_attention; an unknown scorer is
+ * LOKI_ERR_INVALID_ARG. */
 LOKI_API loki_status loki_decode_attention_scored(const loki_cache* cache, const loki_batch* batch,
                                          const void* q, int32_t num_q_heads, const float* P,
                                          int32_t r, int32_t k, const int32_t* k_per_seq,

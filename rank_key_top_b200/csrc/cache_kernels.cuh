@@ -57,7 +57,11 @@ __global__ void __launch_bounds__(256) prefill_kernel(const PrefillParams p) {
         const uint4 vv = *reinterpret_cast<const uint4*>(vs + tok * D + dim);
         *reinterpret_cast<uint4*>(kd + row_offset_in_page(tok, dim, D)) = kv;
         *reinterpret_cast<uint4*>(vd + row_offset_in_page(tok, dim, D)) = vv;
-        if (dim < p.index_dims) *reinterpret_cast<uint4*>(xd + index_offset_in_page(tok, dim)) = kv;
+        if (dim < p.index_dims) {  // dim-major index: one element per dim
+            const T* e = reinterpret_cast<const T*>(&kv);
+#pragma unroll
+            for (int i = 0; i < VEC; ++i) xd[index_offset_in_page(tok, dim + i)] = e[i];
+        }
     }
 }
 

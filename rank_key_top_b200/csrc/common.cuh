@@ -24,9 +24,10 @@ __device__ __forceinline__ void flag_error(uint32_t bits) { atomicOr(&g_device_e
 // Paged cache layout. Block p of kv head h starts at element
 // (p * Hkv + h) * 16 * D in the key and value caches, and at
 // (p * Hkv + h) * 16 * I in the key index (I = index dims).
-//   keys, values: [16 tokens][D]                 (one contiguous row per token)
-//   key index:    [I/16 slabs][16 tokens][16 dims] (the leading r dims of all
-//                 16 tokens are one contiguous run of r*16 elements)
+//   keys, values: [16 tokens][D]     (one contiguous row per token)
+//   key index:    [I dims][16 tokens] (dim-major: one dim of the block's 16
+//                 tokens is one contiguous run of 16 elements, and the
+//                 leading r dims are one contiguous run of r*16 elements)
 // ---------------------------------------------------------------------------
 __host__ __device__ __forceinline__ int64_t page_offset(int64_t block, int h, int Hkv, int D) {
     return (block * Hkv + h) * (int64_t)(kBlockTokens * D);
@@ -35,7 +36,7 @@ __host__ __device__ __forceinline__ int row_offset_in_page(int token, int dim, i
     return token * D + dim;
 }
 __host__ __device__ __forceinline__ int index_offset_in_page(int token, int dim) {
-    return (dim / kSlabDims) * (kBlockTokens * kSlabDims) + token * kSlabDims + (dim % kSlabDims);
+    return dim * kBlockTokens + token;
 }
 
 // ---------------------------------------------------------------------------
@@ -135,6 +136,37 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// mbarriers in shared memory: init, and a bounded wait for a phase.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+// Waits for phase `parity` of `bar`, polling at most kWaitLimit times; on
+// giving up it sets LOKI_DEVERR_TIMEOUT and returns false.
+constexpr uint32_t kWaitLimit = 1u << 24;
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+        if (ok) return true;
+    }
+    flag_error(LOKI_DEVERR_TIMEOUT);
+    return false;
+}
+// One arrival on `bar` once every cp.async this thread issued before has
+// landed (the arrival counts toward the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // ---------------------------------------------------------------------------

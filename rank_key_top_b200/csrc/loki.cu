@@ -47,8 +47,14 @@ loki_status check_batch(const loki_batch* bt) {
     return LOKI_OK;
 }
 
+// Launch errors of this call only: a pending error left by earlier, unrelated
+// work is cleared when a call starts (clear_pending_error), and the error of
+// a failed launch is read and cleared (launch_status), so that it is reported
+// once, by the call that caused it.
+void clear_pending_error() { cudaGetLastError(); }
+
 loki_status launch_status() {
-    return cudaPeekAtLastError() == cudaSuccess ? LOKI_OK : LOKI_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? LOKI_OK : LOKI_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------------------
@@ -104,6 +110,7 @@ loki_status launch_append(const loki_cache* cache, const loki_batch* batch, cons
     p.max_seq_len = batch->max_seq_len;
     const int grid = batch->batch * cache->num_kv_heads;
     const int D = cache->head_dim;
+    clear_pending_error();
     if (cache->dtype == LOKI_BF16) {
         if (D == 64) append_kernel<__nv_bfloat16, 64><<<grid, 256, 0, s>>>(p);
         else append_kernel<__nv_bfloat16, 128><<<grid, 256, 0, s>>>(p);
@@ -156,6 +163,7 @@ loki_status launch_decode(const loki_cache* cache, const loki_batch* batch, cons
     const int G = num_q_heads / Hkv;
     const int pairs = batch->batch * Hkv;
     const DeviceInfo di = device_info();
+    clear_pending_error();
     SparseParams p;
     p.k_cache = cache->k_cache;
     p.v_cache = cache->v_cache;
@@ -253,6 +261,7 @@ loki_status loki_prefill_cache(const loki_cache* cache, const loki_batch* batch,
     dim3 grid(nblk, batch->batch * cache->num_kv_heads);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int D = cache->head_dim;
+    clear_pending_error();
     if (cache->dtype == LOKI_BF16) {
         if (D == 64) prefill_kernel<__nv_bfloat16, 64><<<grid, 256, 0, s>>>(p);
         else prefill_kernel<__nv_bfloat16, 128><<<grid, 256, 0, s>>>(p);
@@ -299,17 +308,8 @@ loki_status loki_prefill_rotate(const loki_cache* cache, const loki_batch* batch
         p.tiles_per_cta = (int)std::max<int64_t>(1, ((int64_t)tiles * pairs + want - 1) / want);
         const dim3 grid((tiles + p.tiles_per_cta - 1) / p.tiles_per_cta, pairs);
         auto launch = [&](auto kern, int smem) {
-            static std::mutex mu;
-            static std::map<const void*, cudaError_t> done;
-            {
-                std::lock_guard<std::mutex> lk(mu);
-                auto it = done.find((const void*)kern);
-                if (it == done.end())
-                    it = done.emplace((const void*)kern,
-                                      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
-                             .first;
-                if (it->second != cudaSuccess) return LOKI_ERR_CUDA;
-            }
+            if (ensure_smem_attr((const void*)kern, smem) != cudaSuccess) return LOKI_ERR_CUDA;
+            clear_pending_error();
             kern<<<grid, kRotThreads, smem, s>>>(p);
             return launch_status();
         };
@@ -317,6 +317,7 @@ loki_status loki_prefill_rotate(const loki_cache* cache, const loki_batch* batch
         return launch(rotate_prefill_tc_kernel<128>, rotate_smem_bytes<128>());
     }
     const dim3 grid((batch->max_seq_len + kBlockTokens - 1) / kBlockTokens, pairs);
+    clear_pending_error();
     if (D == 64) rotate_prefill_f32_kernel<64><<<grid, 256, 0, s>>>(p);
     else rotate_prefill_f32_kernel<128><<<grid, 256, 0, s>>>(p);
     return launch_status();
@@ -338,17 +339,8 @@ loki_status loki_pca_basis(const void* keys, int32_t num_heads, int64_t n, int32
     p.n = n;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     auto launch = [&](auto kern, int smem) {
-        static std::mutex mu;
-        static std::map<const void*, cudaError_t> done;
-        {
-            std::lock_guard<std::mutex> lk(mu);
-            auto it = done.find((const void*)kern);
-            if (it == done.end())
-                it = done.emplace((const void*)kern,
-                                  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
-                         .first;
-            if (it->second != cudaSuccess) return LOKI_ERR_CUDA;
-        }
+        if (ensure_smem_attr((const void*)kern, smem) != cudaSuccess) return LOKI_ERR_CUDA;
+        clear_pending_error();
         kern<<<num_heads, kPcaThreads, smem, s>>>(p);
         return launch_status();
     };
@@ -400,8 +392,8 @@ loki_status loki_index_keys(const loki_cache* cache, const loki_batch* batch, co
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int D = cache->head_dim;
     auto launch = [&](auto kern, int smem) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-            return LOKI_ERR_CUDA;
+        if (ensure_smem_attr((const void*)kern, smem) != cudaSuccess) return LOKI_ERR_CUDA;
+        clear_pending_error();
         kern<<<grid, 256, smem, s>>>(p);
         return launch_status();
     };
@@ -452,13 +444,18 @@ loki_status loki_decode_attention_scored(const loki_cache* cache, const loki_bat
                                          size_t workspace_bytes, loki_stream_t stream) {
     (void)workspace;
     (void)workspace_bytes;
-    if (scorer != LOKI_SCORER_LEADING && scorer != LOKI_SCORER_MAGNITUDE) return LOKI_ERR_INVALID_ARG;
+    int sc;
+    switch (scorer) {
+        case LOKI_SCORER_LEADING: sc = kScoreLeading; break;
+        case LOKI_SCORER_MAGNITUDE: sc = kScoreMagnitude; break;
+        case LOKI_SCORER_MAGNITUDE_SLABS: sc = kScoreSlabs; break;
+        default: return LOKI_ERR_INVALID_ARG;
+    }
     loki_status st = check_decode(cache, batch, q, num_q_heads, P, r, k, recent_window, group_reduce, scale, out);
     if (st != LOKI_OK || batch->batch == 0) return st;
     if ((st = check_decode_fits(cache, batch, num_q_heads, r)) != LOKI_OK) return st;
     return launch_decode(cache, batch, q, num_q_heads, P, r, k, k_per_seq, recent_window, group_reduce, scale, out,
-                         selected_idx, reinterpret_cast<cudaStream_t>(stream), false,
-                         scorer == LOKI_SCORER_MAGNITUDE ? kScoreMagnitude : kScoreLeading);
+                         selected_idx, reinterpret_cast<cudaStream_t>(stream), false, sc);
 }
 
 loki_status loki_decode_attention_asym(const loki_cache* cache, const loki_batch* batch, const void* q,
@@ -506,12 +503,8 @@ struct DenseLaunch {
     static loki_status run(DenseParams p, int batch, cudaStream_t s) {
         using Geom = DenseGeom<T, D, G>;
         auto split_kern = dense_split_kernel<T, D, G>;
-        static std::once_flag once;
-        static cudaError_t attr_err = cudaSuccess;
-        std::call_once(once, [&] {
-            attr_err = cudaFuncSetAttribute(split_kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geom::SMEM_BYTES);
-        });
-        if (attr_err != cudaSuccess) return LOKI_ERR_CUDA;
+        if (ensure_smem_attr((const void*)split_kern, Geom::SMEM_BYTES) != cudaSuccess) return LOKI_ERR_CUDA;
+        clear_pending_error();
         const int pairs = batch * p.Hkv;
         rotate_query_kernel<T, D, G><<<pairs, 256, 0, s>>>(p);
         split_kern<<<dim3(p.splits, pairs), kDenseThreads, Geom::SMEM_BYTES, s>>>(p);

@@ -5,11 +5,13 @@
 // lays them out.
 //
 // bf16 caches: a real GEMM per kv head, [tokens x D] x [D x D], on the 5th
-// generation tensor cores. One CTA (4 warps) keeps P_h in shared memory as
+// generation tensor cores. One CTA (8 warps) keeps P_h in shared memory as
 // two bf16 terms (P = P_hi + P_lo, the second term holding the remainder of
 // the first), streams 128-token tiles of K in with cp.async, and issues
 // tcgen05.mma (M = 128 tokens, N = D, K = D, both operands K-major with the
-// 128-byte swizzle) into a D x 128 fp32 accumulator in tensor memory: the
+// 128-byte swizzle) into a 128-lane x D-column fp32 accumulator in tensor
+// memory (lane = token, column = output dim; warps w and w + 4 read the two
+// column halves of the same 32 lanes): the
 // products of bf16 keys with each term are exact and the sum is accumulated
 // in fp32, so the result carries about 16 significant bits of P before it is
 // rounded to bf16. The epilogue reads the accumulator with tcgen05.ld (warps w
@@ -83,29 +85,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "memory");
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-// Waits for phase `parity` of `bar`, polling at most kRotWaitLimit times; on
-// giving up it sets LOKI_DEVERR_TIMEOUT and returns false.
-constexpr uint32_t kRotWaitLimit = 1u << 24;
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kRotWaitLimit; ++i) {
-        uint32_t ok;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(ok)
-            : "r"(smem_u32(bar)), "r"(parity)
-            : "memory");
-        if (ok) return true;
-    }
-    flag_error(LOKI_DEVERR_TIMEOUT);
-    return false;
-}
 
 // Shared-memory matrix descriptor of a K-major operand with the 128-byte
 // swizzle: rows of 128 bytes (64 bf16 of K), 8-row groups 1024 bytes apart;
@@ -318,9 +297,12 @@ __global__ void __launch_bounds__(kRotThreads) rotate_prefill_tc_kernel(const Ro
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const int dim = c0 + 8 * q;
-                        if (dim < p.index_dims)
-                            *reinterpret_cast<uint4*>(xpage + index_offset_in_page(t & 15, dim)) =
-                                make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+                        if (dim < p.index_dims) {  // dim-major index: one element per dim
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                xpage[index_offset_in_page(t & 15, dim + e)] =
+                                    __ushort_as_bfloat16((unsigned short)(w[4 * q + e / 2] >> (16 * (e & 1))));
+                        }
                     }
                 }
             }

@@ -9,14 +9,16 @@
 //  2. rank-r scoring (AQUA page, related work on LoKi: slice the leading
 //     dimensions after projection; Loki page, abstract: scores in the
 //     low-dimensional space). Each warp owns a private ring of S slots; a
-//     slot receives the leading r index dims of one 16-token block, one
-//     contiguous run of r*16 elements, as 16-byte cp.async pieces from all
-//     lanes; with r <= 32 a warp loads two blocks before scoring either.
+//     slot receives r index dims of one 16-token block (dim-major: one row
+//     of 16 tokens per dim; the leading r dims are one contiguous run of
+//     r*16 elements) as 16-byte cp.async pieces from all lanes; with r <= 32
+//     a warp loads two blocks before scoring either.
 //     Scores become order-preserving uint32 keys in shared memory; the
 //     histogram of their top 11 bits is built on the fly with shared
-//     atomics. Two other scorers share the kernel (template argument SC, at
-//     the kernel's declaration): the index slabs with the most query energy,
-//     and asymmetric factors (q A_q against an index of k A_k).
+//     atomics. Three other scorers share the kernel (template argument SC,
+//     at the kernel's declaration): the single index dims of largest query
+//     magnitude, the index slabs with the most query energy, and asymmetric
+//     factors (q A_q against an index of k A_k).
 //  3. top-k (Loki page, abstract: rank and select tokens): an exact radix
 //     select with digits of 11, 11 and 10 bits. After each digit the CTAs of
 //     the cluster sum their histograms through distributed shared memory, so
@@ -170,20 +172,29 @@ __device__ __noinline__ int2 radix_boundary(const uint32_t* hcur, int nbins, int
 
 // Scorers (template argument SC):
 //  kScoreLeading: q_hat_j against the leading r index dims (Loki).
-//  kScoreMagnitude: the r / 16 index slabs (16 dims each) that hold the most
-//    energy of the group's rotated query (AQUA page, Algorithm 1 in prose: the
-//    dims are picked by the magnitude of q_hat per decode step; the retained
-//    energy is what its information-retention loss measures). A slab is the
-//    unit of choice, so that a block's selected dims stay whole 512-byte
-//    (bf16) runs of the index.
+//  kScoreMagnitude: per (sequence, kv head) and step, the r single index dims
+//    of largest magnitude of the query that ranks the tokens (AQUA page,
+//    Algorithm 1 in prose and appendix on complexity, steps 2-4): |sum_j
+//    q_hat_j[c]| (SUM) or sum_j q_hat_j[c]^2 (MAX), ties to the lower dim. A
+//    chosen dim of a block is one 16-element row of the dim-major index.
+//  kScoreSlabs: the r / 16 index slabs (16 consecutive dims) that hold the
+//    most energy of that query, ties to the lower slab (a coarser variant).
 //  kScoreAsym: q_j A_q[h] against the leading r dims of an index that holds
 //    k A_k (SAKI page, abstract: asymmetric query and key factors of the
 //    score operator); the exact attention still uses q_hat = q P.
-constexpr int kScoreLeading = 0, kScoreMagnitude = 1, kScoreAsym = 2;
+constexpr int kScoreLeading = 0, kScoreMagnitude = 1, kScoreSlabs = 2, kScoreAsym = 3;
+constexpr int kSelDims = 128;  // misc words 128 .. 255: the chosen index dims in slot order
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3,
+                                                  const void* row_ptr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(smem_u32(row_ptr)));
+}
 
 template <typename T, int D, int G, int SC>
 __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const SparseParams p) {
-    constexpr bool MAG = SC == kScoreMagnitude;
+    constexpr bool MAG = SC == kScoreMagnitude || SC == kScoreSlabs;  // dims chosen per step
     constexpr bool ASYM = SC == kScoreAsym;
     using Geom = SparseGeom<T, D, G>;
     using Core = typename Geom::Core;
@@ -219,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     int32_t* misc = reinterpret_cast<int32_t*>(smem + p.off_misc);
     // misc: [0] boundary digit, [1] count above it, [8..39] suffix-sum scratch,
     //       [40..55] warp kept counts, [56..71] warp equal counts, [72] list length,
-    //       [96..103] selected index slabs, [104..111] slab energies (MAG)
+    //       [104..111] slab energies (slab scorer), [128..255] chosen dims (MAG)
 
     // ---- sequence geometry ----
     // CTA crank owns the fixed token range [crank * cta_tokens, + cta_tokens)
@@ -313,14 +324,17 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
             const int pb = entry(it);
             const unsigned char* src = xbytes + page_offset(pb, h, p.Hkv, p.index_dims) * (int64_t)sizeof(T);
             unsigned char* dst = wring + (it & smask) * p.slot_bytes;
-            if constexpr (MAG) {  // slot slab i <- index slab misc[96 + i] of the page
-                constexpr int SLAB = kBlockTokens * kSlabDims * (int)sizeof(T);
-                for (int o = lane * 16; o < p.slot_bytes; o += 32 * 16) {
-                    const int i = o / SLAB;
-                    cp_async16(dst + o, src + misc[96 + i] * SLAB + (o - i * SLAB), true);
-                }
-            } else {
-                for (int o = lane * 16; o < p.slot_bytes; o += 32 * 16) cp_async16(dst + o, src + o, true);
+            // dim row i of the slot <- index dim i (or the i-th chosen dim)
+            // of the block's 16 tokens; bf16 rows swap their two 16-byte
+            // halves on rows 4..7 mod 8, so that ldmatrix.trans is free of
+            // bank conflicts
+            constexpr int PPR = (int)sizeof(T);  // 16-byte pieces of one dim row
+            for (int pc = lane; pc < p.r * PPR; pc += 32) {
+                const int row = pc / PPR, part = pc - row * PPR;
+                const int dim = MAG ? misc[kSelDims + row] : row;
+                const int dpart = sizeof(T) == 2 ? (part ^ ((row >> 2) & 1)) : part;
+                cp_async16(dst + row * 16 * (int)sizeof(T) + dpart * 16, src + dim * 16 * (int)sizeof(T) + part * 16,
+                           true);
             }
         }
         cp_async_commit();
@@ -418,7 +432,41 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
             }
         }
         __syncthreads();
-        if constexpr (MAG) {
+        if constexpr (SC == kScoreMagnitude) {
+            // the r dims of largest magnitude among the first index_dims:
+            // |summed query| (SUM) or the heads' summed squares (MAX), ties to
+            // the lower dim, listed in ascending order
+            float* w = reinterpret_cast<float*>(smem + p.off_keys);  // the keys region is free until scoring
+            const int I = p.index_dims;
+            if (tid < I) {
+                float x = 0.f;
+                if (!p.group_max) {
+                    x = fabsf(qs[tid]);
+                } else {
+                    for (int j = 0; j < G; ++j) x = fmaf(qhat[j * D + tid], qhat[j * D + tid], x);
+                }
+                w[tid] = x;
+            }
+            __syncthreads();
+            bool chosen = false;
+            if (tid < I) {
+                const float x = w[tid];
+                int rank = 0;
+                for (int o = 0; o < I; ++o) rank += w[o] > x || (w[o] == x && o < tid);
+                chosen = rank < p.r;
+            }
+            const unsigned bal = __ballot_sync(kFull, chosen);
+            if (lane == 0 && warp < 4) misc[112 + warp] = __popc(bal);
+            __syncthreads();
+            if (chosen) {
+                int pos = __popc(bal & ((1u << lane) - 1u));
+                for (int v = 0; v < warp; ++v) pos += misc[112 + v];
+                misc[kSelDims + pos] = tid;
+            }
+            __syncthreads();
+            if (p.W == 0) griddep_wait();
+            for (int it = 0; it < S; ++it) refill(it);
+        } else if constexpr (SC == kScoreSlabs) {
             // slab energy: squared norm of the summed query over the slab (SUM),
             // or summed over the group's heads (MAX); the r / 16 largest, ties
             // to the lower slab, listed in ascending slab order
@@ -441,7 +489,10 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
                 for (int sl = 0; sl < nsl; ++sl) {
                     int rank = 0;
                     for (int o = 0; o < nsl; ++o) rank += en[o] > en[sl] || (en[o] == en[sl] && o < sl);
-                    if (rank < R16) misc[96 + n++] = sl;
+                    if (rank < R16) {
+                        for (int c = 0; c < kSlabDims; ++c) misc[kSelDims + n * kSlabDims + c] = sl * kSlabDims + c;
+                        ++n;
+                    }
                 }
             }
             __syncthreads();
@@ -479,7 +530,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
                     for (int e = 0; e < 4; ++e) {
                         float x = 0.f;
                         if (sb < R16) {
-                            const int d = (MAG ? misc[96 + sb] : sb) * 16 + 2 * t + (e & 1) + (e >> 1) * 8;
+                            const int i = sb * 16 + 2 * t + (e & 1) + (e >> 1) * 8;  // slot row
+                            const int d = MAG ? misc[kSelDims + i] : i;
                             if (!p.group_max) {
                                 x = (ng == 0 && g < 2) ? split_part(qs[d], g & 1) : 0.f;
                             } else {
@@ -492,14 +544,20 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
                     qb[ng][sb][0] = pack_bf16(v[0], v[1]);
                     qb[ng][sb][1] = pack_bf16(v[2], v[3]);
                 }
-            const int arow = (lane & 7) + 8 * ((lane >> 3) & 1), ahalf = lane >> 4;
+            // ldmatrix.trans row address of this lane: matrix m = lane / 8 holds
+            // tokens 8 (m & 1) .. + 7 of dims 8 (m >> 1) + (lane & 7) of the k-step
+            const int mrow = (lane & 7) + 8 * (lane >> 4), mhalf = (lane >> 3) & 1;
             // block it's slot into fragments, then the slot's refill
             auto load_block = [&](int it, uint32_t (&a)[RMAX][4]) {
                 wait_slot();
                 const unsigned char* sl = wring + (it & smask) * p.slot_bytes;
 #pragma unroll
                 for (int sb = 0; sb < RMAX; ++sb)
-                    if (sb < R16) ldmatrix_x4(a[sb][0], a[sb][1], a[sb][2], a[sb][3], sl + sb * 512 + arow * 32 + ahalf * 16);
+                    if (sb < R16) {
+                        const int row = sb * 16 + mrow;
+                        ldmatrix_x4_trans(a[sb][0], a[sb][1], a[sb][2], a[sb][3],
+                                          sl + row * 32 + ((mhalf ^ ((row >> 2) & 1)) << 4));
+                    }
                 __syncwarp();
                 refill(it + S);
             };
@@ -553,64 +611,47 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
                 for (int u = 0; u < U; ++u) score_block(it + u, a[u]);
             }
         };
+        // CUDA cores: lane (token = lane % 16, half = lane / 16) sums its half
+        // of the slot's dim rows in fp32; the halves are added
         auto body = [&](auto rmax_tag) {
             constexpr int RMAX = decltype(rmax_tag)::value;
-            const int R16 = p.r / kSlabDims;
-            using V8 = Vec<T, 8>;
-            const int tok = lane >> 1, half = lane & 1;
+            const int tok = lane & 15, hf = lane >> 4;
+            const int rh = p.r / 2;
             for (int it = 0; it < my_blocks; ++it) {
                 wait_slot();
                 const T* sl = reinterpret_cast<const T*>(wring + (it & smask) * p.slot_bytes);
-                typename V8::raw_t raw[RMAX];
+                float x[RMAX * 8];
 #pragma unroll
-                for (int sb = 0; sb < RMAX; ++sb)
-                    if (sb < R16) raw[sb] = V8::load(sl + sb * 256 + tok * 16 + half * 8);
+                for (int i = 0; i < RMAX * 8; ++i) x[i] = i < rh ? Elem<T>::to_f(sl[(hf * rh + i) * 16 + tok]) : 0.f;
                 __syncwarp();
                 refill(it + S);
                 float sc;
                 if (!p.group_max) {
                     float a = 0.f;
 #pragma unroll
-                    for (int sb = 0; sb < RMAX; ++sb) {
-                        if (sb >= R16) break;
-                        float kf[8];
-                        V8::to_float(raw[sb], kf);
-                        const int d0 = (MAG ? misc[96 + sb] : sb) * 16 + half * 8;
-                        const float4 q0 = *reinterpret_cast<const float4*>(qs + d0);
-                        const float4 q1 = *reinterpret_cast<const float4*>(qs + d0 + 4);
-                        a = fmaf(q0.x, kf[0], a);
-                        a = fmaf(q0.y, kf[1], a);
-                        a = fmaf(q0.z, kf[2], a);
-                        a = fmaf(q0.w, kf[3], a);
-                        a = fmaf(q1.x, kf[4], a);
-                        a = fmaf(q1.y, kf[5], a);
-                        a = fmaf(q1.z, kf[6], a);
-                        a = fmaf(q1.w, kf[7], a);
-                    }
-                    sc = a + __shfl_xor_sync(kFull, a, 1);
-                } else {
-                    float ag[G];
-#pragma unroll
-                    for (int j = 0; j < G; ++j) ag[j] = 0.f;
-#pragma unroll
-                    for (int sb = 0; sb < RMAX; ++sb) {
-                        if (sb >= R16) break;
-                        float kf[8];
-                        V8::to_float(raw[sb], kf);
-#pragma unroll
-                        for (int j = 0; j < G; ++j) {
-                            const float* qq = qsc + j * D + (MAG ? misc[96 + sb] : sb) * 16 + half * 8;
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) ag[j] = fmaf(qq[i], kf[i], ag[j]);
+                    for (int i = 0; i < RMAX * 8; ++i)
+                        if (i < rh) {
+                            const int row = hf * rh + i;
+                            a = fmaf(qs[MAG ? misc[kSelDims + row] : row], x[i], a);
                         }
-                    }
+                    sc = a + __shfl_xor_sync(kFull, a, 16);
+                } else {
                     float m = -INFINITY;
 #pragma unroll
-                    for (int j = 0; j < G; ++j) m = fmaxf(m, ag[j] + __shfl_xor_sync(kFull, ag[j], 1));
+                    for (int j = 0; j < G; ++j) {
+                        float a = 0.f;
+#pragma unroll
+                        for (int i = 0; i < RMAX * 8; ++i)
+                            if (i < rh) {
+                                const int row = hf * rh + i;
+                                a = fmaf(qsc[j * D + (MAG ? misc[kSelDims + row] : row)], x[i], a);
+                            }
+                        m = fmaxf(m, a + __shfl_xor_sync(kFull, a, 16));
+                    }
                     sc = m;
                 }
                 const int li = (warp + it * kWarps) * kBlockTokens + tok;
-                if (half == 0 && li < n_cand_loc) {
+                if (hf == 0 && li < n_cand_loc) {
                     const uint32_t key = score_key(sc);
                     keys[li] = key;
                     atomicAdd(&hist[key >> 21], 1u);

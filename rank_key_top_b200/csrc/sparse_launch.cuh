@@ -9,6 +9,7 @@
 #include <algorithm>
 #include <map>
 #include <mutex>
+#include <tuple>
 #include <utility>
 
 #include "sparse_decode.cuh"
@@ -22,28 +23,51 @@ struct DeviceInfo {
 
 inline DeviceInfo device_info() {
     static std::mutex mu;
-    static DeviceInfo cache[64];
-    static bool have[64] = {};
+    static std::map<int, DeviceInfo> cache;
     int dev = 0;
     cudaGetDevice(&dev);
     std::lock_guard<std::mutex> lock(mu);
-    if (dev >= 0 && dev < 64 && have[dev]) return cache[dev];
+    auto it = cache.find(dev);
+    if (it != cache.end()) return it->second;
     DeviceInfo di;
     cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev);
     cudaDeviceGetAttribute(&di.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    if (dev >= 0 && dev < 64) {
-        cache[dev] = di;
-        have[dev] = true;
-    }
+    cudaGetLastError();  // no device: the attributes stay 0 and every shape is unsupported
+    cache[dev] = di;
     return di;
 }
 
-// Whether at least one cluster of this shape can be resident on the device,
-// cached per kernel instantiation, cluster size and shared-memory size.
+// Allows `kern` up to `bytes` of dynamic shared memory on the current device:
+// the attribute belongs to the function on that device, and it is raised
+// (never lowered) as larger launches come, so every size up to the largest
+// requested so far stays launchable.
+inline cudaError_t ensure_smem_attr(const void* kern, int bytes) {
+    static std::mutex mu;
+    static std::map<std::pair<int, const void*>, int> allowed;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    const auto key = std::make_pair(dev, kern);
+    auto it = allowed.find(key);
+    if (it != allowed.end() && it->second >= bytes) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return e;
+    }
+    allowed[key] = bytes;
+    return cudaSuccess;
+}
+
+// Whether at least one cluster of this shape can be resident on the current
+// device, cached per device, kernel instantiation, cluster size and
+// shared-memory size.
 template <typename K>
-bool cluster_fits(K kern, const cudaLaunchConfig_t& cfg, std::map<std::pair<int, int>, bool>& known,
+bool cluster_fits(K kern, const cudaLaunchConfig_t& cfg, std::map<std::tuple<int, int, int>, bool>& known,
                   std::mutex& mu) {
-    const std::pair<int, int> key(cfg.gridDim.x, (int)cfg.dynamicSmemBytes);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const std::tuple<int, int, int> key(dev, (int)cfg.gridDim.x, (int)cfg.dynamicSmemBytes);
     std::lock_guard<std::mutex> lock(mu);
     auto it = known.find(key);
     if (it != known.end()) return it->second;
@@ -102,7 +126,7 @@ void sparse_layout(SparseParams& p, int max_seq_len, int ring_per_warp) {
     p.off_part = off;  // one partial slot per CTA of the cluster (used in rank 0)
     off = align(off + p.C * G * (D + 2) * 4);
     p.off_misc = off;
-    off = align(off + 128 * 4);
+    off = align(off + 256 * 4);
     p.smem_bytes = off;
 }
 
@@ -158,12 +182,15 @@ struct SparseFits {
 
 template <typename T, int D, int G>
 struct SparseLaunch {
-    // scorer: kScoreLeading, kScoreMagnitude or kScoreAsym
+    // scorer: kScoreLeading, kScoreMagnitude, kScoreSlabs or kScoreAsym
     static loki_status run(SparseParams p, int pairs, int max_seq_len, const DeviceInfo& di,
                            cudaStream_t stream, bool programmatic, int scorer) {
-        if (scorer == kScoreMagnitude) return run_kernel<kScoreMagnitude>(p, pairs, max_seq_len, di, stream, programmatic);
-        if (scorer == kScoreAsym) return run_kernel<kScoreAsym>(p, pairs, max_seq_len, di, stream, programmatic);
-        return run_kernel<kScoreLeading>(p, pairs, max_seq_len, di, stream, programmatic);
+        switch (scorer) {
+            case kScoreMagnitude: return run_kernel<kScoreMagnitude>(p, pairs, max_seq_len, di, stream, programmatic);
+            case kScoreSlabs: return run_kernel<kScoreSlabs>(p, pairs, max_seq_len, di, stream, programmatic);
+            case kScoreAsym: return run_kernel<kScoreAsym>(p, pairs, max_seq_len, di, stream, programmatic);
+            default: return run_kernel<kScoreLeading>(p, pairs, max_seq_len, di, stream, programmatic);
+        }
     }
 
     template <int SC>
@@ -172,14 +199,22 @@ struct SparseLaunch {
         if (choose_cluster<T, D, G>(p, max_seq_len, pairs, di.sms, di.max_smem_optin) < 1)
             return LOKI_ERR_UNSUPPORTED;
         auto kern = sparse_decode_kernel<T, D, G, SC>;
-        static std::once_flag once;
-        static cudaError_t attr_err = cudaSuccess;
-        std::call_once(once, [&] {
-            attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, di.max_smem_optin);
-            if (attr_err == cudaSuccess)
-                attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        });
-        if (attr_err != cudaSuccess) return LOKI_ERR_CUDA;
+        // per device: the shared-memory opt-in and non-portable cluster sizes
+        if (ensure_smem_attr((const void*)kern, di.max_smem_optin) != cudaSuccess) return LOKI_ERR_CUDA;
+        {
+            static std::mutex mu;
+            static std::map<int, cudaError_t> cluster_attr;
+            int dev = 0;
+            cudaGetDevice(&dev);
+            std::lock_guard<std::mutex> lock(mu);
+            auto it = cluster_attr.find(dev);
+            if (it == cluster_attr.end()) {
+                cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+                if (e != cudaSuccess) cudaGetLastError();
+                it = cluster_attr.emplace(dev, e).first;
+            }
+            if (it->second != cudaSuccess) return LOKI_ERR_CUDA;
+        }
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(p.C, pairs, 1);
         cfg.blockDim = dim3(kThreads, 1, 1);
@@ -198,11 +233,14 @@ struct SparseLaunch {
         cfg.attrs = attr;
         cfg.numAttrs = programmatic ? 2 : 1;
         // a cluster that can never be resident is reported, not launched
-        static std::map<std::pair<int, int>, bool> known;
+        static std::map<std::tuple<int, int, int>, bool> known;
         static std::mutex known_mu;
         if (!cluster_fits(kern, cfg, known, known_mu)) return LOKI_ERR_UNSUPPORTED;
-        if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return LOKI_ERR_CUDA;
-        return cudaPeekAtLastError() == cudaSuccess ? LOKI_OK : LOKI_ERR_CUDA;
+        if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) {
+            cudaGetLastError();  // reported here, not by a later call
+            return LOKI_ERR_CUDA;
+        }
+        return LOKI_OK;
     }
 };
 

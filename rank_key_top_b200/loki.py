@@ -25,6 +25,7 @@ LOKI_GROUP_SUM = 0
 LOKI_GROUP_MAX = 1
 LOKI_SCORER_LEADING = 0
 LOKI_SCORER_MAGNITUDE = 1
+LOKI_SCORER_MAGNITUDE_SLABS = 2
 
 LOKI_DEVERR_SEQ_LEN = 0x1
 LOKI_DEVERR_BLOCK_ID = 0x2
@@ -204,10 +205,25 @@ def loki_decode_workspace_bytes(cache, batch, num_q_heads, k, recent_window=0):
                                             num_q_heads, k, recent_window)
 
 
+def decode_workspace(cache, batch, num_q_heads, k, recent_window=0, device="cuda"):
+    """A device buffer of loki_decode_workspace_bytes() bytes for the decode
+    calls, or None when they need none."""
+    n = loki_decode_workspace_bytes(cache, batch, num_q_heads, k, recent_window)
+    return torch.empty(n, dtype=torch.uint8, device=device) if n else None
+
+
+def _workspace(workspace, cache, batch, q, k, recent_window):
+    """The caller's workspace, or one allocated for this call (torch's caching
+    allocator) when none is given and the call needs one."""
+    if workspace is None:
+        workspace = decode_workspace(cache, batch, q.shape[1], k, recent_window, q.device)
+    return workspace, (workspace.numel() * workspace.element_size() if workspace is not None else 0)
+
+
 def loki_decode_attention(cache, batch, q, P, r, k, out, k_per_seq=None, recent_window=0,
                           group_reduce=LOKI_GROUP_SUM, scale=0.0, selected_idx=None,
                           workspace=None, stream=None):
-    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    workspace, ws_bytes = _workspace(workspace, cache, batch, q, k, recent_window)
     _check("loki_decode_attention", _lib.loki_decode_attention(
         ctypes.byref(cache.struct), ctypes.byref(batch.struct), _ptr(q), q.shape[1], _ptr(P), r, k,
         _ptr(k_per_seq), recent_window, group_reduce, scale, _ptr(out), _ptr(selected_idx),
@@ -217,7 +233,7 @@ def loki_decode_attention(cache, batch, q, P, r, k, out, k_per_seq=None, recent_
 def loki_decode_attention_scored(cache, batch, q, P, r, k, out, scorer=LOKI_SCORER_LEADING, k_per_seq=None,
                                  recent_window=0, group_reduce=LOKI_GROUP_SUM, scale=0.0, selected_idx=None,
                                  workspace=None, stream=None):
-    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    workspace, ws_bytes = _workspace(workspace, cache, batch, q, k, recent_window)
     _check("loki_decode_attention_scored", _lib.loki_decode_attention_scored(
         ctypes.byref(cache.struct), ctypes.byref(batch.struct), _ptr(q), q.shape[1], _ptr(P), r, k,
         _ptr(k_per_seq), recent_window, group_reduce, scale, scorer, _ptr(out), _ptr(selected_idx),
@@ -227,7 +243,7 @@ def loki_decode_attention_scored(cache, batch, q, P, r, k, out, scorer=LOKI_SCOR
 def loki_decode_attention_asym(cache, batch, q, P, A_q, r, k, out, k_per_seq=None, recent_window=0,
                                group_reduce=LOKI_GROUP_SUM, scale=0.0, selected_idx=None, workspace=None,
                                stream=None):
-    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    workspace, ws_bytes = _workspace(workspace, cache, batch, q, k, recent_window)
     _check("loki_decode_attention_asym", _lib.loki_decode_attention_asym(
         ctypes.byref(cache.struct), ctypes.byref(batch.struct), _ptr(q), q.shape[1], _ptr(P), _ptr(A_q), r, k,
         _ptr(k_per_seq), recent_window, group_reduce, scale, _ptr(out), _ptr(selected_idx),
@@ -249,7 +265,7 @@ def loki_index_keys(cache, batch, k, A_k, stream=None):
 def loki_decode_step(cache, batch, k_new, v_new, q, P, r, k, out, k_per_seq=None, recent_window=0,
                      group_reduce=LOKI_GROUP_SUM, scale=0.0, selected_idx=None, workspace=None, stream=None):
     """Append the step's token, then decode (one call, the attention overlapping the append)."""
-    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    workspace, ws_bytes = _workspace(workspace, cache, batch, q, k, recent_window)
     _check("loki_decode_step", _lib.loki_decode_step(
         ctypes.byref(cache.struct), ctypes.byref(batch.struct), _ptr(k_new), _ptr(v_new), _ptr(q), q.shape[1],
         _ptr(P), r, k, _ptr(k_per_seq), recent_window, group_reduce, scale, _ptr(out), _ptr(selected_idx),

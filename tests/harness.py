@@ -10,7 +10,7 @@ from rank_key_top_b200 import synth
 BF16_RTOL = 2e-3   # max normwise relative error of outputs, bf16 caches
 F32_RTOL = 1e-5    # the same for fp32 caches
 TIE_BAND = 1e-3    # selected sets may differ only where |s_t - s_(k)| <= TIE_BAND |s_(k)|
-SLAB_MARGIN = 1e-3  # magnitude scorer: the last kept slab must beat the first dropped one by this much
+SLAB_MARGIN = 1e-3  # magnitude scorers: the last kept dim (slab) must beat the first dropped one by this much
 
 
 def tol_for(spec):
@@ -78,13 +78,15 @@ def pair_inputs(wl, b, h, q=None):
 
 
 def check_pair(wl, b, h, out_gpu, sel_gpu, r, k, W, group_max=False, scale=0.0, q=None, rtol=None,
-               inputs=None, magnitude_dims=None, asym=None):
+               inputs=None, magnitude_dims=None, asym=None, magnitude="slabs"):
     """Set parity (with the tie band) and output parity for one pair.
 
-    magnitude_dims: the key index's width when the magnitude scorer ran (the
-    oracle then chooses the scoring slabs the same way, and the input must
-    separate the last kept slab from the first dropped one by SLAB_MARGIN, so
-    that both sides' choice is the same whatever their precision).
+    magnitude_dims: the key index's width when a magnitude scorer ran; with
+    magnitude="dims" the oracle chooses single dims (AQUA's per-dimension
+    selection), with "slabs" whole 16-dim slabs, from the same queries. The
+    input must separate the last kept dim (slab) from the first dropped one by
+    SLAB_MARGIN, so that both sides' choice is the same whatever their
+    precision.
     asym: (Kidx, A_q) of the pair when the asymmetric scorer ran: the
     oracle's own key-index rows round(k A_k) and the query factor.
     Returns (output error on the GPU's set, output error on the oracle's set)."""
@@ -98,6 +100,11 @@ def check_pair(wl, b, h, out_gpu, sel_gpu, r, k, W, group_max=False, scale=0.0, 
                                       scale=scale)
     elif magnitude_dims is None:
         res = oracle.decode_pair(Kt, V, qq, P, r=r, k=kb, W=W, group_max=group_max, scale=scale)
+    elif magnitude == "dims":
+        res = oracle.decode_pair_dims(Kt, V, qq, P, r, kb, magnitude_dims, W=W, group_max=group_max, scale=scale)
+        w = np.sort(res.weight)[::-1]
+        if r < w.size:
+            assert w[r - 1] - w[r] > SLAB_MARGIN * w[r - 1], f"pair {(b, h)}: input without a dim-selection margin"
     else:
         res = oracle.decode_pair_magnitude(Kt, V, qq, P, r, kb, magnitude_dims, W=W, group_max=group_max,
                                            scale=scale)

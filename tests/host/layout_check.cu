@@ -85,7 +85,8 @@ void check(const char* tname, int sms, int optin) {
                 CHECK(p.off_part - p.off_hist >= 2 * kHistBins * 4);
                 CHECK(p.off_misc - p.off_part >= p.C * G * (D + 2) * 4);
                 CHECK(p.off_misc - p.off_part >= G * D * 4);  // the asymmetric scorer's query
-                CHECK(p.smem_bytes - p.off_misc >= 128 * 4);
+                CHECK(p.smem_bytes - p.off_misc >= 256 * 4);  // misc words, then the chosen dims
+                CHECK(kSelDims + D <= 256);
                 // spread: a cluster larger than needed only while every cluster still fits at once
                 SparseParams q = {};
                 q.r = r;

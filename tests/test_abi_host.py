@@ -36,7 +36,7 @@ def test_library_exports_every_declared_symbol(loki):
     for name in declared_symbols():
         assert hasattr(lib, name), name
     assert sorted(loki.EXPORTED) == declared_symbols()
-    assert loki.loki_abi_version() == 3
+    assert loki.loki_abi_version() == 4
 
 
 def test_status_strings(loki):
@@ -57,6 +57,7 @@ def test_cache_bytes(loki):
     assert loki.loki_cache_bytes(10, 8, 96, loki.LOKI_F32) == 0
     assert loki.loki_cache_bytes(-1, 8, 128, loki.LOKI_F32) == 0
     assert loki.loki_decode_max_seq_len(128, loki.LOKI_BF16) == 262144
+    assert loki.loki_decode_max_seq_len(96, loki.LOKI_BF16) == 0
 
 
 FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
@@ -103,7 +104,7 @@ def test_decode_rejects_bad_shapes(loki):
     c, b = structs(loki, max_len=65)       # exceeds 16 * max_blocks_per_seq
     assert decode(loki, c, b) == 1
     c, b = structs(loki, max_blocks=20000, max_len=300000)
-    assert decode(loki, c, b) == 2         # above the fused kernel's capacity
+    assert decode(loki, c, b) == 2         # above loki_decode_max_seq_len
     c, b = structs(loki, B=-1)
     assert decode(loki, c, b) == 1
     c = loki.loki_cache(FAKE + 8, FAKE, FAKE, 8, 8, 128, 32, 1)
@@ -148,9 +149,10 @@ def scored(loki, c, b, scorer, Hq=32, r=32, k=8, W=0, q=FAKE, P=FAKE, out=FAKE):
 
 
 @pytest.mark.parametrize("scorer,kw,status", [
-    (2, {}, 1),                     # unknown scorer
+    (3, {}, 1),                     # unknown scorer
     (-1, {}, 1),
-    (1, dict(r=48), 1),             # r above index_dims (32), for either scorer
+    (1, dict(r=48), 1),             # r above index_dims (32), for every scorer
+    (2, dict(r=48), 1),
     (0, dict(r=48), 1),
     (1, dict(k=0, W=0), 1),
     (1, dict(Hq=24), 2),
@@ -236,3 +238,13 @@ def test_dense_rejects(loki):
     assert args(FAKE, need - 1) == 3
     assert args(FAKE + 16, need) == 1      # workspace must be 256-byte aligned
     assert args(FAKE, need, Hq=24) == 2
+
+
+
+def test_decode_needs_no_workspace(loki):
+    """The fused decode kernel keeps every intermediate on chip: the decode
+    calls need no workspace (size 0; NULL is accepted)."""
+    lib = loki.raw()
+    c, b = structs(loki)
+    assert lib.loki_decode_workspace_bytes(ctypes.byref(c), ctypes.byref(b), 32, 8, 0) == 0
+    assert lib.loki_decode_workspace_bytes(ctypes.byref(c), ctypes.byref(b), 32, 2048, 64) == 0

@@ -171,19 +171,19 @@ def read_pair(dev, b, h, L):
     """Reads keys, values and the key index of one pair back through the
     documented layout: block p of head h at element (p * Hkv + h) * 16 * D in
     the key and value caches ([16 tokens][D] each) and at (p * Hkv + h) * 16 * I
-    in the key index ([I/16 slabs][16 tokens][16 dims])."""
+    in the key index ([I dims][16 tokens])."""
     s = dev.wl.spec
     dt = synth.torch_dtype(s.dtype)
     D, Hkv, I = s.head_dim, s.num_kv_heads, dev.cache.index_dims
     kc = dev.cache.k.view(dt).view(-1, Hkv, 16, D)
     vc = dev.cache.v.view(dt).view(-1, Hkv, 16, D)
-    xc = dev.cache.x.view(dt).view(-1, Hkv, I // 16, 16, 16)
+    xc = dev.cache.x.view(dt).view(-1, Hkv, I, 16)
     tbl = dev.wl.block_table[b]
     nblk = (L + 15) // 16
     blocks = tbl[:nblk].long().to(kc.device)
     K = kc[blocks, h].reshape(nblk * 16, D)[:L]
     V = vc[blocks, h].reshape(nblk * 16, D)[:L]
-    X = xc[blocks, h].permute(0, 2, 1, 3).reshape(nblk * 16, I)[:L]
+    X = xc[blocks, h].permute(0, 2, 1).reshape(nblk * 16, I)[:L]
     return K.cpu(), V.cpu(), X.cpu()
 
 
@@ -556,8 +556,65 @@ def test_long_context_outliers_sweep(cuda_lib):
 
 
 # ---------------------------------------------------------------------------
-# Magnitude scorer: the scoring slabs chosen by query energy
+# Magnitude scorers: the scoring dims chosen per step by the query's magnitude
+# (single dims, AQUA's algorithm) or energy (whole 16-dim slabs)
 # ---------------------------------------------------------------------------
+
+def magnitude_dim_queries(wl, group_max, index_dims, seed):
+    """Queries whose rotated dims carry the magnitudes 1.03^i, i = 0 ..
+    index_dims - 1, in a shuffled order per (sequence, kv head): the magnitude
+    the reduce measures (|sum_j q_hat_j[c]| for SUM, sqrt(sum_j q_hat_j[c]^2)
+    for MAX) is set exactly, so the chosen dims have a 3 % margin over the
+    dropped ones. Dims past index_dims get magnitude 1. q = q_hat P^T."""
+    s = wl.spec
+    g, d = s.group, s.head_dim
+    gen = torch.Generator().manual_seed(seed)
+    q = torch.empty(s.batch, s.num_q_heads, d, dtype=torch.float64)
+    for b in range(s.batch):
+        for h in range(s.num_kv_heads):
+            mags = torch.ones(d, dtype=torch.float64)
+            mags[:index_dims] = 1.03 ** torch.randperm(index_dims, generator=gen).double()
+            z = torch.randn(g, d, generator=gen, dtype=torch.float64)
+            if group_max:
+                qhat = z * (mags / z.pow(2).sum(0).sqrt())
+            else:
+                sign = torch.where(torch.rand(d, generator=gen) < 0.5, -1.0, 1.0).double()
+                noise = 0.3 * (z - z.mean(0, keepdim=True)) * mags
+                qhat = (mags * sign) / g + noise
+            q[b, h * g:(h + 1) * g] = qhat @ wl.P[h].double().T
+    return q.to(wl.q.dtype)
+
+
+@pytest.mark.parametrize("dtype,D,Hq,Hkv,index_dims,r,group_max,lens", [
+    ("bf16", 128, 8, 2, 128, 32, False, [20000, 3000, 777, 33]),
+    ("bf16", 128, 16, 2, 64, 16, True, [3000, 777]),
+    ("bf16", 64, 2, 1, 64, 48, False, [3000, 1]),
+    ("f32", 128, 4, 1, 128, 64, True, [3000, 0, 500]),
+    ("f32", 64, 4, 4, 64, 16, False, [2500, 777]),
+    ("bf16", 128, 4, 4, 96, 32, True, [5000, 1200, 16]),
+])
+def test_magnitude_scorer_matches_oracle(cuda_lib, dtype, D, Hq, Hkv, index_dims, r, group_max, lens):
+    """Set and output parity with the oracle's per-dimension selection (AQUA
+    page, Algorithm 1 in prose; appendix on complexity, steps 2-4), which
+    chooses from the same queries; at least one pair must choose dims other
+    than the leading ones, or the case would not test the choice."""
+    s = spec(dtype=dtype, head_dim=D, num_q_heads=Hq, num_kv_heads=Hkv, seq_lens=lens, r=r, k=150,
+             recent_window=5)
+    wl = synth.make_workload(s)
+    wl.q = magnitude_dim_queries(wl, group_max, index_dims, seed=23)
+    dev = harness.Device(wl, cuda_lib, index_dims=index_dims)
+    out, sel = dev.decode(group_max=group_max, scorer=cuda_lib.LOKI_SCORER_MAGNITUDE)
+    assert cuda_lib.loki_device_error() == 0
+    moved = 0
+    for b in range(s.batch):
+        for h in range(s.num_kv_heads):
+            harness.check_pair(wl, b, h, out, sel, r, s.k, s.recent_window, group_max=group_max,
+                               magnitude_dims=index_dims, magnitude="dims")
+            qq, P = harness.pair_inputs(wl, b, h)[2:]
+            dims, _ = oracle.magnitude_dims(qq, P, r, index_dims, group_max)
+            moved += dims.tolist() != list(range(r))
+    assert moved > 0
+
 
 def magnitude_queries(wl, group_max, seed):
     """Queries whose rotated slabs carry the energies 1.3^(2i), i = 0 .. d/16 - 1,
@@ -587,22 +644,21 @@ def magnitude_queries(wl, group_max, seed):
     ("f32", 128, 4, 1, 128, 64, True, [3000, 0, 500]),
     ("f32", 64, 4, 4, 64, 16, False, [2500, 777]),
 ])
-def test_magnitude_scorer_matches_oracle(cuda_lib, dtype, D, Hq, Hkv, index_dims, r, group_max, lens):
-    """Set and output parity with the oracle, which chooses the slabs from
-    the same queries; at least one pair must choose slabs other than the
-    leading ones, or the case would not test the choice."""
+def test_slab_scorer_matches_oracle(cuda_lib, dtype, D, Hq, Hkv, index_dims, r, group_max, lens):
+    """The slab variant against the oracle's slab choice from the same
+    queries; at least one pair must choose slabs other than the leading ones."""
     s = spec(dtype=dtype, head_dim=D, num_q_heads=Hq, num_kv_heads=Hkv, seq_lens=lens, r=r, k=150,
              recent_window=5)
     wl = synth.make_workload(s)
     wl.q = magnitude_queries(wl, group_max, seed=21)
     dev = harness.Device(wl, cuda_lib, index_dims=index_dims)
-    out, sel = dev.decode(group_max=group_max, scorer=cuda_lib.LOKI_SCORER_MAGNITUDE)
+    out, sel = dev.decode(group_max=group_max, scorer=cuda_lib.LOKI_SCORER_MAGNITUDE_SLABS)
     assert cuda_lib.loki_device_error() == 0
     moved = 0
     for b in range(s.batch):
         for h in range(s.num_kv_heads):
             harness.check_pair(wl, b, h, out, sel, r, s.k, s.recent_window, group_max=group_max,
-                               magnitude_dims=index_dims)
+                               magnitude_dims=index_dims, magnitude="slabs")
             qq, P = harness.pair_inputs(wl, b, h)[2:]
             slabs, _ = oracle.magnitude_slabs(qq, P, r, index_dims, group_max)
             moved += slabs.tolist() != list(range(r // 16))
@@ -619,14 +675,15 @@ def test_scored_entry_with_leading_scorer_is_decode_attention(cuda_lib):
 
 
 @pytest.mark.parametrize("group_max", [False, True])
-def test_magnitude_scorer_with_every_slab_is_leading(cuda_lib, group_max):
-    """r = index_dims: every slab is chosen, in ascending order, so the
+@pytest.mark.parametrize("scorer", ["LOKI_SCORER_MAGNITUDE", "LOKI_SCORER_MAGNITUDE_SLABS"])
+def test_magnitude_scorer_with_every_dim_is_leading(cuda_lib, group_max, scorer):
+    """r = index_dims: every dim (slab) is chosen, in ascending order, so a
     magnitude scorer computes what the leading scorer does, bit for bit."""
     s = spec(num_q_heads=4, num_kv_heads=1, seq_lens=[4000, 900], r=64, k=100, recent_window=2)
     wl = synth.make_workload(s)
     dev = harness.Device(wl, cuda_lib, index_dims=64)
     a = dev.decode(group_max=group_max)
-    b = dev.decode(group_max=group_max, scorer=cuda_lib.LOKI_SCORER_MAGNITUDE)
+    b = dev.decode(group_max=group_max, scorer=getattr(cuda_lib, scorer))
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
