@@ -46,7 +46,7 @@ extern "C" {
 #define LOKI_API
 #endif
 
-#define LOKI_ABI_VERSION 4
+#define LOKI_ABI_VERSION 5
 #define LOKI_BLOCK_TOKENS 16 /* tokens per paged-cache block */
 
 typedef void* loki_stream_t; /* a cudaStream_t */
@@ -111,14 +111,40 @@ typedef enum loki_scorer {
  * over the kept tokens. The index costs index_dims/head_dim of the key cache
  * (12.5% of keys + values for index_dims = 32, head_dim = 128). */
 typedef struct loki_cache {
-    void* k_cache;         /* device, loki_cache_bytes(), 16-byte aligned */
-    void* v_cache;         /* device, loki_cache_bytes(), 16-byte aligned */
+    void* k_cache;         /* device, loki_cache_bytes(), 16-byte aligned; not */
+    void* v_cache;         /* NULL, even when every block is offloaded        */
     void* k_index;         /* device, loki_index_bytes(), 16-byte aligned */
     int32_t num_blocks;    /* physical blocks in each cache */
     int32_t num_kv_heads;  /* >= 1 */
     int32_t head_dim;      /* 64 or 128 */
     int32_t index_dims;    /* multiple of 16 in [16, head_dim]; the largest usable r */
     loki_dtype dtype;
+    /* Optional offload of key and value rows to host memory (LRQK page,
+     * abstract: a mixed GPU-CPU cache in which only the missing full-precision
+     * rows of the kept tokens cross to the GPU). With kv_home NULL the fields
+     * below except kv_touch are ignored, and block p's key and value rows are
+     * device page p (k_cache and v_cache hold num_blocks pages). With kv_home
+     * set, block p's rows are
+     *   kv_home[p] >= 0: device page kv_home[p]; k_cache and v_cache hold
+     *                    num_device_pages pages (loki_cache_bytes(
+     *                    num_device_pages, ...) bytes each);
+     *   kv_home[p] < 0:  host page -(kv_home[p] + 1) of k_host and v_host,
+     *                    num_host_pages pages each in the same page layout.
+     * A page holds one block's rows of every kv head (the layout above with p
+     * the page number). The key index stays on the device whatever kv_home
+     * says. Every call reads and writes offloaded rows in place through the
+     * host pools' device mapping; a sparse decode reads only the kept rows of
+     * offloaded blocks. An entry outside its pool sets LOKI_DEVERR_BLOCK_ID and
+     * its rows read as zero and are not written. */
+    const int32_t* kv_home;    /* device [num_blocks], or NULL */
+    void* k_host;              /* device address (loki_host_device_pointer) of  */
+    void* v_host;              /* pinned host memory, 16-byte aligned           */
+    int32_t num_device_pages;  /* with kv_home: pages in k_cache and v_cache, >= 0 */
+    int32_t num_host_pages;    /* with kv_home: pages in k_host and v_host, >= 0 */
+    uint32_t* kv_touch;        /* nullable, device [num_blocks]: every sparse
+                                  decode adds to entry p the number of kept rows
+                                  it gathered from block p (over all kv heads);
+                                  the offload planner's hit counts */
 } loki_cache;
 
 /* Per-sequence addressing of one decode batch. */
@@ -394,6 +420,51 @@ LOKI_API loki_status loki_dense_attention(const loki_cache* cache, const loki_ba
 LOKI_API loki_status loki_dense_attention_static(const loki_cache* cache, const loki_batch* batch,
                                                  const void* q, int32_t num_q_heads, const float* P,
                                                  float scale, float* out, loki_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Host offload of key and value pages (LRQK page, abstract: the hit-and-miss
+ * mechanism of a mixed GPU-CPU cache). Blocks whose rows the decodes keep
+ * selecting are promoted to device pages and the least selected device blocks
+ * take their place on the host, between decode steps.
+ * ------------------------------------------------------------------------ */
+
+/* One swap: block_in (offloaded, in host page host_page) moves to the free
+ * device page device_page; block_out (on the device, in device page
+ * freed_page) moves to host_page; freed_page is then the free device page. */
+typedef struct loki_page_move {
+    int32_t block_in;
+    int32_t block_out;
+    int32_t host_page;
+    int32_t device_page;
+    int32_t freed_page;
+} loki_page_move;
+
+/* Host-only planning of swaps (no CUDA call). kv_home is a host copy of the
+ * cache's map [num_blocks] and spare_page the one device page no block uses;
+ * touch is a host copy of kv_touch. Offloaded blocks in order of decreasing
+ * touch count (ties: lower block id) are paired with device blocks in order of
+ * increasing touch count (ties: lower block id); a pair is swapped while the
+ * offloaded block's count is strictly the larger, at most max_moves swaps.
+ * Writes the swaps to moves, updates kv_home and spare_page to the state after
+ * them and returns their number, or -1 for invalid arguments (a NULL pointer,
+ * num_blocks < 0, max_moves < 0, spare_page < 0 or used by a block). */
+LOKI_API int32_t loki_offload_plan(int32_t num_blocks, int32_t* kv_home, int32_t* spare_page,
+                                   const uint32_t* touch, int32_t max_moves, loki_page_move* moves);
+
+/* Issues the swaps on the stream, in order: per move, block_in's key page and
+ * value page host -> device_page, then block_out's key and value pages
+ * freed_page -> host_page (one cudaMemcpyAsync per page); then the updated map
+ * kv_home_host [num_blocks] -> cache->kv_home. Stream-ordered with the calls
+ * before and after it on the stream. A pinned kv_home_host must stay unchanged
+ * until the stream has passed the copy; a pageable one may change once the
+ * call returns. Page and block numbers outside their pools give
+ * LOKI_ERR_INVALID_ARG before anything is issued. */
+LOKI_API loki_status loki_offload_apply(const loki_cache* cache, const loki_page_move* moves, int32_t num_moves,
+                                        const int32_t* kv_home_host, loki_stream_t stream);
+
+/* The device address of pinned host memory (cudaHostAlloc'd or registered
+ * mapped); LOKI_ERR_CUDA if the memory is not mapped for the device. */
+LOKI_API loki_status loki_host_device_pointer(void* host, void** device);
 
 /* Reads (and with clear != 0 resets) the device error word of the current
  * device: an OR of LOKI_DEVERR_* bits set by kernels since the last clear.

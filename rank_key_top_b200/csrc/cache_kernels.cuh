@@ -18,6 +18,7 @@ struct PrefillParams {
     const int32_t* seq_lens;
     const void* k_rot;
     const void* v;
+    KvMap kv;
     int num_blocks, Hkv, max_blocks, max_seq_len, max_len, index_dims;
 };
 
@@ -40,13 +41,13 @@ __global__ void __launch_bounds__(256) prefill_kernel(const PrefillParams p) {
         if (threadIdx.x == 0) flag_error(LOKI_DEVERR_BLOCK_ID);
         return;
     }
-    const int64_t page = page_offset(pb, h, p.Hkv, D);
     const int64_t ipage = page_offset(pb, h, p.Hkv, p.index_dims);
     const int64_t src_row0 = (((int64_t)b * p.Hkv + h) * p.max_len + (int64_t)jb * kBlockTokens) * D;
     const T* ks = reinterpret_cast<const T*>(p.k_rot) + src_row0;
     const T* vs = reinterpret_cast<const T*>(p.v) + src_row0;
-    T* kd = reinterpret_cast<T*>(p.k_cache) + page;
-    T* vd = reinterpret_cast<T*>(p.v_cache) + page;
+    T *kd, *vd;
+    kv_rows(p.kv, p.k_cache, p.v_cache, pb, h, p.Hkv, D, kd, vd);
+    if (!kd) return;
     T* xd = reinterpret_cast<T*>(p.k_index) + ipage;
     constexpr int per_tok = D / VEC;
     for (int i = threadIdx.x; i < kBlockTokens * per_tok; i += blockDim.x) {
@@ -75,6 +76,7 @@ struct AppendParams {
     const void* v_new;
     const float* P;   // nullable
     const float* Ak;  // nullable: [Hkv][D][index_dims], the index row is k A_k
+    KvMap kv;
     int num_blocks, Hkv, max_blocks, max_seq_len, index_dims;
 };
 
@@ -142,8 +144,9 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
             x = kin[c];
         }
         const T kt = Elem<T>::from_f(x);
-        const int64_t page = page_offset(pb, h, p.Hkv, D);
-        reinterpret_cast<T*>(p.k_cache)[page + row_offset_in_page(row, c, D)] = kt;
+        T *kd, *vd;
+        kv_rows(p.kv, p.k_cache, p.v_cache, pb, h, p.Hkv, D, kd, vd);
+        if (kd) kd[row_offset_in_page(row, c, D)] = kt;
         if (c < p.index_dims) {
             T xv = kt;
             if (p.Ak) {  // key factor of an asymmetric score: (k A_k)[c], summed in row order
@@ -155,8 +158,7 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
             reinterpret_cast<T*>(p.k_index)[page_offset(pb, h, p.Hkv, p.index_dims) + index_offset_in_page(row, c)] =
                 xv;
         }
-        reinterpret_cast<T*>(p.v_cache)[page + row_offset_in_page(row, c, D)] =
-            reinterpret_cast<const T*>(p.v_new)[src + c];
+        if (vd) vd[row_offset_in_page(row, c, D)] = reinterpret_cast<const T*>(p.v_new)[src + c];
     }
 }
 

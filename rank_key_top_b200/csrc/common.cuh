@@ -40,6 +40,57 @@ __host__ __device__ __forceinline__ int index_offset_in_page(int token, int dim)
 }
 
 // ---------------------------------------------------------------------------
+// Where the key and value rows of a physical block live (LRQK page, abstract:
+// a mixed GPU-CPU cache; the low-rank key index always stays on the device).
+// Without a home map, block p's rows are device page p. With one, home[p] >= 0
+// names a device page and home[p] < 0 the pinned host page -(home[p] + 1),
+// read and written through its device mapping.
+// ---------------------------------------------------------------------------
+struct KvMap {
+    const int32_t* home;  // [num_blocks] or nullptr
+    unsigned char* host_k;
+    unsigned char* host_v;
+    uint32_t* touch;      // [num_blocks] or nullptr: kept rows gathered per block
+    int dev_pages, host_pages;
+};
+
+// The page holding block pb's rows and which pool it is in; false (and the
+// block-id error bit) for a home entry outside its pool.
+struct KvPage {
+    int64_t page;
+    bool host;
+};
+__device__ __forceinline__ bool kv_locate(const KvMap& m, int pb, KvPage& loc) {
+    if (!m.home) {
+        loc.page = pb;
+        loc.host = false;
+        return true;
+    }
+    const int e = m.home[pb];
+    loc.host = e < 0;
+    loc.page = loc.host ? -(int64_t)e - 1 : e;
+    if (loc.page >= (loc.host ? m.host_pages : m.dev_pages)) {
+        flag_error(LOKI_DEVERR_BLOCK_ID);
+        return false;
+    }
+    return true;
+}
+// Element pointers of head h's key and value rows of block pb (nullptr when
+// the home entry is invalid).
+template <typename T>
+__device__ __forceinline__ void kv_rows(const KvMap& m, void* k_cache, void* v_cache, int pb, int h, int Hkv,
+                                        int D, T*& k, T*& v) {
+    KvPage loc;
+    if (!kv_locate(m, pb, loc)) {
+        k = v = nullptr;
+        return;
+    }
+    const int64_t off = page_offset(loc.page, h, Hkv, D);
+    k = reinterpret_cast<T*>(loc.host ? m.host_k : reinterpret_cast<unsigned char*>(k_cache)) + off;
+    v = reinterpret_cast<T*>(loc.host ? m.host_v : reinterpret_cast<unsigned char*>(v_cache)) + off;
+}
+
+// ---------------------------------------------------------------------------
 // Typed element access.
 // ---------------------------------------------------------------------------
 template <typename T> struct Elem;

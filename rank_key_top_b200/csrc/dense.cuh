@@ -28,6 +28,7 @@ struct DenseParams {
     float* out;
     float* qhat;   // workspace [batch][Hq][D]
     float* parts;  // workspace [batch * Hkv][splits][G][D + 2]
+    KvMap kv;
     int num_blocks, Hkv, max_blocks, max_seq_len, splits;
     float scale_log2;
 };
@@ -117,22 +118,33 @@ __global__ void __launch_bounds__(kDenseThreads) dense_split_kernel(const DenseP
             const int ch = warp + m * NW;
             const int tc = t_lo + ch * NCH;  // first token of the chunk, < L
             int pb = row_tbl[tc >> 4];
+            bool okp = true;
             if (pb < 0 || pb >= p.num_blocks) {
                 flag_error(LOKI_DEVERR_BLOCK_ID);
                 pb = 0;
+                okp = false;
             }
-            const int64_t at0 = page_offset(pb, h, p.Hkv, D) * (int64_t)sizeof(T) + (int64_t)(tc & 15) * ROWB;
+            // the chunk lies in one block: one page, on the device or (offloaded) on the host
+            KvPage loc;
+            okp = okp && kv_locate(p.kv, pb, loc);
+            if (!okp) loc = KvPage{0, false};
+            const unsigned char* kb = loc.host ? p.kv.host_k : kbytes;
+            const unsigned char* vb = loc.host ? p.kv.host_v : vbytes;
+            const int64_t at0 = page_offset(loc.page, h, p.Hkv, D) * (int64_t)sizeof(T) + (int64_t)(tc & 15) * ROWB;
 #pragma unroll
             for (int i = 0; i < NCH * PIECES / 32; ++i) {
                 const int pc = lane + 32 * i;
                 const int r = pc / PIECES, w = pc - r * PIECES;
                 const int kv = w >= PIECES / 2, c = w - kv * (PIECES / 2);
-                const bool ok = ch * NCH + r < n;
-                const unsigned char* src = ok ? (kv ? vbytes : kbytes) + at0 + (int64_t)r * ROWB + c * 16 : kbytes;
+                const bool ok = okp && ch * NCH + r < n;
+                const unsigned char* src = ok ? (kv ? vb : kb) + at0 + (int64_t)r * ROWB + c * 16 : kbytes;
                 int off;
                 if constexpr (Geom::MMA) off = Geom::MCore::staged_offset(kv, r, c);
                 else off = r * TB + kv * ROWB + c * 16;
-                cp_async16(dst + off, src, ok);
+                if (loc.host)  // mapped host memory: a plain load, then the shared-memory store
+                    *reinterpret_cast<uint4*>(dst + off) = ok ? *reinterpret_cast<const uint4*>(src) : make_uint4(0, 0, 0, 0);
+                else
+                    cp_async16(dst + off, src, ok);
             }
         }
         cp_async_commit();

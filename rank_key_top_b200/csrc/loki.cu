@@ -7,6 +7,7 @@
 #include <cmath>
 #include <map>
 #include <mutex>
+#include <vector>
 
 #include "cache_kernels.cuh"
 #include "dense.cuh"
@@ -35,7 +36,24 @@ loki_status check_cache(const loki_cache* c) {
         return LOKI_ERR_INVALID_ARG;
     if (c->num_blocks > 0 && (!c->k_cache || !c->v_cache || !c->k_index)) return LOKI_ERR_INVALID_ARG;
     if (!aligned16(c->k_cache) || !aligned16(c->v_cache) || !aligned16(c->k_index)) return LOKI_ERR_INVALID_ARG;
+    if (c->kv_home) {
+        if (c->num_device_pages < 0 || c->num_host_pages < 0) return LOKI_ERR_INVALID_ARG;
+        if (c->num_host_pages > 0 && (!c->k_host || !c->v_host)) return LOKI_ERR_INVALID_ARG;
+        if (!aligned16(c->k_host) || !aligned16(c->v_host)) return LOKI_ERR_INVALID_ARG;
+    }
     return LOKI_OK;
+}
+
+// The kernels' view of where key and value rows live.
+KvMap kv_map_of(const loki_cache* c) {
+    KvMap m;
+    m.home = c->kv_home;
+    m.host_k = c->kv_home ? reinterpret_cast<unsigned char*>(c->k_host) : nullptr;
+    m.host_v = c->kv_home ? reinterpret_cast<unsigned char*>(c->v_host) : nullptr;
+    m.touch = c->kv_touch;
+    m.dev_pages = c->kv_home ? c->num_device_pages : c->num_blocks;
+    m.host_pages = c->kv_home ? c->num_host_pages : 0;
+    return m;
 }
 
 loki_status check_batch(const loki_batch* bt) {
@@ -97,6 +115,7 @@ loki_status launch_append(const loki_cache* cache, const loki_batch* batch, cons
     p.Ak = Ak;
     p.k_cache = cache->k_cache;
     p.v_cache = cache->v_cache;
+    p.kv = kv_map_of(cache);
     p.k_index = cache->k_index;
     p.index_dims = cache->index_dims;
     p.block_table = batch->block_table;
@@ -167,6 +186,7 @@ loki_status launch_decode(const loki_cache* cache, const loki_batch* batch, cons
     SparseParams p;
     p.k_cache = cache->k_cache;
     p.v_cache = cache->v_cache;
+    p.kv = kv_map_of(cache);
     p.k_index = cache->k_index;
     p.block_table = batch->block_table;
     p.seq_lens = batch->seq_lens;
@@ -245,6 +265,7 @@ loki_status loki_prefill_cache(const loki_cache* cache, const loki_batch* batch,
     PrefillParams p;
     p.k_cache = cache->k_cache;
     p.v_cache = cache->v_cache;
+    p.kv = kv_map_of(cache);
     p.k_index = cache->k_index;
     p.index_dims = cache->index_dims;
     p.block_table = batch->block_table;
@@ -285,6 +306,7 @@ loki_status loki_prefill_rotate(const loki_cache* cache, const loki_batch* batch
     RotateParams p;
     p.k_cache = cache->k_cache;
     p.v_cache = cache->v_cache;
+    p.kv = kv_map_of(cache);
     p.k_index = cache->k_index;
     p.block_table = batch->block_table;
     p.seq_lens = batch->seq_lens;
@@ -548,6 +570,7 @@ loki_status loki_dense_attention(const loki_cache* cache, const loki_batch* batc
     DenseParams p;
     p.k_cache = cache->k_cache;
     p.v_cache = cache->v_cache;
+    p.kv = kv_map_of(cache);
     p.block_table = batch->block_table;
     p.seq_lens = batch->seq_lens;
     p.q = q;
@@ -614,3 +637,108 @@ extern "C" loki_status loki_dense_attention_static(const loki_cache* cache, cons
     return loki_dense_attention(cache, batch, q, num_q_heads, P, scale, out, scratch,
                                 (size_t)LOKI_DENSE_STATIC_SCRATCH_BYTES, stream);
 }
+
+// ---------------------------------------------------------------------------
+// Host offload of key and value pages (LRQK page, abstract: only the kept
+// rows of offloaded blocks cross the host link; the blocks the selection
+// keeps hitting are brought to the device between steps).
+// ---------------------------------------------------------------------------
+namespace {
+
+size_t block_page_bytes(const loki_cache* c) {
+    return (size_t)c->num_kv_heads * kBlockTokens * (size_t)c->head_dim * elem_size(c->dtype);
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t loki_offload_plan(int32_t num_blocks, int32_t* kv_home, int32_t* spare_page, const uint32_t* touch,
+                          int32_t max_moves, loki_page_move* moves) {
+    if (num_blocks < 0 || max_moves < 0 || !spare_page || *spare_page < 0) return -1;
+    if (num_blocks > 0 && (!kv_home || !touch)) return -1;
+    if (max_moves > 0 && !moves) return -1;
+    std::vector<int32_t> on_host, on_dev;
+    for (int32_t b = 0; b < num_blocks; ++b) {
+        if (kv_home[b] == *spare_page) return -1;
+        (kv_home[b] < 0 ? on_host : on_dev).push_back(b);
+    }
+    const size_t n = std::min({(size_t)max_moves, on_host.size(), on_dev.size()});
+    // hottest offloaded blocks first, coldest device blocks first; ties to the lower id
+    std::partial_sort(on_host.begin(), on_host.begin() + n, on_host.end(), [&](int32_t a, int32_t b) {
+        return touch[a] != touch[b] ? touch[a] > touch[b] : a < b;
+    });
+    std::partial_sort(on_dev.begin(), on_dev.begin() + n, on_dev.end(), [&](int32_t a, int32_t b) {
+        return touch[a] != touch[b] ? touch[a] < touch[b] : a < b;
+    });
+    int32_t done = 0;
+    for (size_t i = 0; i < n; ++i) {
+        const int32_t in = on_host[i], out = on_dev[i];
+        if (touch[in] <= touch[out]) break;
+        loki_page_move m;
+        m.block_in = in;
+        m.block_out = out;
+        m.host_page = -(kv_home[in] + 1);
+        m.device_page = *spare_page;
+        m.freed_page = kv_home[out];
+        kv_home[in] = m.device_page;
+        kv_home[out] = -(m.host_page + 1);
+        *spare_page = m.freed_page;
+        moves[done++] = m;
+    }
+    return done;
+}
+
+loki_status loki_offload_apply(const loki_cache* cache, const loki_page_move* moves, int32_t num_moves,
+                               const int32_t* kv_home_host, loki_stream_t stream) {
+    loki_status st = check_cache(cache);
+    if (st != LOKI_OK) return st;
+    if (!cache->kv_home || num_moves < 0 || (num_moves > 0 && !moves)) return LOKI_ERR_INVALID_ARG;
+    if (cache->num_blocks > 0 && !kv_home_host) return LOKI_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < num_moves; ++i) {
+        const loki_page_move& m = moves[i];
+        if (m.block_in < 0 || m.block_in >= cache->num_blocks || m.block_out < 0 ||
+            m.block_out >= cache->num_blocks || m.host_page < 0 || m.host_page >= cache->num_host_pages ||
+            m.device_page < 0 || m.device_page >= cache->num_device_pages || m.freed_page < 0 ||
+            m.freed_page >= cache->num_device_pages)
+            return LOKI_ERR_INVALID_ARG;
+    }
+    const size_t pb = block_page_bytes(cache);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    char* dk = reinterpret_cast<char*>(cache->k_cache);
+    char* dv = reinterpret_cast<char*>(cache->v_cache);
+    char* hk = reinterpret_cast<char*>(cache->k_host);
+    char* hv = reinterpret_cast<char*>(cache->v_host);
+    clear_pending_error();
+    bool ok = true;
+    for (int32_t i = 0; i < num_moves && ok; ++i) {
+        const loki_page_move& m = moves[i];
+        // promote block_in into the free page, then demote block_out into the
+        // host page block_in has just left (stream order keeps them apart)
+        ok = cudaMemcpyAsync(dk + m.device_page * pb, hk + m.host_page * pb, pb, cudaMemcpyDefault, s) == cudaSuccess &&
+             cudaMemcpyAsync(dv + m.device_page * pb, hv + m.host_page * pb, pb, cudaMemcpyDefault, s) == cudaSuccess &&
+             cudaMemcpyAsync(hk + m.host_page * pb, dk + m.freed_page * pb, pb, cudaMemcpyDefault, s) == cudaSuccess &&
+             cudaMemcpyAsync(hv + m.host_page * pb, dv + m.freed_page * pb, pb, cudaMemcpyDefault, s) == cudaSuccess;
+    }
+    if (ok && cache->num_blocks > 0)
+        ok = cudaMemcpyAsync(const_cast<int32_t*>(cache->kv_home), kv_home_host, (size_t)cache->num_blocks * 4,
+                             cudaMemcpyHostToDevice, s) == cudaSuccess;
+    if (!ok) {
+        cudaGetLastError();
+        return LOKI_ERR_CUDA;
+    }
+    return LOKI_OK;
+}
+
+loki_status loki_host_device_pointer(void* host, void** device) {
+    if (!host || !device) return LOKI_ERR_INVALID_ARG;
+    void* d = nullptr;
+    if (cudaHostGetDevicePointer(&d, host, 0) != cudaSuccess || !d) {
+        cudaGetLastError();
+        return LOKI_ERR_CUDA;
+    }
+    *device = d;
+    return LOKI_OK;
+}
+
+}  // extern "C"

@@ -34,6 +34,7 @@ struct RotateParams {
     const void* k;  // [batch][Hkv][max_len][D], unrotated
     const void* v;  // [batch][Hkv][max_len][D]
     const float* P;
+    KvMap kv;
     int num_blocks, Hkv, max_blocks, max_seq_len, max_len, index_dims;
     int tiles_per_cta;
 };
@@ -175,8 +176,6 @@ __global__ void __launch_bounds__(kRotThreads) rotate_prefill_tc_kernel(const Ro
     const unsigned char* vsrc =
         reinterpret_cast<const unsigned char*>(p.v) + ((int64_t)b * p.Hkv + h) * p.max_len * (int64_t)(D * 2);
     const int32_t* trow = p.block_table + (int64_t)b * p.max_blocks;
-    __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(p.k_cache);
-    __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(p.v_cache);
     __nv_bfloat16* xc = reinterpret_cast<__nv_bfloat16*>(p.k_index);
     bool ok_all = true;
 
@@ -240,8 +239,11 @@ __global__ void __launch_bounds__(kRotThreads) rotate_prefill_tc_kernel(const Ro
                 if (lane == 0) flag_error(LOKI_DEVERR_BLOCK_ID);
                 continue;
             }
+            __nv_bfloat16 *kd, *vd;
+            kv_rows(p.kv, p.k_cache, p.v_cache, pb, h, p.Hkv, D, kd, vd);
+            if (!vd) continue;
             vbytes[bi] = min(kBlockTokens, L - tb) * (D * 2);
-            vdst[bi] = reinterpret_cast<unsigned char*>(vc + page_offset(pb, h, p.Hkv, D));
+            vdst[bi] = reinterpret_cast<unsigned char*>(vd);
             const unsigned char* src = vsrc + (int64_t)tb * (D * 2);
 #pragma unroll
             for (int j = 0; j < PPL; ++j) {
@@ -253,11 +255,16 @@ __global__ void __launch_bounds__(kRotThreads) rotate_prefill_tc_kernel(const Ro
         const int r = 32 * (warp & 3) + lane;
         const int t = t_base + r;
         int pb = -1;
+        __nv_bfloat16* kpage = nullptr;  // this token's key page
         if (t < L) {
             pb = trow[t >> 4];
             if (pb < 0 || pb >= p.num_blocks) {
                 flag_error(LOKI_DEVERR_BLOCK_ID);
                 pb = -1;
+            } else {
+                __nv_bfloat16* vd;
+                kv_rows(p.kv, p.k_cache, p.v_cache, pb, h, p.Hkv, D, kpage, vd);
+                if (!kpage) pb = -1;
             }
         }
         const bool ok = mbar_wait_bounded(bar, (uint32_t)ti & 1u);
@@ -288,7 +295,7 @@ __global__ void __launch_bounds__(kRotThreads) rotate_prefill_tc_kernel(const Ro
                     const __nv_bfloat16 e1 = __float2bfloat16_rn(__uint_as_float(acc[2 * j + 1]));
                     w[j] = (uint32_t)__bfloat16_as_ushort(e0) | ((uint32_t)__bfloat16_as_ushort(e1) << 16);
                 }
-                __nv_bfloat16* krow = kc + page_offset(pb, h, p.Hkv, D) + row_offset_in_page(t & 15, c0, D);
+                __nv_bfloat16* krow = kpage + row_offset_in_page(t & 15, c0, D);
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
                     *reinterpret_cast<uint4*>(krow + 8 * q) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
@@ -357,8 +364,9 @@ __global__ void __launch_bounds__(256) rotate_prefill_f32_kernel(const RotatePar
 #pragma unroll
     for (int i = 0; i < RPG; ++i) pv[i] = *reinterpret_cast<const float4*>(Ph + (rg * RPG + i) * D + 4 * cq);
     const int64_t src0 = (((int64_t)b * p.Hkv + h) * p.max_len) * D;
-    float* kc = reinterpret_cast<float*>(p.k_cache) + page_offset(pb, h, p.Hkv, D);
-    float* vc = reinterpret_cast<float*>(p.v_cache) + page_offset(pb, h, p.Hkv, D);
+    float *kc, *vc;
+    kv_rows(p.kv, p.k_cache, p.v_cache, pb, h, p.Hkv, D, kc, vc);
+    if (!kc) return;
     float* xc = reinterpret_cast<float*>(p.k_index) + page_offset(pb, h, p.Hkv, p.index_dims);
     const float* ks = reinterpret_cast<const float*>(p.k) + src0;
     const float* vs = reinterpret_cast<const float*>(p.v) + src0;

@@ -67,6 +67,7 @@ struct SparseParams {
     const float* Aq;  // [Hkv][D][index_dims] query factor (asymmetric scorer only)
     float* out;
     int32_t* sel;
+    KvMap kv;
     int num_blocks, Hkv, max_blocks, max_seq_len, index_dims;
     int r, k, W, group_max;
     float scale_log2;
@@ -794,6 +795,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
         __syncthreads();
     }
     const int n_list = misc[72];
+    if (p.kv.touch)  // per block: the kept rows this call gathers from it
+        for (int i = tid; i < n_list; i += kThreads) atomicAdd(p.kv.touch + tbl[list[i] >> 4], 1u);
 
     // ---- optional export of the kept set ----
     if (p.sel) {
@@ -826,22 +829,50 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
             if (m < my_n) {
                 unsigned char* dst = wst + (m % GS) * Geom::CHUNK_BYTES;
                 const int ch = warp + m * kWarps;
-                for (int pc = lane; pc < NCH * PIECES; pc += 32) {
-                    const int n = pc / PIECES, w = pc - n * PIECES;
-                    const int kv = w >= PIECES / 2, c = w - kv * (PIECES / 2);
-                    const int idx = ch * NCH + n;
-                    const bool ok = idx < n_list;
-                    const unsigned char* src = kbytes;
-                    if (ok) {
-                        const int li = list[idx];
-                        const int64_t at = page_offset(tbl[li >> 4], h, p.Hkv, D) * (int64_t)sizeof(T) +
-                                           (int64_t)(li & 15) * ROWB + c * 16;
-                        src = (kv ? vbytes : kbytes) + at;
+                if (!p.kv.home) {
+                    for (int pc = lane; pc < NCH * PIECES; pc += 32) {
+                        const int n = pc / PIECES, w = pc - n * PIECES;
+                        const int kv = w >= PIECES / 2, c = w - kv * (PIECES / 2);
+                        const int idx = ch * NCH + n;
+                        const bool ok = idx < n_list;
+                        const unsigned char* src = kbytes;
+                        if (ok) {
+                            const int li = list[idx];
+                            const int64_t at = page_offset(tbl[li >> 4], h, p.Hkv, D) * (int64_t)sizeof(T) +
+                                               (int64_t)(li & 15) * ROWB + c * 16;
+                            src = (kv ? vbytes : kbytes) + at;
+                        }
+                        int off;
+                        if constexpr (Geom::MMA) off = Geom::MCore::staged_offset(kv, n, c);
+                        else off = n * TB + kv * ROWB + c * 16;
+                        cp_async16(dst + off, src, ok);
                     }
-                    int off;
-                    if constexpr (Geom::MMA) off = Geom::MCore::staged_offset(kv, n, c);
-                    else off = n * TB + kv * ROWB + c * 16;
-                    cp_async16(dst + off, src, ok);
+                } else {
+                    // rows of offloaded blocks come over the host link by plain
+                    // loads of their mapped pages: only the kept rows cross it
+                    for (int pc = lane; pc < NCH * PIECES; pc += 32) {
+                        const int n = pc / PIECES, w = pc - n * PIECES;
+                        const int kv = w >= PIECES / 2, c = w - kv * (PIECES / 2);
+                        const int idx = ch * NCH + n;
+                        bool ok = idx < n_list, host = false;
+                        const unsigned char* src = kbytes;
+                        if (ok) {
+                            const int li = list[idx];
+                            KvPage loc;
+                            ok = kv_locate(p.kv, tbl[li >> 4], loc);
+                            if (ok) {
+                                host = loc.host;
+                                const int64_t at = page_offset(loc.page, h, p.Hkv, D) * (int64_t)sizeof(T) +
+                                                   (int64_t)(li & 15) * ROWB + c * 16;
+                                src = (host ? (kv ? p.kv.host_v : p.kv.host_k) : (kv ? vbytes : kbytes)) + at;
+                            }
+                        }
+                        int off;
+                        if constexpr (Geom::MMA) off = Geom::MCore::staged_offset(kv, n, c);
+                        else off = n * TB + kv * ROWB + c * 16;
+                        if (host) *reinterpret_cast<uint4*>(dst + off) = *reinterpret_cast<const uint4*>(src);
+                        else cp_async16(dst + off, src, ok);
+                    }
                 }
             }
             cp_async_commit();

@@ -44,7 +44,15 @@ _lib = ctypes.CDLL(LIB_PATH)
 class loki_cache(ctypes.Structure):
     _fields_ = [("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p), ("k_index", ctypes.c_void_p),
                 ("num_blocks", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
-                ("head_dim", ctypes.c_int32), ("index_dims", ctypes.c_int32), ("dtype", ctypes.c_int)]
+                ("head_dim", ctypes.c_int32), ("index_dims", ctypes.c_int32), ("dtype", ctypes.c_int),
+                ("kv_home", ctypes.c_void_p), ("k_host", ctypes.c_void_p), ("v_host", ctypes.c_void_p),
+                ("num_device_pages", ctypes.c_int32), ("num_host_pages", ctypes.c_int32),
+                ("kv_touch", ctypes.c_void_p)]
+
+
+class loki_page_move(ctypes.Structure):
+    _fields_ = [("block_in", ctypes.c_int32), ("block_out", ctypes.c_int32), ("host_page", ctypes.c_int32),
+                ("device_page", ctypes.c_int32), ("freed_page", ctypes.c_int32)]
 
 
 class loki_batch(ctypes.Structure):
@@ -82,6 +90,10 @@ _SIGS = {
     "loki_dense_workspace_bytes": (_SZ, [_C, _B, _I32]),
     "loki_dense_attention": (ctypes.c_int, [_C, _B, _P, _I32, _P, ctypes.c_float, _P, _P, _SZ, _P]),
     "loki_dense_attention_static": (ctypes.c_int, [_C, _B, _P, _I32, _P, ctypes.c_float, _P, _P]),
+    "loki_offload_plan": (_I32, [_I32, _P, ctypes.POINTER(ctypes.c_int32), _P, _I32,
+                                 ctypes.POINTER(loki_page_move)]),
+    "loki_offload_apply": (ctypes.c_int, [_C, ctypes.POINTER(loki_page_move), _I32, _P, _P]),
+    "loki_host_device_pointer": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_void_p)]),
     "loki_device_error": (ctypes.c_int, [_I32, ctypes.POINTER(ctypes.c_uint32)]),
     "loki_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "loki_abi_version": (_I32, []),
@@ -144,6 +156,47 @@ class Cache:
         self.x = torch.empty(max(ibytes, 16), dtype=torch.uint8, device=device)
         self.struct = loki_cache(self.k.data_ptr(), self.v.data_ptr(), self.x.data_ptr(), num_blocks,
                                  num_kv_heads, head_dim, index_dims, code)
+
+
+class OffloadCache(Cache):
+    """A cache whose key and value rows are split between device pages and
+    pinned host pages (the key index stays on the device): block b's rows are
+    device page home[b] for home[b] >= 0, host page -(home[b] + 1) otherwise.
+    device_pages must leave one device page unused (the planner's spare).
+
+    Keeps the host copy of the map (`home`), the spare page and the per-block
+    touch counters (`touch`, device) that the sparse decode fills."""
+
+    def __init__(self, num_blocks, num_kv_heads, head_dim, dtype, home, device_pages, host_pages,
+                 device="cuda", index_dims=64):
+        home = torch.as_tensor(home, dtype=torch.int32).cpu().contiguous()
+        if home.numel() != num_blocks:
+            raise ValueError("home needs one entry per block")
+        code = dtype_code(dtype)
+        dbytes = loki_cache_bytes(device_pages, num_kv_heads, head_dim, code)
+        hbytes = loki_cache_bytes(host_pages, num_kv_heads, head_dim, code)
+        ibytes = loki_index_bytes(num_blocks, num_kv_heads, index_dims, code)
+        used = set(int(e) for e in home.tolist() if e >= 0)
+        free = [pg for pg in range(device_pages) if pg not in used]
+        if not free:
+            raise ValueError("device_pages leaves no spare page")
+        self.dtype = dtype
+        self.index_dims = index_dims
+        self.page_bytes = loki_cache_bytes(1, num_kv_heads, head_dim, code)
+        self.k = torch.empty(max(dbytes, 16), dtype=torch.uint8, device=device)
+        self.v = torch.empty(max(dbytes, 16), dtype=torch.uint8, device=device)
+        self.x = torch.empty(max(ibytes, 16), dtype=torch.uint8, device=device)
+        self.hk = torch.empty(max(hbytes, 16), dtype=torch.uint8, pin_memory=True)
+        self.hv = torch.empty(max(hbytes, 16), dtype=torch.uint8, pin_memory=True)
+        self.home = home
+        self.spare = ctypes.c_int32(free[0])
+        self.home_dev = home.to(device)
+        self.touch = torch.zeros(max(num_blocks, 1), dtype=torch.int32, device=device)
+        self.struct = loki_cache(self.k.data_ptr(), self.v.data_ptr(), self.x.data_ptr(), num_blocks,
+                                 num_kv_heads, head_dim, index_dims, code,
+                                 self.home_dev.data_ptr(), loki_host_device_pointer(self.hk),
+                                 loki_host_device_pointer(self.hv), device_pages, host_pages,
+                                 self.touch.data_ptr())
 
 
 class Batch:
@@ -312,3 +365,46 @@ def loki_abi_version():
 def raw():
     """The loaded ctypes library (for ABI tests)."""
     return _lib
+
+
+# --------------------------------------------------------------------------
+# Host offload (OffloadCache)
+# --------------------------------------------------------------------------
+
+def loki_host_device_pointer(host_tensor):
+    """Device address of a pinned host tensor's memory."""
+    out = ctypes.c_void_p()
+    _check("loki_host_device_pointer", _lib.loki_host_device_pointer(ctypes.c_void_p(host_tensor.data_ptr()),
+                                                                     ctypes.byref(out)))
+    return out.value
+
+
+def loki_offload_plan(home, spare, touch, max_moves):
+    """home: int32 CPU tensor (updated in place); spare: ctypes.c_int32
+    (updated); touch: CPU tensor of per-block counts. Returns the moves."""
+    assert home.dtype == torch.int32 and home.is_contiguous()
+    touch = touch.to(torch.int32).contiguous()
+    moves = (loki_page_move * max(max_moves, 1))()
+    n = _lib.loki_offload_plan(home.numel(), ctypes.c_void_p(home.data_ptr()), ctypes.byref(spare),
+                               ctypes.c_void_p(touch.data_ptr()), max_moves, moves)
+    if n < 0:
+        raise LokiError("loki_offload_plan", LOKI_ERR_INVALID_ARG)
+    return [moves[i] for i in range(n)]
+
+
+def loki_offload_apply(cache, moves, home, stream=None):
+    arr = (loki_page_move * max(len(moves), 1))(*moves)
+    _check("loki_offload_apply", _lib.loki_offload_apply(ctypes.byref(cache.struct), arr, len(moves),
+                                                         ctypes.c_void_p(home.data_ptr()), _stream(stream)))
+
+
+def offload_rebalance(cache, max_moves, stream=None):
+    """Between decode steps: read the touch counts, plan up to max_moves
+    swaps, issue them on the stream and clear the counts. Returns the moves."""
+    stream = torch.cuda.current_stream() if stream is None else stream
+    with torch.cuda.stream(stream):
+        touch = cache.touch.cpu()
+        moves = loki_offload_plan(cache.home, cache.spare, touch, max_moves)
+        loki_offload_apply(cache, moves, cache.home, stream=stream)
+        cache.touch.zero_()
+    return moves

@@ -36,7 +36,7 @@ def test_library_exports_every_declared_symbol(loki):
     for name in declared_symbols():
         assert hasattr(lib, name), name
     assert sorted(loki.EXPORTED) == declared_symbols()
-    assert loki.loki_abi_version() == 4
+    assert loki.loki_abi_version() == 5
 
 
 def test_status_strings(loki):
