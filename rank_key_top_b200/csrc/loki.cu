@@ -201,6 +201,8 @@ loki_status launch_decode(const loki_cache* cache, const loki_batch* batch, cons
     p.max_blocks = batch->max_blocks_per_seq;
     p.max_seq_len = batch->max_seq_len;
     p.index_dims = cache->index_dims;
+    p.batch = batch->batch;
+    p.longest_first = 0;
     p.r = r;
     p.k = k;
     p.W = recent_window;

@@ -69,6 +69,8 @@ struct SparseParams {
     int32_t* sel;
     KvMap kv;
     int num_blocks, Hkv, max_blocks, max_seq_len, index_dims;
+    int batch;
+    int longest_first;  // clusters take the sequences longest first (batch <= 64)
     int r, k, W, group_max;
     float scale_log2;
     int C;           // CTAs per (sequence, kv head), = cluster size
@@ -206,10 +208,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     cg::cluster_group cluster = cg::this_cluster();
 
     const int crank = (int)cluster.block_rank();
-    const int pair = blockIdx.y;
-    const int b = pair / p.Hkv;
-    const int h = pair - b * p.Hkv;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int h = (int)blockIdx.y % p.Hkv;
     const int Hq = p.Hkv * G;
 
     uint32_t* keys = reinterpret_cast<uint32_t*>(smem + p.off_keys);
@@ -231,7 +231,31 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     int32_t* misc = reinterpret_cast<int32_t*>(smem + p.off_misc);
     // misc: [0] boundary digit, [1] count above it, [8..39] suffix-sum scratch,
     //       [40..55] warp kept counts, [56..71] warp equal counts, [72] list length,
-    //       [104..111] slab energies (slab scorer), [128..255] chosen dims (MAG)
+    //       [73] the sequence (longest first), [104..111] slab energies (slab
+    //       scorer), [128..255] chosen dims (MAG)
+
+    // ---- which sequence ----
+    // Over several waves of clusters the sequences go longest first (ties:
+    // the lower index), so that the short ones fill the last wave: cluster
+    // row j takes the sequence of rank j. Warp 0 ranks up to 64 lengths.
+    int b = (int)blockIdx.y / p.Hkv;
+    if (p.longest_first) {
+        if (warp == 0) {
+            const int l0 = lane < p.batch ? p.seq_lens[lane] : 0;
+            const int l1 = lane + 32 < p.batch ? p.seq_lens[lane + 32] : 0;
+            int r0 = 0, r1 = 0;
+            for (int i = 0; i < p.batch; ++i) {
+                const int li = __shfl_sync(kFull, i < 32 ? l0 : l1, i & 31);
+                r0 += (li > l0 || (li == l0 && i < lane)) ? 1 : 0;
+                r1 += (li > l1 || (li == l1 && i < lane + 32)) ? 1 : 0;
+            }
+            if (lane < p.batch && r0 == b) misc[73] = lane;
+            if (lane + 32 < p.batch && r1 == b) misc[73] = lane + 32;
+        }
+        __syncthreads();
+        b = misc[73];
+    }
+    const int pair = b * p.Hkv + h;
 
     // ---- sequence geometry ----
     // CTA crank owns the fixed token range [crank * cta_tokens, + cta_tokens)

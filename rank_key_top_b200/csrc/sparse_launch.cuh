@@ -59,28 +59,6 @@ inline cudaError_t ensure_smem_attr(const void* kern, int bytes) {
     return cudaSuccess;
 }
 
-// Whether at least one cluster of this shape can be resident on the current
-// device, cached per device, kernel instantiation, cluster size and
-// shared-memory size.
-template <typename K>
-bool cluster_fits(K kern, const cudaLaunchConfig_t& cfg, std::map<std::tuple<int, int, int>, bool>& known,
-                  std::mutex& mu) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    const std::tuple<int, int, int> key(dev, (int)cfg.gridDim.x, (int)cfg.dynamicSmemBytes);
-    std::lock_guard<std::mutex> lock(mu);
-    auto it = known.find(key);
-    if (it != known.end()) return it->second;
-    int n = 0;
-    cudaLaunchConfig_t probe = cfg;
-    probe.gridDim = dim3(cfg.gridDim.x, 1, 1);
-    const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kern, &probe);
-    if (e != cudaSuccess) cudaGetLastError();
-    const bool fits = e == cudaSuccess && n > 0;
-    known[key] = fits;
-    return fits;
-}
-
 // Shared-memory layout of one CTA for C CTAs per (sequence, kv head), with a
 // key-index ring of ring_per_warp bytes per warp.
 template <typename T, int D, int G>
@@ -140,32 +118,89 @@ bool sparse_layout_fit(SparseParams& p, int max_seq_len, int smem_optin) {
     return false;
 }
 
-// Cluster size: enough CTAs that each holds at most kCtaTokenCap tokens and
-// the layout fits in shared memory, then the largest size that still fits
-// every cluster on the GPU at once (one CTA per SM), keeps at least 512
-// tokens per CTA and whose layout fits (rank 0's merge slots grow with the
-// cluster). Returns -1 when no size up to 16 fits.
-template <typename T, int D, int G>
-int choose_cluster(SparseParams& p, int max_seq_len, int pairs, int sms, int smem_optin) {
+// A CTA's fixed cost (launch share, prologue, select, merge) in units of the
+// time it takes to stream one 16-token block; measured on B200 at about
+// 20 us against 50 ns per block for rank 32.
+constexpr int kCtaFixedBlocks = 400;
+
+// Cluster size. The smallest size C0 whose CTAs hold at most kCtaTokenCap
+// tokens each and whose layout fits in shared memory; then, among C0 and the
+// larger sizes whose layout fits and that keep at least 512 tokens per CTA,
+// the one with the least modelled time
+//   waves(C) * (kCtaFixedBlocks + blocks per CTA(C)),
+// waves(C) = ceil(pairs / resident(C)), where resident(C) is how many
+// clusters of C CTAs the GPU holds at once (ties: the smaller C).
+// resident(C, smem) returns that count from the device (0: the cluster never
+// fits), or -1 when unknown, in which case sms / C stands in for it. Returns
+// -1 when no size up to 16 fits.
+template <typename T, int D, int G, typename R>
+int choose_cluster(SparseParams& p, int max_seq_len, int pairs, int sms, int smem_optin, R&& resident) {
     const int nblk = (max_seq_len + kBlockTokens - 1) / kBlockTokens;
     const int cap_blocks = kCtaTokenCap / kBlockTokens;
-    int C = std::max(1, (nblk + cap_blocks - 1) / cap_blocks);
-    for (;; ++C) {
-        if (C > 16) return -1;
-        p.C = C;
+    int C0 = std::max(1, (nblk + cap_blocks - 1) / cap_blocks);
+    for (;; ++C0) {
+        if (C0 > 16) return -1;
+        p.C = C0;
         if (sparse_layout_fit<T, D, G>(p, max_seq_len, smem_optin)) break;
     }
-    int best = C;
-    for (int cand = C + 1; cand <= 16; ++cand) {
-        if ((int64_t)pairs * cand > sms) break;
-        if (nblk / cand < 32) break;
+    int best = -1;
+    int64_t best_cost = 0;
+    for (int cand = C0; cand <= 16; ++cand) {
+        if (cand > C0 && nblk / cand < 32) break;
         p.C = cand;
-        if (sparse_layout_fit<T, D, G>(p, max_seq_len, smem_optin)) best = cand;
+        if (!sparse_layout_fit<T, D, G>(p, max_seq_len, smem_optin)) continue;
+        int res = resident(cand, p.smem_bytes);
+        if (res < 0) res = sms / cand;
+        if (res < 1) continue;
+        const int64_t waves = (pairs + res - 1) / res;
+        const int64_t cost = waves * (kCtaFixedBlocks + (nblk + cand - 1) / cand);
+        if (best < 0 || cost < best_cost) {
+            best = cand;
+            best_cost = cost;
+        }
     }
-    C = best;
-    p.C = C;
+    if (best < 0) return -1;
+    p.C = best;
     sparse_layout_fit<T, D, G>(p, max_seq_len, smem_optin);
-    return C;
+    return best;
+}
+
+template <typename T, int D, int G>
+int choose_cluster(SparseParams& p, int max_seq_len, int pairs, int sms, int smem_optin) {
+    return choose_cluster<T, D, G>(p, max_seq_len, pairs, sms, smem_optin, [](int, int) { return -1; });
+}
+
+// Clusters of `cluster` CTAs of this kernel with `smem` bytes of shared
+// memory each that the current device holds at once, cached per device,
+// cluster size and shared-memory size (0 when none fits or the query fails).
+template <typename K>
+int resident_clusters(K kern, int cluster, int smem, std::map<std::tuple<int, int, int>, int>& known,
+                      std::mutex& mu) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const std::tuple<int, int, int> key(dev, cluster, smem);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = known.find(key);
+    if (it != known.end()) return it->second;
+    cudaLaunchConfig_t probe = {};
+    probe.gridDim = dim3(cluster, 1, 1);
+    probe.blockDim = dim3(kThreads, 1, 1);
+    probe.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = cluster;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    probe.attrs = &attr;
+    probe.numAttrs = 1;
+    int n = 0;
+    const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kern, &probe);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+    }
+    known[key] = n;
+    return n;
 }
 
 // Whether the decode kernel has a cluster size and layout for this shape
@@ -196,10 +231,9 @@ struct SparseLaunch {
     template <int SC>
     static loki_status run_kernel(SparseParams p, int pairs, int max_seq_len, const DeviceInfo& di,
                                   cudaStream_t stream, bool programmatic) {
-        if (choose_cluster<T, D, G>(p, max_seq_len, pairs, di.sms, di.max_smem_optin) < 1)
-            return LOKI_ERR_UNSUPPORTED;
         auto kern = sparse_decode_kernel<T, D, G, SC>;
         // per device: the shared-memory opt-in and non-portable cluster sizes
+        // (both before the residency queries of the cluster choice)
         if (ensure_smem_attr((const void*)kern, di.max_smem_optin) != cudaSuccess) return LOKI_ERR_CUDA;
         {
             static std::mutex mu;
@@ -215,6 +249,13 @@ struct SparseLaunch {
             }
             if (it->second != cudaSuccess) return LOKI_ERR_CUDA;
         }
+        static std::map<std::tuple<int, int, int>, int> resident;
+        static std::mutex resident_mu;
+        auto res = [&](int c, int smem) { return resident_clusters(kern, c, smem, resident, resident_mu); };
+        if (choose_cluster<T, D, G>(p, max_seq_len, pairs, di.sms, di.max_smem_optin, res) < 1)
+            return LOKI_ERR_UNSUPPORTED;
+        // several waves of clusters: longest sequences first
+        p.longest_first = p.batch > 1 && p.batch <= 64 && pairs > res(p.C, p.smem_bytes) ? 1 : 0;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(p.C, pairs, 1);
         cfg.blockDim = dim3(kThreads, 1, 1);
@@ -233,9 +274,7 @@ struct SparseLaunch {
         cfg.attrs = attr;
         cfg.numAttrs = programmatic ? 2 : 1;
         // a cluster that can never be resident is reported, not launched
-        static std::map<std::tuple<int, int, int>, bool> known;
-        static std::mutex known_mu;
-        if (!cluster_fits(kern, cfg, known, known_mu)) return LOKI_ERR_UNSUPPORTED;
+        if (res(p.C, p.smem_bytes) < 1) return LOKI_ERR_UNSUPPORTED;
         if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) {
             cudaGetLastError();  // reported here, not by a later call
             return LOKI_ERR_CUDA;

@@ -242,6 +242,17 @@ def make_workload(spec: Spec, pairs=None) -> Workload:
                     kps, table, num_blocks, bases)
 
 
+def draw_anisotropic_queries(spec: Spec, h: int, n: int, tag: int) -> np.ndarray:
+    """n original-basis query rows of kv head h whose spectrum runs against
+    the keys': z diag(tau) U^T with tau the keys' scales sigma in reverse
+    order, fp64. These queries weight most the directions that the keys'
+    variance ranks lowest, the setting in which asymmetric query/key factors
+    and key PCA rank tokens differently (SAKI page, abstract)."""
+    basis = head_basis(spec, h)
+    z = torch.randn(n, spec.head_dim, generator=_gen(spec.seed, 11, h, tag), dtype=torch.float64).numpy()
+    return (z * basis.sigma[::-1]) @ basis.U.T
+
+
 def draw_new_tokens(spec: Spec, step: int):
     """Unrotated keys and values of one decode step, [B, Hkv, d] in cache type."""
     B, Hkv, d = spec.batch, spec.num_kv_heads, spec.head_dim

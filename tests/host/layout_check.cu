@@ -87,7 +87,9 @@ void check(const char* tname, int sms, int optin) {
                 CHECK(p.off_misc - p.off_part >= G * D * 4);  // the asymmetric scorer's query
                 CHECK(p.smem_bytes - p.off_misc >= 256 * 4);  // misc words, then the chosen dims
                 CHECK(kSelDims + D <= 256);
-                // spread: a cluster larger than needed only while every cluster still fits at once
+                // spread: a cluster larger than needed only where it shortens the
+                // modelled time (waves of resident clusters, sms / C of them, times
+                // the blocks of one CTA) and keeps 512 tokens per CTA
                 SparseParams q = {};
                 q.r = r;
                 const int cap_blocks = kCtaTokenCap / kBlockTokens;
@@ -98,7 +100,15 @@ void check(const char* tname, int sms, int optin) {
                     if (sparse_layout_fit<T, D, G>(q, L, optin)) break;
                 }
                 CHECK(C >= cmin);
-                if (C > cmin) CHECK((long)pairs * C <= sms);
+                if (C > cmin) {
+                    auto cost = [&](int c) {
+                        const long res = sms / c;
+                        return res < 1 ? (1L << 62)
+                                       : ((pairs + res - 1) / res) * (long)(kCtaFixedBlocks + (nblk + c - 1) / c);
+                    };
+                    CHECK(cost(C) < cost(cmin));
+                    CHECK(nblk / C >= 32);
+                }
             }
     if (shortest_unsupported < (1 << 30))
         std::printf("unsupported from L=%d: T=%s D=%d G=%d\n", shortest_unsupported, tname, D, G);

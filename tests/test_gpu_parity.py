@@ -64,6 +64,9 @@ EDGE = {
     "d64-bf16-g4": dict(num_q_heads=8, num_kv_heads=2, head_dim=64, seq_lens=[2500, 1], r=48, k=40,
                         recent_window=5),
     "many-pairs": dict(num_q_heads=32, num_kv_heads=8, seq_lens=[1500] * 4, k=100, recent_window=16),
+    # more pairs than resident clusters: the sequences go longest first (ties, empty ones)
+    "many-waves-ragged": dict(num_q_heads=32, num_kv_heads=32, seq_lens=[5, 3000, 0, 3000, 17, 1200, 3000, 64,
+                                                                         2999, 1], k=40, recent_window=2),
 }
 
 
