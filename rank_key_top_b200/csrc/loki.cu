@@ -213,6 +213,40 @@ loki_status launch_decode(const loki_cache* cache, const loki_batch* batch, cons
                                       scorer);
 }
 
+// The driver's tensor-map encoder, looked up once through the runtime (the
+// library links only the runtime).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn() {
+    static EncodeTiledFn fn = []() -> EncodeTiledFn {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        return reinterpret_cast<EncodeTiledFn>(ptr);
+    }();
+    return fn;
+}
+
+// Tensor map of key rows [rows][D] bf16 (row stride D * 2 bytes) with a
+// 64-column x box_rows box and the 128-byte swizzle of the MMA operand; rows
+// past the end read as zero.
+bool encode_key_map(CUtensorMap* map, const void* keys, int64_t rows, int D, int box_rows) {
+    EncodeTiledFn fn = encode_tiled_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(keys), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 extern "C" {
@@ -325,16 +359,29 @@ loki_status loki_prefill_rotate(const loki_cache* cache, const loki_batch* batch
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int D = cache->head_dim;
     if (cache->dtype == LOKI_BF16) {
-        // enough tiles per CTA that a CTA's split of P is reused, with about
-        // two CTAs per SM in flight
-        const int tiles = (batch->max_seq_len + kRotTile - 1) / kRotTile;
-        const int64_t want = 2LL * std::max(1, device_info().sms);
-        p.tiles_per_cta = (int)std::max<int64_t>(1, ((int64_t)tiles * pairs + want - 1) / want);
-        const dim3 grid((tiles + p.tiles_per_cta - 1) / p.tiles_per_cta, pairs);
+        // the keys as a 2-D tensor [batch * Hkv * max_len rows][D], box 64 x 128, 128-byte swizzle
+        const int64_t rows = (int64_t)pairs * max_len;
+        if (rows + kRotTile > INT32_MAX) return LOKI_ERR_UNSUPPORTED;
+        CUtensorMap tmap, kmap;
+        if (!encode_key_map(&tmap, k, rows, D, kRotTile)) return LOKI_ERR_CUDA;
+        // the key cache's device pages as [pages * Hkv * 16 rows][D], the store side
+        const int64_t dev_pages = cache->kv_home ? cache->num_device_pages : cache->num_blocks;
+        const int64_t krows = std::max<int64_t>(1, dev_pages) * cache->num_kv_heads * kBlockTokens;
+        if (krows > INT32_MAX) return LOKI_ERR_UNSUPPORTED;
+        if (!encode_key_map(&kmap, cache->k_cache, krows, D, kBlockTokens)) return LOKI_ERR_CUDA;
+        p.tiles_per_pair = (batch->max_seq_len + kRotTile - 1) / kRotTile;
+        p.total_tiles = (int64_t)pairs * p.tiles_per_pair;
         auto launch = [&](auto kern, int smem) {
             if (ensure_smem_attr((const void*)kern, smem) != cudaSuccess) return LOKI_ERR_CUDA;
+            int per_sm = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kRotThreads, smem) != cudaSuccess ||
+                per_sm < 1) {
+                cudaGetLastError();
+                return LOKI_ERR_CUDA;
+            }
+            const int64_t ctas = std::min<int64_t>(p.total_tiles, (int64_t)per_sm * std::max(1, device_info().sms));
             clear_pending_error();
-            kern<<<grid, kRotThreads, smem, s>>>(p);
+            kern<<<(unsigned)ctas, kRotThreads, smem, s>>>(p, tmap, kmap);
             return launch_status();
         };
         if (D == 64) return launch(rotate_prefill_tc_kernel<64>, rotate_smem_bytes<64>());
