@@ -125,26 +125,39 @@ __global__ void __launch_bounds__(kDenseThreads) dense_split_kernel(const DenseP
                 okp = false;
             }
             // the chunk lies in one block: one page, on the device or (offloaded) on the host
-            KvPage loc;
-            okp = okp && kv_locate(p.kv, pb, loc);
-            if (!okp) loc = KvPage{0, false};
-            const unsigned char* kb = loc.host ? p.kv.host_k : kbytes;
-            const unsigned char* vb = loc.host ? p.kv.host_v : vbytes;
-            const int64_t at0 = page_offset(loc.page, h, p.Hkv, D) * (int64_t)sizeof(T) + (int64_t)(tc & 15) * ROWB;
+            KvPage loc{pb, false};
+            if (p.kv.home) {
+                okp = okp && kv_locate(p.kv, pb, loc);
+                if (!okp) loc = KvPage{0, false};
+            }
+            if (!loc.host) {
+                const int64_t at0 = page_offset(loc.page, h, p.Hkv, D) * (int64_t)sizeof(T) + (int64_t)(tc & 15) * ROWB;
 #pragma unroll
-            for (int i = 0; i < NCH * PIECES / 32; ++i) {
-                const int pc = lane + 32 * i;
-                const int r = pc / PIECES, w = pc - r * PIECES;
-                const int kv = w >= PIECES / 2, c = w - kv * (PIECES / 2);
-                const bool ok = okp && ch * NCH + r < n;
-                const unsigned char* src = ok ? (kv ? vb : kb) + at0 + (int64_t)r * ROWB + c * 16 : kbytes;
-                int off;
-                if constexpr (Geom::MMA) off = Geom::MCore::staged_offset(kv, r, c);
-                else off = r * TB + kv * ROWB + c * 16;
-                if (loc.host)  // mapped host memory: a plain load, then the shared-memory store
-                    *reinterpret_cast<uint4*>(dst + off) = ok ? *reinterpret_cast<const uint4*>(src) : make_uint4(0, 0, 0, 0);
-                else
+                for (int i = 0; i < NCH * PIECES / 32; ++i) {
+                    const int pc = lane + 32 * i;
+                    const int r = pc / PIECES, w = pc - r * PIECES;
+                    const int kv = w >= PIECES / 2, c = w - kv * (PIECES / 2);
+                    const bool ok = okp && ch * NCH + r < n;
+                    const unsigned char* src = ok ? (kv ? vbytes : kbytes) + at0 + (int64_t)r * ROWB + c * 16 : kbytes;
+                    int off;
+                    if constexpr (Geom::MMA) off = Geom::MCore::staged_offset(kv, r, c);
+                    else off = r * TB + kv * ROWB + c * 16;
                     cp_async16(dst + off, src, ok);
+                }
+            } else {  // mapped host memory: plain loads, then the shared-memory stores
+                const int64_t at0 = page_offset(loc.page, h, p.Hkv, D) * (int64_t)sizeof(T) + (int64_t)(tc & 15) * ROWB;
+                for (int i = 0; i < NCH * PIECES / 32; ++i) {
+                    const int pc = lane + 32 * i;
+                    const int r = pc / PIECES, w = pc - r * PIECES;
+                    const int kv = w >= PIECES / 2, c = w - kv * (PIECES / 2);
+                    const bool ok = ch * NCH + r < n;
+                    int off;
+                    if constexpr (Geom::MMA) off = Geom::MCore::staged_offset(kv, r, c);
+                    else off = r * TB + kv * ROWB + c * 16;
+                    *reinterpret_cast<uint4*>(dst + off) =
+                        ok ? *reinterpret_cast<const uint4*>((kv ? p.kv.host_v : p.kv.host_k) + at0 + (int64_t)r * ROWB + c * 16)
+                           : make_uint4(0, 0, 0, 0);
+                }
             }
         }
         cp_async_commit();
