@@ -618,24 +618,26 @@ def main():
         finish(world)
         return
 
-    # end to end through the public API: pinned host inputs in, output back
-    # a step's inputs (q, k_new, v_new) travel as one pinned buffer and one copy
-    nq, nk, nv = qs[0].numel(), ks[0].numel(), vs[0].numel()
-    hin = [torch.cat([q.flatten(), k.flatten(), v.flatten()]).cpu().pin_memory() for q, k, v in zip(qs, ks, vs)]
-    din = torch.empty(nq + nk + nv, dtype=qs[0].dtype, device=dev)
-    dq = din[:nq].view(qs[0].shape)
-    dk = din[nq:nq + nk].view(ks[0].shape)
-    dv = din[nq + nk:].view(vs[0].shape)
+    # end to end through the public API: loki_decode_step_host takes the step's
+    # inputs (q, k_new, v_new) in pinned host memory, copies them in, runs the
+    # step and copies the output back, all on the stream; one graph per input slot
+    hq = [q.cpu().pin_memory() for q in qs]
+    hk = [k.cpu().pin_memory() for k in ks]
+    hv = [v.cpu().pin_memory() for v in vs]
     hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    staging = torch.empty(loki.loki_decode_step_host_bytes(cache, batch, spec.num_q_heads), dtype=torch.uint8,
+                          device=dev)
     e0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     e1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     e2e_graphs = []
-    for i in range(pool):   # host copies in, the step, the output back: one graph per input slot
+    for i in range(pool):
+        loki.loki_decode_step_host(cache, batch, hk[i], hv[i], hq[i], P, spec.r, spec.k, hout, staging,
+                                   k_per_seq=kps, recent_window=spec.recent_window, stream=stream)
+        torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            din.copy_(hin[i], non_blocking=True)
-            step(i, dq, dk, dv)
-            hout.copy_(out, non_blocking=True)
+            loki.loki_decode_step_host(cache, batch, hk[i], hv[i], hq[i], P, spec.r, spec.k, hout, staging,
+                                       k_per_seq=kps, recent_window=spec.recent_window, stream=stream)
         e2e_graphs.append(g)
     for phase in ("warm", "timed"):
         n = args.warmup if phase == "warm" else K
@@ -648,8 +650,9 @@ def main():
                 e1[i].record(stream)
         torch.cuda.synchronize()
     e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(e0, e1)), world)
-    h2d = din.numel() * din.element_size()
-    d2h = out.numel() * out.element_size()
+    h2d = sum(t.numel() * t.element_size() for t in (hq[0], hk[0], hv[0]))
+    d2h = hout.numel() * hout.element_size()
+    assert loki.loki_device_error() == 0
 
     # the GPU's own dense-attention kernel on the same cache, same conditions
     ws = torch.empty(loki.loki_dense_workspace_bytes(cache, batch, spec.num_q_heads), dtype=torch.uint8,
@@ -755,7 +758,9 @@ def main():
                      "launch_ms": decode_ms / K},
         "cpu_baseline": cb,
         "e2e": {"value": world * K / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+                "d2h_bytes_per_step": d2h,
+                "path": "loki_decode_step_host: q, k_new, v_new from pinned host buffers, the step, out back to a "
+                        "pinned host buffer; one CUDA graph per input slot"},
         "clocks": clocks,
         "gpu_launches": 2 * K,
         "step_launch": "CUDA graph per step: loki_decode_step (append kernel, then the decode kernel as its "

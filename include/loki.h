@@ -369,6 +369,32 @@ LOKI_API loki_status loki_decode_step(const loki_cache* cache, const loki_batch*
                              void* workspace, size_t workspace_bytes,
                              loki_stream_t stream);
 
+/* Bytes of the device staging buffer loki_decode_step_host needs for these
+ * sizes: the step's k_new, v_new and q (cache dtype) and its output (fp32),
+ * each region 256-byte aligned; 0 for invalid arguments. */
+LOKI_API size_t loki_decode_step_host_bytes(const loki_cache* cache, const loki_batch* batch,
+                                            int32_t num_q_heads);
+
+/* loki_decode_step for a caller that holds the step's inputs and output in
+ * host memory. k_new_host, v_new_host ([batch][num_kv_heads][head_dim]) and
+ * q_host ([batch][num_q_heads][head_dim]), all in the cache dtype, are copied
+ * into `staging` (device, loki_decode_step_host_bytes bytes, 256-byte
+ * aligned), the step runs as loki_decode_step with the same remaining
+ * arguments (no kept-index export), and the output ([batch][num_q_heads]
+ * [head_dim] fp32) is copied back to out_host: one cudaMemcpyAsync per buffer,
+ * all on `stream`. With pinned host memory the call is asynchronous and the
+ * host buffers must stay untouched until the stream has passed the copies;
+ * pageable memory makes the copies synchronous with the host. Every argument
+ * is checked before anything is issued; an error issues nothing. The caller
+ * owns every buffer; the library allocates nothing. */
+LOKI_API loki_status loki_decode_step_host(const loki_cache* cache, const loki_batch* batch,
+                                           const void* k_new_host, const void* v_new_host,
+                                           const void* q_host, int32_t num_q_heads, const float* P,
+                                           int32_t r, int32_t k, const int32_t* k_per_seq,
+                                           int32_t recent_window, loki_group_reduce group_reduce,
+                                           float scale, float* out_host, void* staging,
+                                           size_t staging_bytes, loki_stream_t stream);
+
 /* Largest max_seq_len loki_decode_attention accepts for this cache shape
  * (262144 tokens). Some group sizes fit less in a CTA's shared memory: for
  * those, longer sequences are rejected with LOKI_ERR_UNSUPPORTED before any

@@ -545,6 +545,75 @@ loki_status loki_decode_attention_asym(const loki_cache* cache, const loki_batch
                          selected_idx, reinterpret_cast<cudaStream_t>(stream), false, kScoreAsym, A_q);
 }
 
+// Regions of loki_decode_step_host's staging buffer: k_new, v_new, q, out.
+struct StepStaging {
+    size_t k_off, v_off, q_off, o_off, k_bytes, q_bytes, o_bytes, total;
+};
+static bool step_staging(const loki_cache* cache, const loki_batch* batch, int32_t num_q_heads, StepStaging* st) {
+    if (check_cache(cache) != LOKI_OK || check_batch(batch) != LOKI_OK || num_q_heads < 1) return false;
+    const size_t es = elem_size(cache->dtype), D = (size_t)cache->head_dim, B = (size_t)batch->batch;
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    st->k_bytes = B * cache->num_kv_heads * D * es;
+    st->q_bytes = B * (size_t)num_q_heads * D * es;
+    st->o_bytes = B * (size_t)num_q_heads * D * 4;
+    st->k_off = 0;
+    st->v_off = up(st->k_bytes);
+    st->q_off = st->v_off + up(st->k_bytes);
+    st->o_off = st->q_off + up(st->q_bytes);
+    st->total = st->o_off + up(st->o_bytes);
+    return true;
+}
+
+size_t loki_decode_step_host_bytes(const loki_cache* cache, const loki_batch* batch, int32_t num_q_heads) {
+    StepStaging st;
+    return step_staging(cache, batch, num_q_heads, &st) ? st.total : 0;
+}
+
+loki_status loki_decode_step_host(const loki_cache* cache, const loki_batch* batch, const void* k_new_host,
+                                  const void* v_new_host, const void* q_host, int32_t num_q_heads, const float* P,
+                                  int32_t r, int32_t k, const int32_t* k_per_seq, int32_t recent_window,
+                                  loki_group_reduce group_reduce, float scale, float* out_host, void* staging,
+                                  size_t staging_bytes, loki_stream_t stream) {
+    StepStaging st;
+    if (!step_staging(cache, batch, num_q_heads, &st)) {
+        loki_status e = check_cache(cache);
+        if (e == LOKI_OK) e = check_batch(batch);
+        return e == LOKI_OK ? LOKI_ERR_INVALID_ARG : e;
+    }
+    if (batch->batch == 0) return LOKI_OK;
+    if (!k_new_host || !v_new_host || !q_host || !out_host) return LOKI_ERR_INVALID_ARG;
+    if (!staging || staging_bytes < st.total) return LOKI_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(staging) & 255u) != 0) return LOKI_ERR_INVALID_ARG;
+    char* dev = reinterpret_cast<char*>(staging);
+    void* dk = dev + st.k_off;
+    void* dv = dev + st.v_off;
+    void* dq = dev + st.q_off;
+    float* dout = reinterpret_cast<float*>(dev + st.o_off);
+    // every argument of the step, checked before the first copy
+    loki_status e = check_append(cache, batch, dk, dv, P);
+    if (e != LOKI_OK) return e;
+    e = check_decode(cache, batch, dq, num_q_heads, P, r, k, recent_window, group_reduce, scale, dout);
+    if (e != LOKI_OK) return e;
+    if ((e = check_decode_fits(cache, batch, num_q_heads, r)) != LOKI_OK) return e;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    clear_pending_error();
+    if (cudaMemcpyAsync(dk, k_new_host, st.k_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(dv, v_new_host, st.k_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(dq, q_host, st.q_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+        cudaGetLastError();
+        return LOKI_ERR_CUDA;
+    }
+    if ((e = launch_append(cache, batch, dk, dv, P, s)) != LOKI_OK) return e;
+    if ((e = launch_decode(cache, batch, dq, num_q_heads, P, r, k, k_per_seq, recent_window, group_reduce, scale, dout,
+                           nullptr, s, true)) != LOKI_OK)
+        return e;
+    if (cudaMemcpyAsync(out_host, dout, st.o_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
+        cudaGetLastError();
+        return LOKI_ERR_CUDA;
+    }
+    return LOKI_OK;
+}
+
 loki_status loki_decode_step(const loki_cache* cache, const loki_batch* batch, const void* k_new, const void* v_new,
                              const void* q, int32_t num_q_heads, const float* P, int32_t r, int32_t k,
                              const int32_t* k_per_seq, int32_t recent_window, loki_group_reduce group_reduce,

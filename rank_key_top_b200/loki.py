@@ -86,6 +86,9 @@ _SIGS = {
     "loki_index_keys": (ctypes.c_int, [_C, _B, _P, _P, _I32, _P]),
     "loki_decode_step": (ctypes.c_int, [_C, _B, _P, _P, _P, _I32, _P, _I32, _I32, _P, _I32,
                                         ctypes.c_int, ctypes.c_float, _P, _P, _P, _SZ, _P]),
+    "loki_decode_step_host_bytes": (_SZ, [_C, _B, _I32]),
+    "loki_decode_step_host": (ctypes.c_int, [_C, _B, _P, _P, _P, _I32, _P, _I32, _I32, _P, _I32,
+                                             ctypes.c_int, ctypes.c_float, _P, _P, _SZ, _P]),
     "loki_decode_max_seq_len": (_I32, [_I32, ctypes.c_int]),
     "loki_dense_workspace_bytes": (_SZ, [_C, _B, _I32]),
     "loki_dense_attention": (ctypes.c_int, [_C, _B, _P, _I32, _P, ctypes.c_float, _P, _P, _SZ, _P]),
@@ -313,6 +316,20 @@ def loki_index_keys(cache, batch, k, A_k, stream=None):
     """Fill the key index with k A_k; k is [batch, Hkv, max_len, head_dim]."""
     _check("loki_index_keys", _lib.loki_index_keys(
         ctypes.byref(cache.struct), ctypes.byref(batch.struct), _ptr(k), _ptr(A_k), k.shape[2], _stream(stream)))
+
+
+def loki_decode_step_host_bytes(cache, batch, num_q_heads):
+    return _lib.loki_decode_step_host_bytes(ctypes.byref(cache.struct), ctypes.byref(batch.struct), num_q_heads)
+
+
+def loki_decode_step_host(cache, batch, k_new_host, v_new_host, q_host, P, r, k, out_host, staging, k_per_seq=None,
+                          recent_window=0, group_reduce=LOKI_GROUP_SUM, scale=0.0, stream=None):
+    """The decode step with its inputs and output in (pinned) host tensors;
+    staging: a device uint8 tensor of loki_decode_step_host_bytes bytes."""
+    _check("loki_decode_step_host", _lib.loki_decode_step_host(
+        ctypes.byref(cache.struct), ctypes.byref(batch.struct), _ptr(k_new_host), _ptr(v_new_host), _ptr(q_host),
+        q_host.shape[1], _ptr(P), r, k, _ptr(k_per_seq), recent_window, group_reduce, scale, _ptr(out_host),
+        _ptr(staging), staging.numel() * staging.element_size(), _stream(stream)))
 
 
 def loki_decode_step(cache, batch, k_new, v_new, q, P, r, k, out, k_per_seq=None, recent_window=0,

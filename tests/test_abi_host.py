@@ -248,3 +248,41 @@ def test_decode_needs_no_workspace(loki):
     c, b = structs(loki)
     assert lib.loki_decode_workspace_bytes(ctypes.byref(c), ctypes.byref(b), 32, 8, 0) == 0
     assert lib.loki_decode_workspace_bytes(ctypes.byref(c), ctypes.byref(b), 32, 2048, 64) == 0
+
+
+def step_host(loki, c, b, k_new=FAKE, v_new=FAKE, q=FAKE, Hq=32, r=32, k=8, W=0, P=FAKE, out=FAKE, staging=FAKE,
+              staging_bytes=1 << 30):
+    return loki.raw().loki_decode_step_host(ctypes.byref(c), ctypes.byref(b), k_new, v_new, q, Hq, P, r, k, None, W,
+                                            0, 0.0, out, staging, staging_bytes, None)
+
+
+def test_decode_step_host_staging_bytes(loki):
+    """k_new, v_new, q in the cache dtype and out in fp32, each region rounded up to 256 bytes."""
+    c, b = structs(loki, B=2, Hkv=8, D=128, dtype=1)
+    raw = loki.raw()
+    kv = 2 * 8 * 128 * 2            # 4096 bytes each
+    q = 2 * 32 * 128 * 2            # 16384
+    o = 2 * 32 * 128 * 4            # 32768
+    assert raw.loki_decode_step_host_bytes(ctypes.byref(c), ctypes.byref(b), 32) == 2 * kv + q + o
+    c, b = structs(loki, B=1, Hkv=3, D=64, dtype=0)
+    up = lambda x: (x + 255) // 256 * 256
+    assert raw.loki_decode_step_host_bytes(ctypes.byref(c), ctypes.byref(b), 3) == (
+        2 * up(3 * 64 * 4) + up(3 * 64 * 4) + up(3 * 64 * 4))
+    assert raw.loki_decode_step_host_bytes(ctypes.byref(c), ctypes.byref(b), 0) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(k_new=None), 1),           # host buffers are required
+    (dict(v_new=None), 1),
+    (dict(q=None), 1),
+    (dict(out=None), 1),
+    (dict(staging=None), 3),         # the staging buffer must exist and be large enough
+    (dict(staging_bytes=1024), 3),
+    (dict(staging=FAKE + 16), 1),    # and 256-byte aligned
+    (dict(k=0, W=0), 1),             # the step's own arguments, before any copy
+    (dict(r=24), 2),
+    (dict(P=FAKE + 4), 1),
+])
+def test_decode_step_host_rejects(loki, kw, status):
+    c, b = structs(loki)
+    assert step_host(loki, c, b, **kw) == status

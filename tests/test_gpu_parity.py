@@ -826,3 +826,33 @@ def test_asym_decode_with_pca_factor_is_leading(cuda_lib, group_max):
                                         selected_idx=sel)
     torch.cuda.synchronize()
     assert torch.equal(a[0], out.cpu()) and torch.equal(a[1], sel.cpu())
+
+@pytest.mark.parametrize("dtype,W", [("bf16", 8), ("f32", 0)])
+def test_decode_step_host_equals_decode_step(cuda_lib, dtype, W):
+    """loki_decode_step_host (inputs and output in pinned host memory, copies
+    on the stream) gives bit for bit what loki_decode_step gives."""
+    s = spec(num_q_heads=8, num_kv_heads=2, seq_lens=[1999, 3000], k=200, recent_window=W, dtype=dtype)
+    wl = synth.make_workload(s)
+    k_new, v_new = synth.draw_new_tokens(s, step=4)
+    lens = torch.tensor([n + 1 for n in s.seq_lens], dtype=torch.int32)
+    outs = []
+    for host in (False, True):
+        dev = harness.Device(wl, cuda_lib)
+        dev.batch = cuda_lib.Batch(wl.block_table.cuda(), lens.cuda(), int(lens.max()))
+        if host:
+            out = torch.full((s.batch, s.num_q_heads, s.head_dim), float("nan")).pin_memory()
+            staging = torch.empty(cuda_lib.loki_decode_step_host_bytes(dev.cache, dev.batch, s.num_q_heads),
+                                  dtype=torch.uint8, device="cuda")
+            cuda_lib.loki_decode_step_host(dev.cache, dev.batch, k_new.pin_memory(), v_new.pin_memory(),
+                                           wl.q.pin_memory(), dev.P, s.r, s.k, out, staging, recent_window=W)
+            torch.cuda.synchronize()
+            outs.append(out.clone())
+        else:
+            out = torch.full((s.batch, s.num_q_heads, s.head_dim), float("nan"), device="cuda")
+            cuda_lib.loki_decode_step(dev.cache, dev.batch, k_new.cuda(), v_new.cuda(), dev.q, dev.P, s.r, s.k, out,
+                                      recent_window=W)
+            torch.cuda.synchronize()
+            outs.append(out.cpu())
+    assert cuda_lib.loki_device_error(clear=True) == 0
+    assert not torch.isnan(outs[1]).any()
+    assert torch.equal(outs[0], outs[1])
