@@ -856,3 +856,46 @@ def test_decode_step_host_equals_decode_step(cuda_lib, dtype, W):
     assert cuda_lib.loki_device_error(clear=True) == 0
     assert not torch.isnan(outs[1]).any()
     assert torch.equal(outs[0], outs[1])
+
+
+def test_decode_step_host_in_a_cuda_graph(cuda_lib):
+    """The host-buffer step captured once into a CUDA graph and replayed with
+    new host inputs written in place gives what an eager call gives."""
+    s = spec(num_q_heads=8, num_kv_heads=2, seq_lens=[1200, 2500], k=100, recent_window=4)
+    wl = synth.make_workload(s)
+    lens = torch.tensor([n + 1 for n in s.seq_lens], dtype=torch.int32)
+    dev = harness.Device(wl, cuda_lib)
+    dev.batch = cuda_lib.Batch(wl.block_table.cuda(), lens.cuda(), int(lens.max()))
+    staging = torch.empty(cuda_lib.loki_decode_step_host_bytes(dev.cache, dev.batch, s.num_q_heads),
+                          dtype=torch.uint8, device="cuda")
+    hk, hv = (t.pin_memory() for t in synth.draw_new_tokens(s, step=0))
+    hq = wl.q.clone().pin_memory()
+    hout = torch.empty(s.batch, s.num_q_heads, s.head_dim).pin_memory()
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        cuda_lib.loki_decode_step_host(dev.cache, dev.batch, hk, hv, hq, dev.P, s.r, s.k, hout, staging,
+                                       recent_window=4, stream=stream)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            cuda_lib.loki_decode_step_host(dev.cache, dev.batch, hk, hv, hq, dev.P, s.r, s.k, hout, staging,
+                                           recent_window=4, stream=stream)
+    results = []
+    for step in (1, 2):
+        k_new, v_new = synth.draw_new_tokens(s, step=step)
+        hk.copy_(k_new)
+        hv.copy_(v_new)
+        hq.copy_(synth.draw_query_batch(s, step))
+        g.replay()
+        torch.cuda.synchronize()
+        graph_out = hout.clone()
+        eager = torch.empty_like(hout).pin_memory()
+        cuda_lib.loki_decode_step_host(dev.cache, dev.batch, hk, hv, hq, dev.P, s.r, s.k, eager, staging,
+                                       recent_window=4)
+        torch.cuda.synchronize()
+        results.append((graph_out, eager.clone()))
+    assert cuda_lib.loki_device_error(clear=True) == 0
+    for a, b in results:
+        assert not torch.isnan(a).any()
+        assert torch.equal(a, b)
+    assert not torch.equal(results[0][0], results[1][0])   # the replays saw the new inputs
