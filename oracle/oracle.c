@@ -34,7 +34,15 @@
  *   - ties in the approximate score go to the lower token index;
  *   - the recent window W is forced, top-k is taken among the other tokens;
  *   - the exact logits use the full head dimension and 1/sqrt(d) by default;
- *   - softmax is renormalised over the kept set only.
+ *   - softmax is renormalised over the kept set only;
+ *   - AQUA's per-dimension selection for a query group ranks a dim by the
+ *     magnitude of the group's summed query (SUM) or by the heads' summed
+ *     squares (MAX), ties to the lower dim;
+ *   - the asymmetric factors minimise the score distortion with uncentred
+ *     second moments (the SAKI abstract stops before its noise correction).
+ * Every function below is pinned by tests/test_oracle_pins.py against values
+ * the pages or the mathematics fix (closed forms, brute force, invariants,
+ * hand-derived fixtures); none is left unpinned.
  */
 #include <math.h>
 #include <stdint.h>
