@@ -202,3 +202,22 @@ def test_rebalance_moves_hot_blocks_and_keeps_results(cuda_lib):
     assert torch.equal(out_f, out_o) and torch.equal(sel_f, sel_o)
     assert np.array_equal(off.touch.cpu().numpy()[:wl.num_blocks], touch)
     assert cuda_lib.offload_rebalance(off, max_moves=10 ** 6) == []
+
+
+def test_offloaded_decode_full_size(cuda_lib):
+    """The bench's workload (8 × 32768 tokens, 32 / 8 heads, r 32, k 2048 + 64)
+    with every second block's rows on the host, in the bench's launch
+    configuration: outputs and kept sets bit-identical to the all-device cache,
+    and sampled pairs against the oracle."""
+    s = synth.named_spec("gqa32x8-d128-L32768-bf16")
+    wl = synth.make_workload(s)
+    dev = harness.Device(wl, cuda_lib, index_dims=s.r)
+    out_f, sel_f = dev.decode()
+    off = offloaded(cuda_lib, wl, s.r, host_every=2)
+    cuda_lib.loki_prefill_cache(off, dev.batch, wl.Kt.cuda(), wl.V.cuda())
+    dev.cache = off
+    out_o, sel_o = dev.decode()
+    assert cuda_lib.loki_device_error(clear=True) == 0
+    assert torch.equal(out_f, out_o) and torch.equal(sel_f, sel_o)
+    for b, h in [(0, 0), (5, 3)]:
+        harness.check_pair(wl, b, h, out_o, sel_o, s.r, s.k, s.recent_window)

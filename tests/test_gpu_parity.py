@@ -899,3 +899,31 @@ def test_decode_step_host_in_a_cuda_graph(cuda_lib):
         assert not torch.isnan(a).any()
         assert torch.equal(a, b)
     assert not torch.equal(results[0][0], results[1][0])   # the replays saw the new inputs
+
+
+def test_per_dim_scorer_full_size(cuda_lib):
+    """The per-dimension magnitude scorer in the bench's configuration (the
+    32768-token GQA workload, an index of all 128 dims, r 32, k 2048 + 64):
+    sampled pairs whose r-th and (r+1)-th dim magnitudes are apart by more than
+    the selection margin, against the oracle's per-dimension decode."""
+    import oracle
+    s = synth.named_spec("gqa32x8-d128-L32768-bf16")
+    wl = synth.make_workload(s)
+    dev = harness.Device(wl, cuda_lib, index_dims=s.head_dim)
+    out, sel = dev.decode(scorer=cuda_lib.LOKI_SCORER_MAGNITUDE)
+    assert cuda_lib.loki_device_error() == 0
+    checked = 0
+    for b in range(s.batch):
+        for h in range(s.num_kv_heads):
+            _, _, qq, P = harness.pair_inputs(wl, b, h)
+            _, w = oracle.magnitude_dims(qq, P, s.r, s.head_dim)
+            w = np.sort(w)[::-1]
+            if w[s.r - 1] - w[s.r] <= harness.SLAB_MARGIN * w[s.r - 1]:
+                continue
+            harness.check_pair(wl, b, h, out, sel, s.r, s.k, s.recent_window, magnitude_dims=s.head_dim,
+                               magnitude="dims")
+            checked += 1
+            if checked == 3:
+                return
+    assert checked > 0, "no pair with a dim-selection margin"
+
