@@ -241,7 +241,10 @@ def unrotated_keys(wl):
 
 
 @pytest.mark.parametrize("dtype,D,lens", [("bf16", 128, [300, 1000, 0, 1, 129]), ("bf16", 64, [257, 40]),
-                                          ("f32", 128, [300, 17, 0]), ("f32", 64, [65])])
+                                          ("f32", 128, [300, 17, 0]), ("f32", 64, [65]),
+                                          # more tiles than CTAs: tile ranges that cross into the next
+                                          # (sequence, kv head), with skipped tiles past short sequences
+                                          ("bf16", 128, [5000, 1, 2900, 4100]), ("bf16", 64, [3000, 2000, 10])])
 def test_prefill_rotate_matches_oracle(cuda_lib, dtype, D, lens):
     """K~ = round(K P) for every prompt token, the value rows copied and the
     key index filled, read back through the documented layout. bf16 uses the
