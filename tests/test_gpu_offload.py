@@ -221,3 +221,27 @@ def test_offloaded_decode_full_size(cuda_lib):
     assert torch.equal(out_f, out_o) and torch.equal(sel_f, sel_o)
     for b, h in [(0, 0), (5, 3)]:
         harness.check_pair(wl, b, h, out_o, sel_o, s.r, s.k, s.recent_window)
+
+
+def test_home_entry_outside_its_pool_is_flagged(cuda_lib):
+    """A map entry past its pool is caught by the kernels' own range check
+    (LOKI_DEVERR_BLOCK_ID): the block's rows are neither read nor written."""
+    s = spec(seq_lens=[900, 700])
+    wl = synth.make_workload(s)
+    dev = harness.Device(wl, cuda_lib, index_dims=32)
+    off = offloaded(cuda_lib, wl, 32, host_every=2)
+    cuda_lib.loki_prefill_cache(off, dev.batch, wl.Kt.cuda(), wl.V.cuda())
+    torch.cuda.synchronize()
+    assert cuda_lib.loki_device_error(clear=True) == 0
+    bad = off.home.clone()
+    p = int(wl.block_table[0, 3])
+    bad[p] = -(off.struct.num_host_pages + 7)       # past the host pool
+    off.home_dev.copy_(bad.cuda())
+    dev.cache = off
+    out, _ = dev.decode()
+    assert cuda_lib.loki_device_error(clear=True) & cuda_lib.LOKI_DEVERR_BLOCK_ID
+    assert torch.isfinite(out).all()
+    bad[p] = off.struct.num_device_pages + 3        # past the device pool
+    off.home_dev.copy_(bad.cuda())
+    dev.dense()
+    assert cuda_lib.loki_device_error(clear=True) & cuda_lib.LOKI_DEVERR_BLOCK_ID
