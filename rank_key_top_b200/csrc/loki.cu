@@ -2,6 +2,7 @@
 // Every kernel is included here so that the device error word and all
 // kernels share one translation unit.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -21,6 +22,14 @@ using namespace loki;
 namespace {
 
 constexpr double kLog2e = 1.4426950408889634;
+
+// An NVTX range around one entry point's host work (its checks and
+// launches), so that a timeline tool shows which call issued which kernels.
+// Without a tool attached the calls do nothing.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
 
 size_t elem_size(loki_dtype dt) { return dt == LOKI_BF16 ? 2 : 4; }
 
@@ -291,6 +300,7 @@ loki_status loki_device_error(int32_t clear, uint32_t* bits) {
 
 loki_status loki_prefill_cache(const loki_cache* cache, const loki_batch* batch, const void* k_rot,
                                const void* v, int32_t max_len, loki_stream_t stream) {
+    NvtxRange nvtx_range("loki_prefill_cache");
     loki_status st = check_cache(cache);
     if (st != LOKI_OK) return st;
     if ((st = check_batch(batch)) != LOKI_OK) return st;
@@ -331,6 +341,7 @@ loki_status loki_prefill_cache(const loki_cache* cache, const loki_batch* batch,
 
 loki_status loki_prefill_rotate(const loki_cache* cache, const loki_batch* batch, const void* k, const void* v,
                                 const float* P, int32_t max_len, loki_stream_t stream) {
+    NvtxRange nvtx_range("loki_prefill_rotate");
     loki_status st = check_cache(cache);
     if (st != LOKI_OK) return st;
     if ((st = check_batch(batch)) != LOKI_OK) return st;
@@ -396,6 +407,7 @@ loki_status loki_prefill_rotate(const loki_cache* cache, const loki_batch* batch
 
 loki_status loki_pca_basis(const void* keys, int32_t num_heads, int64_t n, int32_t head_dim, loki_dtype dtype,
                            float* P, float* eigvals, loki_stream_t stream) {
+    NvtxRange nvtx_range("loki_pca_basis");
     if (num_heads < 0 || n < 0) return LOKI_ERR_INVALID_ARG;
     if (dtype != LOKI_F32 && dtype != LOKI_BF16) return LOKI_ERR_INVALID_ARG;
     if (head_dim != 64 && head_dim != 128) return LOKI_ERR_UNSUPPORTED;
@@ -425,6 +437,7 @@ loki_status loki_pca_basis(const void* keys, int32_t num_heads, int64_t n, int32
 
 loki_status loki_append_keys(const loki_cache* cache, const loki_batch* batch, const void* k_new,
                              const void* v_new, const float* P, loki_stream_t stream) {
+    NvtxRange nvtx_range("loki_append_keys");
     const loki_status st = check_append(cache, batch, k_new, v_new, P);
     if (st != LOKI_OK || batch->batch == 0) return st;
     return launch_append(cache, batch, k_new, v_new, P, reinterpret_cast<cudaStream_t>(stream));
@@ -432,6 +445,7 @@ loki_status loki_append_keys(const loki_cache* cache, const loki_batch* batch, c
 
 loki_status loki_append_keys_asym(const loki_cache* cache, const loki_batch* batch, const void* k_new,
                                   const void* v_new, const float* P, const float* A_k, loki_stream_t stream) {
+    NvtxRange nvtx_range("loki_append_keys_asym");
     const loki_status st = check_append(cache, batch, k_new, v_new, P);
     if (st != LOKI_OK || batch->batch == 0) return st;
     if (!A_k || !aligned16(A_k)) return LOKI_ERR_INVALID_ARG;
@@ -440,6 +454,7 @@ loki_status loki_append_keys_asym(const loki_cache* cache, const loki_batch* bat
 
 loki_status loki_index_keys(const loki_cache* cache, const loki_batch* batch, const void* k, const float* A_k,
                             int32_t max_len, loki_stream_t stream) {
+    NvtxRange nvtx_range("loki_index_keys");
     loki_status st = check_cache(cache);
     if (st != LOKI_OK) return st;
     if ((st = check_batch(batch)) != LOKI_OK) return st;
@@ -498,6 +513,7 @@ loki_status loki_decode_attention(const loki_cache* cache, const loki_batch* bat
                                   loki_group_reduce group_reduce, float scale, float* out,
                                   int32_t* selected_idx, void* workspace, size_t workspace_bytes,
                                   loki_stream_t stream) {
+    NvtxRange nvtx_range("loki_decode_attention");
     (void)workspace;
     (void)workspace_bytes;
     loki_status st = check_decode(cache, batch, q, num_q_heads, P, r, k, recent_window, group_reduce, scale, out);
@@ -513,6 +529,7 @@ loki_status loki_decode_attention_scored(const loki_cache* cache, const loki_bat
                                          loki_group_reduce group_reduce, float scale, loki_scorer scorer,
                                          float* out, int32_t* selected_idx, void* workspace,
                                          size_t workspace_bytes, loki_stream_t stream) {
+    NvtxRange nvtx_range("loki_decode_attention_scored");
     (void)workspace;
     (void)workspace_bytes;
     int sc;
@@ -535,6 +552,7 @@ loki_status loki_decode_attention_asym(const loki_cache* cache, const loki_batch
                                        loki_group_reduce group_reduce, float scale, float* out,
                                        int32_t* selected_idx, void* workspace, size_t workspace_bytes,
                                        loki_stream_t stream) {
+    NvtxRange nvtx_range("loki_decode_attention_asym");
     (void)workspace;
     (void)workspace_bytes;
     loki_status st = check_decode(cache, batch, q, num_q_heads, P, r, k, recent_window, group_reduce, scale, out);
@@ -574,6 +592,7 @@ loki_status loki_decode_step_host(const loki_cache* cache, const loki_batch* bat
                                   int32_t r, int32_t k, const int32_t* k_per_seq, int32_t recent_window,
                                   loki_group_reduce group_reduce, float scale, float* out_host, void* staging,
                                   size_t staging_bytes, loki_stream_t stream) {
+    NvtxRange nvtx_range("loki_decode_step_host");
     StepStaging st;
     if (!step_staging(cache, batch, num_q_heads, &st)) {
         loki_status e = check_cache(cache);
@@ -619,6 +638,7 @@ loki_status loki_decode_step(const loki_cache* cache, const loki_batch* batch, c
                              const int32_t* k_per_seq, int32_t recent_window, loki_group_reduce group_reduce,
                              float scale, float* out, int32_t* selected_idx, void* workspace,
                              size_t workspace_bytes, loki_stream_t stream) {
+    NvtxRange nvtx_range("loki_decode_step");
     (void)workspace;
     (void)workspace_bytes;
     loki_status st = check_append(cache, batch, k_new, v_new, P);
@@ -670,6 +690,7 @@ size_t loki_dense_workspace_bytes(const loki_cache* cache, const loki_batch* bat
 loki_status loki_dense_attention(const loki_cache* cache, const loki_batch* batch, const void* q,
                                  int32_t num_q_heads, const float* P, float scale, float* out,
                                  void* workspace, size_t workspace_bytes, loki_stream_t stream) {
+    NvtxRange nvtx_range("loki_dense_attention");
     loki_status st = check_cache(cache);
     if (st != LOKI_OK) return st;
     if ((st = check_batch(batch)) != LOKI_OK) return st;
@@ -746,6 +767,7 @@ loki_status static_scratch_address(void** out) {
 extern "C" loki_status loki_dense_attention_static(const loki_cache* cache, const loki_batch* batch, const void* q,
                                                    int32_t num_q_heads, const float* P, float scale, float* out,
                                                    loki_stream_t stream) {
+    NvtxRange nvtx_range("loki_dense_attention_static");
     void* scratch = nullptr;
     loki_status st = static_scratch_address(&scratch);
     if (st != LOKI_OK) return st;
@@ -809,6 +831,7 @@ int32_t loki_offload_plan(int32_t num_blocks, int32_t* kv_home, int32_t* spare_p
 
 loki_status loki_offload_apply(const loki_cache* cache, const loki_page_move* moves, int32_t num_moves,
                                const int32_t* kv_home_host, loki_stream_t stream) {
+    NvtxRange nvtx_range("loki_offload_apply");
     loki_status st = check_cache(cache);
     if (st != LOKI_OK) return st;
     if (!cache->kv_home || num_moves < 0 || (num_moves > 0 && !moves)) return LOKI_ERR_INVALID_ARG;
