@@ -166,6 +166,7 @@ __device__ __noinline__ int2 radix_boundary(const uint32_t* hcur, int nbins, int
         if (run < (uint32_t)krem && run + hv[j] >= (uint32_t)krem) {
             misc[0] = 4 * tid + j;
             misc[1] = (int)run;
+            misc[2] = (int)hv[j];  // the boundary bin's count over the cluster
         }
         run += hv[j];
     }
@@ -229,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     // in `part`, whose first G x D floats only rank 0's own merge writes
     const float* qsc = ASYM ? part : qhat;
     int32_t* misc = reinterpret_cast<int32_t*>(smem + p.off_misc);
-    // misc: [0] boundary digit, [1] count above it, [8..39] suffix-sum scratch,
+    // misc: [0] boundary digit, [1] count above it, [2] its bin count, [8..39] suffix-sum scratch,
     //       [40..55] warp kept counts, [56..71] warp equal counts, [72] list length,
     //       [73] the sequence (longest first), [104..111] slab energies (slab
     //       scorer), [128..255] chosen dims (MAG)
@@ -758,30 +759,41 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
         uint32_t* h1 = hist + kHistBins;
         for (int i = lane; i < nw; i += 32) atomicAdd(&h1[(wcand[i] >> 10) & 2047u], 1u);
         const int2 d1 = radix_boundary(h1, 2048, krem, misc, p.C);
+        const int bin1 = misc[2];  // read before the next search overwrites it
         krem -= d1.y;
-        // digit 2 (last 10 bits) into buffer 0: every CTA of the cluster has
-        // read it, the cluster barrier of the previous search orders that
-        for (int i = tid; i < kHistBins; i += kThreads) hist[i] = 0;
-        __syncthreads();
         const uint32_t pre22 = (beta0 << 21) | ((uint32_t)d1.x << 10);
-        for (int i = lane; i < nw; i += 32) {
-            const uint32_t x = wcand[i];
-            if ((x & 0xFFFFFC00u) == pre22) atomicAdd(&hist[x & 1023u], 1u);
-        }
-        const int2 d2 = radix_boundary(hist, 1024, krem, misc, p.C);
-        const uint32_t tau = pre22 | (uint32_t)d2.x;
-        krem -= d2.y;
-        // keys equal to tau: the last histogram counted them per CTA in bin (tau & 1023)
-        int eq_before = 0;
-        for (int c = 0; c < crank; ++c) eq_before += (int)cluster.map_shared_rank(hist, c)[tau & 1023u];
-        const int eq_mine = (int)hist[tau & 1023u];
-        quota = min(max(krem - eq_before, 0), eq_mine);
-        // the candidates against tau
-        for (uint32_t t = rowcand; t; t &= t - 1u) {
-            const int bit = __ffs(t) - 1;
-            const uint32_t x = keys[row0 + bit];
-            rowgt |= (uint32_t)(x > tau) << bit;
-            roweq |= (uint32_t)(x == tau) << bit;
+        if (bin1 == krem && pre22 != 0u) {
+            // every key of the boundary bin is kept (the same decision in every
+            // CTA of the cluster): the kept keys are those >= pre22, no ties to split
+            const uint32_t tau = pre22 - 1u;
+            for (uint32_t t = rowcand; t; t &= t - 1u) {
+                const int bit = __ffs(t) - 1;
+                rowgt |= (uint32_t)(keys[row0 + bit] > tau) << bit;
+            }
+        } else {
+            // digit 2 (last 10 bits) into buffer 0: every CTA of the cluster has
+            // read it, the cluster barrier of the previous search orders that
+            for (int i = tid; i < kHistBins; i += kThreads) hist[i] = 0;
+            __syncthreads();
+            for (int i = lane; i < nw; i += 32) {
+                const uint32_t x = wcand[i];
+                if ((x & 0xFFFFFC00u) == pre22) atomicAdd(&hist[x & 1023u], 1u);
+            }
+            const int2 d2 = radix_boundary(hist, 1024, krem, misc, p.C);
+            const uint32_t tau = pre22 | (uint32_t)d2.x;
+            krem -= d2.y;
+            // keys equal to tau: the last histogram counted them per CTA in bin (tau & 1023)
+            int eq_before = 0;
+            for (int c = 0; c < crank; ++c) eq_before += (int)cluster.map_shared_rank(hist, c)[tau & 1023u];
+            const int eq_mine = (int)hist[tau & 1023u];
+            quota = min(max(krem - eq_before, 0), eq_mine);
+            // the candidates against tau
+            for (uint32_t t = rowcand; t; t &= t - 1u) {
+                const int bit = __ffs(t) - 1;
+                const uint32_t x = keys[row0 + bit];
+                rowgt |= (uint32_t)(x > tau) << bit;
+                roweq |= (uint32_t)(x == tau) << bit;
+            }
         }
     }
 
