@@ -708,7 +708,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     // boundary bin (kept whatever tau is) and the keys inside it (the
     // candidates, a few percent); digits 1 and 2 and the final comparison with
     // tau look at the candidates only. The three digits share one copy of the
-    // boundary search (radix_boundary).
+    // boundary search (radix_boundary). Digit 2 is skipped when digit 1's
+    // boundary bin is kept whole (its count over the cluster is what is still
+    // needed): then every candidate at or above the bin's 22-bit prefix is kept.
     const int mode = keff >= ncand ? 0 : (keff == 0 ? 1 : 2);
     const int row0 = 32 * tid;
     const int nv = n_cand_loc - row0;  // valid keys in this row (may exceed 32)
