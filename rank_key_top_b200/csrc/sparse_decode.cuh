@@ -151,7 +151,8 @@ __device__ __noinline__ int2 radix_boundary(const uint32_t* hcur, int nbins, int
     cluster.sync();  // every thread of every CTA: the histograms are complete and visible
     uint32_t hv[4] = {0u, 0u, 0u, 0u};  // bins 4 tid .. 4 tid + 3
     if (4 * tid < nbins) {
-        for (int c = 0; c < C; ++c) {
+#pragma unroll 4
+        for (int c = 0; c < C; ++c) {  // unrolled: the ranks' loads are in flight together
             const uint4 v = reinterpret_cast<const uint4*>(cluster.map_shared_rank(hcur, c))[tid];
             hv[0] += v.x;
             hv[1] += v.y;
