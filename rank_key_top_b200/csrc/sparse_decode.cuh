@@ -355,13 +355,23 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
             // of the block's 16 tokens; bf16 rows swap their two 16-byte
             // halves on rows 4..7 mod 8, so that ldmatrix.trans is free of
             // bank conflicts
-            constexpr int PPR = (int)sizeof(T);  // 16-byte pieces of one dim row
-            for (int pc = lane; pc < p.r * PPR; pc += 32) {
-                const int row = pc / PPR, part = pc - row * PPR;
-                const int dim = MAG ? misc[kSelDims + row] : row;
-                const int dpart = sizeof(T) == 2 ? (part ^ ((row >> 2) & 1)) : part;
-                cp_async16(dst + row * 16 * (int)sizeof(T) + dpart * 16, src + dim * 16 * (int)sizeof(T) + part * 16,
-                           true);
+            if constexpr (!MAG) {
+                // the leading r dims: one contiguous run of the page (bf16:
+                // the half swap of rows 4..7 mod 8 is bit 4 of the byte
+                // offset flipped where bit 7 is set). The scoring loop is
+                // issue-bound; the per-piece row arithmetic of the general
+                // form below cost about 2.5 us at 32k tokens.
+                for (int o = lane * 16; o < p.slot_bytes; o += 32 * 16)
+                    cp_async16(dst + (sizeof(T) == 2 ? (o ^ ((o >> 3) & 16)) : o), src + o, true);
+            } else {
+                constexpr int PPR = (int)sizeof(T);  // 16-byte pieces of one dim row
+                for (int pc = lane; pc < p.r * PPR; pc += 32) {
+                    const int row = pc / PPR, part = pc - row * PPR;
+                    const int dim = misc[kSelDims + row];
+                    const int dpart = sizeof(T) == 2 ? (part ^ ((row >> 2) & 1)) : part;
+                    cp_async16(dst + row * 16 * (int)sizeof(T) + dpart * 16, src + dim * 16 * (int)sizeof(T) + part * 16,
+                               true);
+                }
             }
         }
         cp_async_commit();
@@ -574,17 +584,16 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
             // ldmatrix.trans row address of this lane: matrix m = lane / 8 holds
             // tokens 8 (m & 1) .. + 7 of dims 8 (m >> 1) + (lane & 7) of the k-step
             const int mrow = (lane & 7) + 8 * (lane >> 4), mhalf = (lane >> 3) & 1;
+            // byte offset of that row in slab 0 (slab sb adds 512: 16 rows of 32 bytes,
+            // and row + 16 sb swaps its halves exactly when row does)
+            const int loff = mrow * 32 + ((mhalf ^ ((mrow >> 2) & 1)) << 4);
             // block it's slot into fragments, then the slot's refill
             auto load_block = [&](int it, uint32_t (&a)[RMAX][4]) {
                 wait_slot();
                 const unsigned char* sl = wring + (it & smask) * p.slot_bytes;
 #pragma unroll
                 for (int sb = 0; sb < RMAX; ++sb)
-                    if (sb < R16) {
-                        const int row = sb * 16 + mrow;
-                        ldmatrix_x4_trans(a[sb][0], a[sb][1], a[sb][2], a[sb][3],
-                                          sl + row * 32 + ((mhalf ^ ((row >> 2) & 1)) << 4));
-                    }
+                    if (sb < R16) ldmatrix_x4_trans(a[sb][0], a[sb][1], a[sb][2], a[sb][3], sl + sb * 512 + loff);
                 __syncwarp();
                 refill(it + S);
             };
@@ -863,60 +872,67 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
         unsigned char* wst = stage + warp * GS * Geom::CHUNK_BYTES;
         const int nchunks = (n_list + NCH - 1) / NCH;
         const int my_n = nchunks > warp ? (nchunks - warp + kWarps - 1) / kWarps : 0;
-        // stage chunk m of this warp (tokens list[ch*NCH .. ch*NCH+NCH)) into slot m % GS
-        auto fetch = [&](int m) {
+        // stage chunk m of this warp (tokens list[ch*NCH .. ch*NCH+NCH)) into
+        // slot m % GS. The bf16 path runs one of two copies of the gather loop,
+        // chosen once per launch: with the home-map branch taken per chunk the
+        // all-device gather measured about 1.3 us slower at 32k tokens.
+        auto fetch_dev = [&](int m) {
             if (m < my_n) {
                 unsigned char* dst = wst + (m % GS) * Geom::CHUNK_BYTES;
                 const int ch = warp + m * kWarps;
-                if (!p.kv.home) {
-                    for (int pc = lane; pc < NCH * PIECES; pc += 32) {
-                        const int n = pc / PIECES, w = pc - n * PIECES;
-                        const int kv = w >= PIECES / 2, c = w - kv * (PIECES / 2);
-                        const int idx = ch * NCH + n;
-                        const bool ok = idx < n_list;
-                        const unsigned char* src = kbytes;
-                        if (ok) {
-                            const int li = list[idx];
-                            const int64_t at = page_offset(tbl[li >> 4], h, p.Hkv, D) * (int64_t)sizeof(T) +
-                                               (int64_t)(li & 15) * ROWB + c * 16;
-                            src = (kv ? vbytes : kbytes) + at;
-                        }
-                        int off;
-                        if constexpr (Geom::MMA) off = Geom::MCore::staged_offset(kv, n, c);
-                        else off = n * TB + kv * ROWB + c * 16;
-                        cp_async16(dst + off, src, ok);
+                for (int pc = lane; pc < NCH * PIECES; pc += 32) {
+                    const int n = pc / PIECES, w = pc - n * PIECES;
+                    const int kv = w >= PIECES / 2, c = w - kv * (PIECES / 2);
+                    const int idx = ch * NCH + n;
+                    const bool ok = idx < n_list;
+                    const unsigned char* src = kbytes;
+                    if (ok) {
+                        const int li = list[idx];
+                        const int64_t at = page_offset(tbl[li >> 4], h, p.Hkv, D) * (int64_t)sizeof(T) +
+                                           (int64_t)(li & 15) * ROWB + c * 16;
+                        src = (kv ? vbytes : kbytes) + at;
                     }
-                } else {
-                    // rows of offloaded blocks come over the host link by plain
-                    // loads of their mapped pages: only the kept rows cross it
-                    for (int pc = lane; pc < NCH * PIECES; pc += 32) {
-                        const int n = pc / PIECES, w = pc - n * PIECES;
-                        const int kv = w >= PIECES / 2, c = w - kv * (PIECES / 2);
-                        const int idx = ch * NCH + n;
-                        bool ok = idx < n_list, host = false;
-                        const unsigned char* src = kbytes;
-                        if (ok) {
-                            const int li = list[idx];
-                            KvPage loc;
-                            ok = kv_locate(p.kv, tbl[li >> 4], loc);
-                            if (ok) {
-                                host = loc.host;
-                                const int64_t at = page_offset(loc.page, h, p.Hkv, D) * (int64_t)sizeof(T) +
-                                                   (int64_t)(li & 15) * ROWB + c * 16;
-                                src = (host ? (kv ? p.kv.host_v : p.kv.host_k) : (kv ? vbytes : kbytes)) + at;
-                            }
-                        }
-                        int off;
-                        if constexpr (Geom::MMA) off = Geom::MCore::staged_offset(kv, n, c);
-                        else off = n * TB + kv * ROWB + c * 16;
-                        if (host) *reinterpret_cast<uint4*>(dst + off) = *reinterpret_cast<const uint4*>(src);
-                        else cp_async16(dst + off, src, ok);
-                    }
+                    int off;
+                    if constexpr (Geom::MMA) off = Geom::MCore::staged_offset(kv, n, c);
+                    else off = n * TB + kv * ROWB + c * 16;
+                    cp_async16(dst + off, src, ok);
                 }
             }
             cp_async_commit();
         };
-        auto run = [&](auto& core) {
+        // rows of offloaded blocks come over the host link by plain loads of
+        // their mapped pages: only the kept rows cross it
+        auto fetch_map = [&](int m) {
+            if (m < my_n) {
+                unsigned char* dst = wst + (m % GS) * Geom::CHUNK_BYTES;
+                const int ch = warp + m * kWarps;
+                for (int pc = lane; pc < NCH * PIECES; pc += 32) {
+                    const int n = pc / PIECES, w = pc - n * PIECES;
+                    const int kv = w >= PIECES / 2, c = w - kv * (PIECES / 2);
+                    const int idx = ch * NCH + n;
+                    bool ok = idx < n_list, host = false;
+                    const unsigned char* src = kbytes;
+                    if (ok) {
+                        const int li = list[idx];
+                        KvPage loc;
+                        ok = kv_locate(p.kv, tbl[li >> 4], loc);
+                        if (ok) {
+                            host = loc.host;
+                            const int64_t at = page_offset(loc.page, h, p.Hkv, D) * (int64_t)sizeof(T) +
+                                               (int64_t)(li & 15) * ROWB + c * 16;
+                            src = (host ? (kv ? p.kv.host_v : p.kv.host_k) : (kv ? vbytes : kbytes)) + at;
+                        }
+                    }
+                    int off;
+                    if constexpr (Geom::MMA) off = Geom::MCore::staged_offset(kv, n, c);
+                    else off = n * TB + kv * ROWB + c * 16;
+                    if (host) *reinterpret_cast<uint4*>(dst + off) = *reinterpret_cast<const uint4*>(src);
+                    else cp_async16(dst + off, src, ok);
+                }
+            }
+            cp_async_commit();
+        };
+        auto run = [&](auto& core, auto&& fetch) {
             for (int m = 0; m < GS - 1; ++m) fetch(m);
             for (int m = 0; m < my_n; ++m) {
                 fetch(m + GS - 1);
@@ -947,11 +963,18 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
         if constexpr (Geom::MMA) {
             typename Geom::MCore core;
             core.init(qhat, p.scale_log2, lane);
-            run(core);
+            if (!p.kv.home) run(core, fetch_dev);
+            else run(core, fetch_map);
         } else {
+            // (the fp32 path keeps one loop with the branch per chunk: two
+            // copies of it measured about 1.8 us slower on the single-head
+            // d64 L1024 workload)
             Core core;
             core.init(qhat, p.scale_log2, lane);
-            run(core);
+            run(core, [&](int m) {
+                if (!p.kv.home) fetch_dev(m);
+                else fetch_map(m);
+            });
         }
     }
     __syncthreads();
