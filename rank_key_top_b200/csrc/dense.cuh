@@ -5,7 +5,8 @@
 //   dense_split_kernel   one CTA per (split, sequence, kv head) stages the
 //                        split's key and value rows with cp.async, runs the
 //                        attention core over them and writes its (o, m, l)
-//                        partial to the workspace
+//                        partial to the workspace; a split is 1024 tokens, or
+//                        2048 when that still leaves several waves of CTAs
 //   merge_kernel         combines the splits of each query head
 // The partials in global memory are the workspace (scratch) of this path.
 #pragma once
@@ -16,7 +17,7 @@
 
 namespace loki {
 
-constexpr int kDenseSplitTokens = 1024;
+constexpr int kDenseSplitTokens = 1024;  // the workspace is sized for splits of this many tokens
 
 struct DenseParams {
     const void* k_cache;
@@ -30,6 +31,7 @@ struct DenseParams {
     float* parts;  // workspace [batch * Hkv][splits][G][D + 2]
     KvMap kv;
     int num_blocks, Hkv, max_blocks, max_seq_len, splits;
+    int split_tokens;  // kDenseSplitTokens or a multiple of it
     float scale_log2;
 };
 
@@ -101,8 +103,8 @@ __global__ void __launch_bounds__(kDenseThreads) dense_split_kernel(const DenseP
         if (tid == 0 && split == 0) flag_error(LOKI_DEVERR_SEQ_LEN);
         L = L < 0 ? 0 : p.max_seq_len;
     }
-    const int t_lo = split * kDenseSplitTokens;
-    const int n = max(0, min(L, t_lo + kDenseSplitTokens) - t_lo);
+    const int t_lo = split * p.split_tokens;
+    const int n = max(0, min(L, t_lo + p.split_tokens) - t_lo);
     for (int i = tid; i < G * D; i += kDenseThreads) qs[i] = p.qhat[((int64_t)b * Hq + h * G) * D + i];
 
     const unsigned char* kbytes = reinterpret_cast<const unsigned char*>(p.k_cache);

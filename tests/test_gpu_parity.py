@@ -531,6 +531,24 @@ def test_dense_edge(cuda_lib):
             harness.check_dense_pair(wl, b, h, out)
 
 
+def test_dense_long_splits_ragged(cuda_lib):
+    """Enough pairs that the dense path takes its longer splits (2048 tokens:
+    160 pairs x 4 splits of the longest sequence fill four waves of CTAs):
+    lengths around the split and block edges, one empty sequence."""
+    lens = [8191, 0, 1, 2047, 2048, 2049, 4095, 4097, 6144, 16, 17, 3000, 8000, 5555, 2050, 7777] * 2
+    lens += [8191, 1024, 1023, 6000, 4096, 2, 8190, 100]
+    s = spec(num_q_heads=16, num_kv_heads=4, seq_lens=lens, head_dim=128, k=5, seed=29)
+    assert s.batch * s.num_kv_heads * ((max(lens) + 2047) // 2048) >= 4 * 148
+    wl = synth.make_workload(s, pairs={(b, h) for b in range(len(lens)) for h in (0, 3)})
+    out = harness.Device(wl, cuda_lib).dense()
+    assert cuda_lib.loki_device_error() == 0
+    assert torch.all(out[1] == 0)
+    for b in range(s.batch):
+        if lens[b] > 0:
+            for h in (0, 3):
+                harness.check_dense_pair(wl, b, h, out)
+
+
 # ---------------------------------------------------------------------------
 # Full-size workloads, every pair
 # ---------------------------------------------------------------------------
