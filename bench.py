@@ -619,8 +619,9 @@ def main():
         return
 
     # end to end through the public API: loki_decode_step_host takes the step's
-    # inputs (q, k_new, v_new) in pinned host memory, copies them in, runs the
-    # step and copies the output back, all on the stream; one graph per input slot
+    # inputs (q, k_new, v_new) and its output in pinned host memory, which its
+    # kernels read and write in place over the host link, all on the stream;
+    # one graph per input slot
     hq = [q.cpu().pin_memory() for q in qs]
     hk = [k.cpu().pin_memory() for k in ks]
     hv = [v.cpu().pin_memory() for v in vs]
@@ -759,8 +760,9 @@ def main():
         "cpu_baseline": cb,
         "e2e": {"value": world * K / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
-                "path": "loki_decode_step_host: q, k_new, v_new from pinned host buffers, the step, out back to a "
-                        "pinned host buffer; one CUDA graph per input slot"},
+                "path": "loki_decode_step_host: q, k_new, v_new read from pinned host buffers and out written "
+                        "to a pinned host buffer by the step's kernels (mapped, in place); one CUDA graph per "
+                        "input slot"},
         "clocks": clocks,
         "gpu_launches": 2 * K,
         "step_launch": "CUDA graph per step: loki_decode_step (append kernel, then the decode kernel as its "

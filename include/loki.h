@@ -376,17 +376,25 @@ LOKI_API size_t loki_decode_step_host_bytes(const loki_cache* cache, const loki_
                                             int32_t num_q_heads);
 
 /* loki_decode_step for a caller that holds the step's inputs and output in
- * host memory. k_new_host, v_new_host ([batch][num_kv_heads][head_dim]) and
- * q_host ([batch][num_q_heads][head_dim]), all in the cache dtype, are copied
- * into `staging` (device, loki_decode_step_host_bytes bytes, 256-byte
- * aligned), the step runs as loki_decode_step with the same remaining
- * arguments (no kept-index export), and the output ([batch][num_q_heads]
- * [head_dim] fp32) is copied back to out_host: one cudaMemcpyAsync per buffer,
- * all on `stream`. With pinned host memory the call is asynchronous and the
- * host buffers must stay untouched until the stream has passed the copies;
- * pageable memory makes the copies synchronous with the host. Every argument
- * is checked before anything is issued; an error issues nothing. The caller
- * owns every buffer; the library allocates nothing. */
+ * host memory: k_new_host, v_new_host ([batch][num_kv_heads][head_dim]) and
+ * q_host ([batch][num_q_heads][head_dim]), all in the cache dtype, and
+ * out_host ([batch][num_q_heads][head_dim] fp32). The step runs as
+ * loki_decode_step with the same remaining arguments (no kept-index export),
+ * all on `stream`, in one of two ways:
+ *  - all four buffers page-locked and mapped into the device's address space
+ *    (cudaHostAlloc / cudaMallocHost memory, or cudaHostRegister'ed memory,
+ *    under unified addressing; out_host 4-byte and q_host 16-byte aligned):
+ *    the kernels read the inputs and write the output in place over the host
+ *    link, and `staging` is not touched;
+ *  - otherwise the inputs are copied into `staging` (device,
+ *    loki_decode_step_host_bytes bytes, 256-byte aligned) and the output back
+ *    from it, one cudaMemcpyAsync per buffer; pageable memory makes those
+ *    copies synchronous with the host.
+ * `staging` is required either way. With page-locked memory the call is
+ * asynchronous: the host buffers must stay untouched, and out_host unread,
+ * until the stream has passed the step. Every argument is checked before
+ * anything is issued; an error issues nothing. The caller owns every buffer;
+ * the library allocates nothing. */
 LOKI_API loki_status loki_decode_step_host(const loki_cache* cache, const loki_batch* batch,
                                            const void* k_new_host, const void* v_new_host,
                                            const void* q_host, int32_t num_q_heads, const float* P,

@@ -582,6 +582,21 @@ static bool step_staging(const loki_cache* cache, const loki_batch* batch, int32
     return true;
 }
 
+// The address under which the current device reads and writes a host buffer
+// in place, if it can: page-locked memory mapped into the device's address
+// space (cudaHostAlloc / cudaMallocHost memory, and cudaHostRegister'ed
+// memory, under unified addressing, where that address is the host address
+// itself). nullptr for pageable memory or any other answer.
+static void* mapped_host_address(const void* host) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, host) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    if (a.type != cudaMemoryTypeHost || a.devicePointer != host) return nullptr;
+    return a.devicePointer;
+}
+
 size_t loki_decode_step_host_bytes(const loki_cache* cache, const loki_batch* batch, int32_t num_q_heads) {
     StepStaging st;
     return step_staging(cache, batch, num_q_heads, &st) ? st.total : 0;
@@ -603,6 +618,32 @@ loki_status loki_decode_step_host(const loki_cache* cache, const loki_batch* bat
     if (!k_new_host || !v_new_host || !q_host || !out_host) return LOKI_ERR_INVALID_ARG;
     if (!staging || staging_bytes < st.total) return LOKI_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(staging) & 255u) != 0) return LOKI_ERR_INVALID_ARG;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // Mapped page-locked buffers are read and written in place by the kernels
+    // (the append reads k_new and v_new, the decode's prologue reads q and its
+    // merge writes out, all with plain loads and stores over the host link):
+    // no copy engine on the step's path. Otherwise the buffers go through
+    // `staging`, one cudaMemcpyAsync each.
+    {
+        void* mk = mapped_host_address(k_new_host);
+        void* mv = mapped_host_address(v_new_host);
+        void* mq = mapped_host_address(q_host);
+        void* mo = mapped_host_address(out_host);
+        if (mk && mv && mq && mo && (reinterpret_cast<uintptr_t>(mo) & 3u) == 0) {
+            float* out_mapped = reinterpret_cast<float*>(mo);
+            loki_status e = check_append(cache, batch, mk, mv, P);
+            if (e == LOKI_OK) e = check_decode(cache, batch, mq, num_q_heads, P, r, k, recent_window, group_reduce,
+                                               scale, out_mapped);
+            if (e == LOKI_OK) {
+                if ((e = check_decode_fits(cache, batch, num_q_heads, r)) != LOKI_OK) return e;
+                clear_pending_error();
+                if ((e = launch_append(cache, batch, mk, mv, P, s)) != LOKI_OK) return e;
+                return launch_decode(cache, batch, mq, num_q_heads, P, r, k, k_per_seq, recent_window, group_reduce,
+                                     scale, out_mapped, nullptr, s, true);
+            }
+            // (an unaligned q falls through to the staged copies)
+        }
+    }
     char* dev = reinterpret_cast<char*>(staging);
     void* dk = dev + st.k_off;
     void* dv = dev + st.v_off;
@@ -614,7 +655,6 @@ loki_status loki_decode_step_host(const loki_cache* cache, const loki_batch* bat
     e = check_decode(cache, batch, dq, num_q_heads, P, r, k, recent_window, group_reduce, scale, dout);
     if (e != LOKI_OK) return e;
     if ((e = check_decode_fits(cache, batch, num_q_heads, r)) != LOKI_OK) return e;
-    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     clear_pending_error();
     if (cudaMemcpyAsync(dk, k_new_host, st.k_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
         cudaMemcpyAsync(dv, v_new_host, st.k_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||

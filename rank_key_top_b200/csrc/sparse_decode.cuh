@@ -290,10 +290,15 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
 #pragma unroll
         for (int i = 0; i < RPG; ++i) pv[i] = *reinterpret_cast<const float4*>(Ph + (rg * RPG + i) * D + 4 * cq);
     }
+    // the group's queries, G x D elements: 16-byte piece i read by thread i
+    // (whole 128-byte requests, which matters when q is read in place from
+    // host memory) and staged in the q_hat region until the first barrier
     const T* qg = reinterpret_cast<const T*>(p.q) + ((int64_t)b * Hq + h * G) * D;
+    constexpr int QP = G * D * (int)sizeof(T) / 16;
+    static_assert(QP <= kThreads && QP * 16 == G * D * (int)sizeof(T), "query pieces");
+    uint4 qpiece = make_uint4(0u, 0u, 0u, 0u);
+    if (tid < QP) qpiece = reinterpret_cast<const uint4*>(qg)[tid];
     typename Vec<T, RPG>::raw_t qraw[G];
-#pragma unroll
-    for (int j = 0; j < G; ++j) qraw[j] = Vec<T, RPG>::load(qg + j * D + rg * RPG);
     int L = p.seq_lens[b];
     if (L < 0 || L > p.max_seq_len) {
         if (tid == 0 && crank == 0) flag_error(LOKI_DEVERR_SEQ_LEN);
@@ -391,7 +396,12 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_decode_kernel(const Sparse
     for (int i = tid; i < 2 * kHistBins; i += kThreads) hist[i] = 0;
     if (j0 < nblk_loc) tbl[j0] = tb0;
     if (j1 < nblk_loc) tbl[j1] = tb1;
+    if (tid < QP) reinterpret_cast<uint4*>(qhat)[tid] = qpiece;
     __syncthreads();
+    // this thread's RPG rows of each query (q_hat overwrites the staging only
+    // after the next barrier)
+#pragma unroll
+    for (int j = 0; j < G; ++j) qraw[j] = Vec<T, RPG>::load(reinterpret_cast<const T*>(qhat) + j * D + rg * RPG);
 
     {   // q_hat = q P[h]: each thread sums its RPG rows for its 4 columns
         float qv[G][RPG];

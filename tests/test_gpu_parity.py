@@ -879,6 +879,60 @@ def test_decode_step_host_equals_decode_step(cuda_lib, dtype, W):
     assert torch.equal(outs[0], outs[1])
 
 
+def test_decode_step_host_in_place_and_staged_paths_agree(cuda_lib):
+    """The host-buffer step's two paths give what loki_decode_step gives, bit
+    for bit: pinned buffers (read and written in place by the kernels, here
+    as views at an offset inside larger pinned tensors), pageable buffers
+    (staged copies), and pinned buffers with q 2 bytes off 16-byte alignment
+    (staged copies as well)."""
+    s = spec(num_q_heads=8, num_kv_heads=2, seq_lens=[1500, 2100], k=150, recent_window=8)
+    wl = synth.make_workload(s)
+    k_new, v_new = synth.draw_new_tokens(s, step=6)
+    lens = torch.tensor([n + 1 for n in s.seq_lens], dtype=torch.int32)
+    shape = (s.batch, s.num_q_heads, s.head_dim)
+
+    def pinned_view(t, shift):
+        flat = torch.zeros(t.numel() + 64, dtype=t.dtype).pin_memory()
+        v = flat[shift:shift + t.numel()].view(t.shape)
+        v.copy_(t)
+        return v
+
+    outs = {}
+    for mode in ("device", "in_place", "pageable", "unaligned_q"):
+        dev = harness.Device(wl, cuda_lib)
+        dev.batch = cuda_lib.Batch(wl.block_table.cuda(), lens.cuda(), int(lens.max()))
+        if mode == "device":
+            out = torch.full(shape, float("nan"), device="cuda")
+            cuda_lib.loki_decode_step(dev.cache, dev.batch, k_new.cuda(), v_new.cuda(), dev.q, dev.P, s.r, s.k, out,
+                                      recent_window=8)
+            torch.cuda.synchronize()
+            outs[mode] = out.cpu()
+            continue
+        if mode == "in_place":
+            hk, hv, hq = pinned_view(k_new, 8), pinned_view(v_new, 24), pinned_view(wl.q, 16)
+            hout = pinned_view(torch.full(shape, float("nan")), 4)
+        elif mode == "pageable":
+            hk, hv, hq = k_new.clone(), v_new.clone(), wl.q.clone()
+            hout = torch.full(shape, float("nan"))
+        else:
+            hk, hv = k_new.pin_memory(), v_new.pin_memory()
+            hq = pinned_view(wl.q, 1)   # 2 bytes past a 16-byte boundary (bf16)
+            assert hq.data_ptr() % 16 == 2
+            hout = torch.full(shape, float("nan")).pin_memory()
+        staging = torch.full((cuda_lib.loki_decode_step_host_bytes(dev.cache, dev.batch, s.num_q_heads),), 0xAB,
+                             dtype=torch.uint8, device="cuda")
+        cuda_lib.loki_decode_step_host(dev.cache, dev.batch, hk, hv, hq, dev.P, s.r, s.k, hout, staging,
+                                       recent_window=8)
+        torch.cuda.synchronize()
+        outs[mode] = hout.clone()
+        # the in-place path leaves the staging buffer alone; the copies go through it
+        assert bool((staging == 0xAB).all()) == (mode == "in_place"), mode
+    assert cuda_lib.loki_device_error(clear=True) == 0
+    assert not torch.isnan(outs["device"]).any()
+    for mode in ("in_place", "pageable", "unaligned_q"):
+        assert torch.equal(outs[mode], outs["device"]), mode
+
+
 def test_decode_step_host_in_a_cuda_graph(cuda_lib):
     """The host-buffer step captured once into a CUDA graph and replayed with
     new host inputs written in place gives what an eager call gives."""
