@@ -629,7 +629,9 @@ loki_status loki_decode_step_host(const loki_cache* cache, const loki_batch* bat
         void* mv = mapped_host_address(v_new_host);
         void* mq = mapped_host_address(q_host);
         void* mo = mapped_host_address(out_host);
-        if (mk && mv && mq && mo && (reinterpret_cast<uintptr_t>(mo) & 3u) == 0) {
+        const uintptr_t es = elem_size(cache->dtype);  // the append reads single elements
+        if (mk && mv && mq && mo && reinterpret_cast<uintptr_t>(mk) % es == 0 &&
+            reinterpret_cast<uintptr_t>(mv) % es == 0 && (reinterpret_cast<uintptr_t>(mo) & 3u) == 0) {
             float* out_mapped = reinterpret_cast<float*>(mo);
             loki_status e = check_append(cache, batch, mk, mv, P);
             if (e == LOKI_OK) e = check_decode(cache, batch, mq, num_q_heads, P, r, k, recent_window, group_reduce,
@@ -641,7 +643,8 @@ loki_status loki_decode_step_host(const loki_cache* cache, const loki_batch* bat
                 return launch_decode(cache, batch, mq, num_q_heads, P, r, k, k_per_seq, recent_window, group_reduce,
                                      scale, out_mapped, nullptr, s, true);
             }
-            // (an unaligned q falls through to the staged copies)
+            // (an unaligned q falls through to the staged copies, as do
+            // inputs off their element alignment and an unaligned out)
         }
     }
     char* dev = reinterpret_cast<char*>(staging);
